@@ -1,0 +1,58 @@
+"""Workload shapes of the routed-branch forward (sizes only, no arithmetic).
+
+Each entry names a layer by what it is.  L tokens of width d, an N_r x N_c grid
+of atomic experts (N = N_r * N_c), K experts per token, groups of B experts.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, asdict
+
+
+@dataclass(frozen=True)
+class LayerConfig:
+    name: str
+    L: int
+    d: int
+    N_r: int
+    N_c: int
+    K: int
+    B: int
+    zipf: bool = False          # additive Zipf(s=1.1) log-bias on router rows/columns
+
+    @property
+    def N(self) -> int:
+        return self.N_r * self.N_c
+
+    @property
+    def G(self) -> int:
+        return (self.N + self.B - 1) // self.B
+
+    @property
+    def M(self) -> int:
+        return self.L * self.K
+
+    def with_L(self, L: int) -> "LayerConfig":
+        return LayerConfig(f"{self.name.split('_L')[0]}_L{L}", L, self.d, self.N_r, self.N_c,
+                           self.K, self.B, self.zipf)
+
+    def asdict(self) -> dict:
+        out = asdict(self)
+        out["N"] = self.N
+        return out
+
+
+TINY = LayerConfig("tiny_L256_d256_N4096_K16_B32", 256, 256, 64, 64, 16, 32)
+SMALL = LayerConfig("small_L4096_d768_N262144_K64_B64", 4096, 768, 512, 512, 64, 64)
+HEADLINE = LayerConfig("headline_L4096_d1024_N1700416_K64_B128", 4096, 1024, 1304, 1304, 64, 128)
+SKEW = LayerConfig("skew_L16384_d2048_N1048576_K128_B128_zipf", 16384, 2048, 1024, 1024, 128, 128,
+                   zipf=True)
+SWEEP_BASE = LayerConfig("sweep_d2048_N1700416_K64_B128", 4096, 2048, 1304, 1304, 64, 128)
+SWEEP_L = (1, 16, 256, 4096, 65536)
+
+
+def sweep(L: int) -> LayerConfig:
+    return LayerConfig(f"sweep_L{L}_d2048_N1700416_K64_B128", L, 2048, 1304, 1304, 64, 128)
+
+
+ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L]
+BY_NAME = {c.name: c for c in ALL}

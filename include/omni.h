@@ -1,0 +1,195 @@
+/*
+ * omni.h -- C ABI of the B200 (sm_100a) routed-branch forward of an OmniMoE
+ * layer.  Library: atomic_expert_layer_b200/libomni.so.
+ *
+ * Sources, cited by page title and section:
+ *   [R] "OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at Scale",
+ *       review at paper.rainbus.top, method paragraph (steps 1-3: atomic
+ *       experts and Dynamic Expert Assembly; Cartesian product router;
+ *       expert-centric scheduling with grouped GEMM).
+ *   [G] same title, gist.science summary, section 2.1 (atomic experts, DEA,
+ *       shared MLP) and section 2.2 (Cartesian product router; expert-centric
+ *       scheduling: task collection, grouping by contiguous expert-id ranges,
+ *       token order inside a group, grouped GEMM).
+ *
+ * Notation follows [R]: L tokens of width d; N = N_r * N_c atomic experts,
+ * expert n sits at grid cell (i, j) with n = i * N_c + j; W and V hold the
+ * w_in and w_out vectors of all experts as rows (N x d); W_r, W_c are the
+ * router projections; K experts are selected per token; B experts form a
+ * group, expert e belongs to group q = e / B; G = ceil(N / B) groups;
+ * M = L * K tasks.
+ *
+ * Conventions shared by every entry point:
+ *   - All array arguments are DEVICE pointers to caller-owned, contiguous,
+ *     row-major buffers.  The library never allocates or frees device memory;
+ *     scratch comes from the caller's workspace `ws` of `ws_bytes` bytes, at
+ *     least omni_workspace_size(...) for the same sizes, 256-byte aligned.
+ *     One workspace must not be used by two calls that overlap in time.
+ *   - bf16 values are passed as their 16-bit patterns (omni_bf16).
+ *   - W_r is stored as N_r rows of d (row i is the routing vector of grid row
+ *     i), i.e. the d x N_r matrix of [R] in column-major order; likewise W_c.
+ *     Then s_r = x W_r^T in this storage.
+ *   - Every call enqueues its work on `stream` (NULL = legacy default stream)
+ *     and returns without synchronising.  Pointers must stay valid until the
+ *     stream reaches the work.
+ *   - Return value: OMNI_OK, or a negative omni_status.  Argument problems are
+ *     found on the host before anything is enqueued.  OMNI_ERR_CUDA means a
+ *     launch failed.  Problems found on the device (an expert id out of range,
+ *     a bounded wait that ran out) are recorded in a status word inside `ws`;
+ *     read it with omni_get_device_status.  Each entry point clears that word
+ *     when it starts.  No function prints, throws or exits.
+ *   - bf16 pointers must be 16-byte aligned; d must be a multiple of 8.
+ */
+#ifndef OMNI_H_
+#define OMNI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                 /* = cudaStream_t */
+typedef struct CUstream_st *omni_stream_t;
+typedef uint16_t omni_bf16;         /* bf16 bit pattern */
+
+typedef enum {
+    OMNI_OK = 0,
+    OMNI_ERR_INVALID_ARG = -1,      /* null pointer, non-positive size, K > N, misaligned pointer */
+    OMNI_ERR_UNSUPPORTED = -2,      /* a size outside what the kernels handle (see each call)    */
+    OMNI_ERR_WORKSPACE = -3,        /* ws_bytes below omni_workspace_size(...)                    */
+    OMNI_ERR_CUDA = -4,             /* a CUDA launch or runtime call failed                      */
+    OMNI_ERR_DEVICE = -5            /* recorded on the device; see omni_get_device_status        */
+} omni_status;
+
+/* flags */
+#define OMNI_ROUTER_LOGPROBS_IN 1u  /* omni_router_topk: p_r, p_c are inputs (skip s = xW^T and LogSoftmax) */
+#define OMNI_Y_ACCUMULATE       2u  /* y += routed(x) instead of y = routed(x)                           */
+
+/* Device status codes written into the workspace status word. */
+#define OMNI_DEV_OK              0
+#define OMNI_DEV_BAD_EXPERT      1  /* an expert id outside [0, N) reached the schedule   */
+#define OMNI_DEV_WAIT_TIMEOUT    2  /* a bounded barrier wait ran out (no hang)           */
+#define OMNI_DEV_BAD_SCHEDULE    3  /* schedule arrays inconsistent (offsets/ids)          */
+
+/* Size limits of this build (OMNI_ERR_UNSUPPORTED beyond them). */
+#define OMNI_MAX_AXIS   8192        /* N_r, N_c                                   */
+#define OMNI_MAX_K      512         /* K                                          */
+#define OMNI_MAX_B      1024        /* B                                          */
+#define OMNI_MAX_D      2048        /* d for the expert stage; d % 256 == 0 there */
+
+/* Library version, for the binding's sanity check. */
+int omni_version(void);
+
+/* Human-readable name of an omni_status or a device status code (static string). */
+const char *omni_status_string(int status);
+const char *omni_device_status_string(int dev_status);
+
+/*
+ * Bytes of workspace that every entry point needs for these sizes (the same
+ * layout serves all four calls).  Returns 0 if the sizes are invalid.
+ */
+size_t omni_workspace_size(int L, int d, int N_r, int N_c, int K, int B);
+
+/*
+ * Cartesian product router, [R] step 2 and [G] section 2.2.
+ *   s_r = x W_r^T, s_c = x W_c^T            (bf16 inputs, fp32 accumulation)
+ *   p_r = LogSoftmax(s_r), p_c = LogSoftmax(s_c)   (fp32, per token)
+ *   S_ij = p_r[i] + p_c[j]  (one fp32 addition; the N-entry grid is never built)
+ * and the exact global top-K of S per token, ordered by the key
+ *   (S desc, p_r[i] desc, p_c[j] desc, n asc),
+ * with gates g = softmax of the K selected S (the pages leave g_x open; this
+ * is the reading taken).
+ *   x    [L, d]   bf16          W_r [N_r, d] bf16      W_c [N_c, d] bf16
+ *   p_r  [L, N_r] fp32  output, or input with OMNI_ROUTER_LOGPROBS_IN
+ *   p_c  [L, N_c] fp32  output, or input with OMNI_ROUTER_LOGPROBS_IN
+ *   idx  [L, K]   int32 output, n = i * N_c + j, in key order
+ *   score[L, K]   fp32  output, S of each selected cell
+ *   gate [L, K]   fp32  output, softmax over the token's K scores
+ * With OMNI_ROUTER_LOGPROBS_IN, x / W_r / W_c / d are not read (may be NULL / 0).
+ * Row and column candidates are the top min(K, N_r) rows and min(K, N_c)
+ * columns.  Limits: K <= N_r * N_c, K <= OMNI_MAX_K, N_r, N_c <= OMNI_MAX_AXIS.
+ * p must be finite (NaN / Inf give an unspecified but in-range selection).
+ */
+int omni_router_topk(const omni_bf16 *x, const omni_bf16 *W_r, const omni_bf16 *W_c,
+                     int L, int d, int N_r, int N_c, int K,
+                     float *p_r, float *p_c, int32_t *idx, float *score, float *gate,
+                     unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
+
+/*
+ * Expert-centric scheduling, [R] step 3 and [G] section 2.2.
+ * Task m = t * K + k is (token t, expert e = idx[t, k], gate[t, k]).  Tasks are
+ * sorted by (q = e / B, t, e) -- group id, then token id, then expert id (the
+ * pages fix the first two keys; the third makes the order unique) -- and the
+ * groups are bucketed:
+ *   task_token, task_expert [M] int32, task_gate [M] fp32   sorted tasks
+ *   group_offsets [G + 1] int32   exclusive prefix sum of group_counts
+ *   group_counts  [G]     int32   tasks per group
+ *   active_groups [G]     int32   groups with >= 1 task, ascending; entries
+ *                                 past num_active are left unspecified
+ *   num_active    [1]     int32   number of active groups
+ *   num_distinct  [1]     int32   number of distinct experts among the tasks
+ * idx [L, K] int32 and gate [L, K] fp32 are inputs (e.g. from omni_router_topk);
+ * expert ids must lie in [0, N) and be distinct within a token (an id out of
+ * range sets OMNI_DEV_BAD_EXPERT and that task is dropped from the counts).
+ * Limits: M <= 2^31 - 1, B <= OMNI_MAX_B, K <= OMNI_MAX_K.
+ * The output is bit-identical from run to run (the sort key is unique).
+ */
+int omni_schedule(const int32_t *idx, const float *gate, int L, int K, int N, int B,
+                  int32_t *task_token, int32_t *task_expert, float *task_gate,
+                  int32_t *group_offsets, int32_t *group_counts, int32_t *active_groups,
+                  int32_t *num_active, int32_t *num_distinct,
+                  void *ws, size_t ws_bytes, omni_stream_t stream);
+
+/*
+ * Grouped expert computation, [R] steps 1 and 3 and [G] section 2.2
+ * ("grouped GEMM"): for every active group q with tokens X_q, expert rows
+ * W_q, V_q and gate matrix G_q (gate of task (t, e), 0 where there is none),
+ *   O_q = (G_q . SiLU(X_q W_q^T)) V_q,      y[t] += O_q[t]  for its tokens.
+ * sigma is read as SiLU (one w_in per expert leaves SwiGLU without a gate).
+ * Only the (token, expert) pairs that are tasks are computed: the zero
+ * entries of G_q are skipped, not multiplied.
+ *   x [L, d] bf16, W [N, d] bf16, V [N, d] bf16
+ *   schedule arrays as produced by omni_schedule for the same L, K, N, B
+ *   y [L, d] fp32  output (overwritten, or accumulated with OMNI_Y_ACCUMULATE)
+ * Summation order inside y is not fixed (fp32 atomic adds), so y may differ
+ * in the last bits between runs.  Limits: d % 256 == 0, d <= OMNI_MAX_D,
+ * B <= OMNI_MAX_B.
+ */
+int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
+                            int L, int d, int K, int N, int B,
+                            const int32_t *task_token, const int32_t *task_expert,
+                            const float *task_gate, const int32_t *group_offsets,
+                            const int32_t *active_groups, const int32_t *num_active,
+                            float *y, unsigned flags, void *ws, size_t ws_bytes,
+                            omni_stream_t stream);
+
+/*
+ * The whole routed branch: omni_router_topk, omni_schedule and
+ * omni_grouped_expert_fwd back to back on `stream`, with every intermediate in
+ * `ws` and no host synchronisation:  y = routed(x)  (the shared dense MLP of
+ * [G] section 2.1 is not part of it).
+ *   x [L, d], W [N, d], V [N, d], W_r [N_r, d], W_c [N_c, d]  bf16
+ *   y [L, d] fp32 output;  idx_out [L, K] int32, gate_out [L, K] fp32 are
+ *   optional copies of the routing (NULL to skip).
+ * Limits: those of the three calls above.
+ */
+int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
+                    const omni_bf16 *W_r, const omni_bf16 *W_c,
+                    int L, int d, int N_r, int N_c, int K, int B,
+                    float *y, int32_t *idx_out, float *gate_out,
+                    unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
+
+/*
+ * Synchronises `stream`, copies the status word of `ws` into *status_out
+ * (an OMNI_DEV_* code) and clears it.  For tests and error handling; it is
+ * the only call that blocks the host.
+ */
+int omni_get_device_status(void *ws, size_t ws_bytes, omni_stream_t stream, int *status_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OMNI_H_ */
