@@ -1,0 +1,94 @@
+"""B200 (sm_100a) routed-branch forward of an OmniMoE layer.
+
+The computation lives in libomni.so (hand-written CUDA, C ABI in
+include/omni.h).  This package only loads it and marshals torch tensors:
+  - ``omni_*`` functions mirror the C entry points argument for argument;
+  - ``router_topk``, ``schedule``, ``grouped_expert_fwd``, ``routed_fwd``
+    allocate the output tensors and a workspace, then call them.
+"""
+from __future__ import annotations
+
+import torch
+
+from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_Y_ACCUMULATE, OmniError, load,  # noqa: F401
+                   expert_workspace, omni_expert_workspace_size, omni_get_device_status,
+                   omni_grouped_expert_fwd, omni_routed_fwd, omni_router_topk,
+                   omni_router_workspace_size, omni_schedule, omni_schedule_workspace_size,
+                   omni_selftest_wait_timeout,
+                   omni_workspace_size, router_workspace, schedule_workspace, workspace)
+
+__all__ = [
+    "load", "OmniError", "OMNI_ROUTER_LOGPROBS_IN", "OMNI_Y_ACCUMULATE",
+    "omni_workspace_size", "omni_router_topk", "omni_schedule", "omni_grouped_expert_fwd",
+    "omni_routed_fwd", "omni_get_device_status", "workspace",
+    "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd",
+]
+
+
+def router_topk(x, W_r, W_c, K, ws=None, p_r=None, p_c=None, logprobs_in=False, stream=None):
+    """Top-K experts per token.  With logprobs_in, p_r / p_c are inputs and
+    x may be None (then pass W_r / W_c as None too)."""
+    if logprobs_in:
+        L, N_r = p_r.shape
+        N_c = p_c.shape[1]
+        d = 0
+        dev = p_r.device
+    else:
+        L, d = x.shape
+        N_r, N_c = W_r.shape[0], W_c.shape[0]
+        dev = x.device
+        p_r = torch.empty((L, N_r), dtype=torch.float32, device=dev) if p_r is None else p_r
+        p_c = torch.empty((L, N_c), dtype=torch.float32, device=dev) if p_c is None else p_c
+    idx = torch.empty((L, K), dtype=torch.int32, device=dev)
+    score = torch.empty((L, K), dtype=torch.float32, device=dev)
+    gate = torch.empty((L, K), dtype=torch.float32, device=dev)
+    ws = router_workspace(L, N_r, N_c, K, dev) if ws is None else ws
+    omni_router_topk(x, W_r, W_c, L, d, N_r, N_c, K, p_r, p_c, idx, score, gate,
+                     OMNI_ROUTER_LOGPROBS_IN if logprobs_in else 0, ws, stream)
+    return dict(p_r=p_r, p_c=p_c, idx=idx, score=score, gate=gate)
+
+
+def schedule(idx, gate, N, B, ws=None, stream=None):
+    L, K = idx.shape
+    dev = idx.device
+    M, G = L * K, (N + B - 1) // B
+    out = dict(task_token=torch.empty(M, dtype=torch.int32, device=dev),
+               task_expert=torch.empty(M, dtype=torch.int32, device=dev),
+               task_gate=torch.empty(M, dtype=torch.float32, device=dev),
+               group_offsets=torch.empty(G + 1, dtype=torch.int32, device=dev),
+               group_counts=torch.empty(G, dtype=torch.int32, device=dev),
+               active_groups=torch.empty(G, dtype=torch.int32, device=dev),
+               num_active=torch.empty(1, dtype=torch.int32, device=dev),
+               num_distinct=torch.empty(1, dtype=torch.int32, device=dev))
+    ws = schedule_workspace(L, K, N, B, dev) if ws is None else ws
+    omni_schedule(idx, gate, L, K, N, B, out["task_token"], out["task_expert"], out["task_gate"],
+                  out["group_offsets"], out["group_counts"], out["active_groups"],
+                  out["num_active"], out["num_distinct"], ws, stream)
+    return out
+
+
+def grouped_expert_fwd(x, W, V, sched, K, B, y=None, accumulate=False, ws=None, stream=None):
+    L, d = x.shape
+    N = W.shape[0]
+    y = torch.empty((L, d), dtype=torch.float32, device=x.device) if y is None else y
+    ws = expert_workspace(L, d, K, N, B, x.device) if ws is None else ws
+    omni_grouped_expert_fwd(x, W, V, L, d, K, N, B, sched["task_token"], sched["task_expert"],
+                            sched["task_gate"], sched["group_offsets"], sched["active_groups"],
+                            sched["num_active"], y, OMNI_Y_ACCUMULATE if accumulate else 0, ws,
+                            stream)
+    return y
+
+
+def routed_fwd(x, W, V, W_r, W_c, K, B, y=None, ws=None, want_routing=False, accumulate=False,
+               stream=None):
+    L, d = x.shape
+    N_r, N_c = W_r.shape[0], W_c.shape[0]
+    y = torch.empty((L, d), dtype=torch.float32, device=x.device) if y is None else y
+    ws = workspace(L, d, N_r, N_c, K, B, x.device) if ws is None else ws
+    idx = gate = None
+    if want_routing:
+        idx = torch.empty((L, K), dtype=torch.int32, device=x.device)
+        gate = torch.empty((L, K), dtype=torch.float32, device=x.device)
+    omni_routed_fwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, B, y, idx, gate,
+                    OMNI_Y_ACCUMULATE if accumulate else 0, ws, stream)
+    return (y, idx, gate) if want_routing else y

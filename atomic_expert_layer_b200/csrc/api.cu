@@ -1,0 +1,338 @@
+// api.cu -- the C ABI of libomni (declared in include/omni.h): argument
+// checks, workspace layout and the order of kernel launches.  No allocation,
+// no host synchronisation except in omni_get_device_status.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstring>
+
+#include "omni_common.cuh"
+#include "omni_internal.h"
+
+namespace omni {
+
+namespace {
+constexpr int kVersion = 1;
+
+inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+}  // namespace
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+bool make_sizes(int L, int d, int N_r, int N_c, int K, int B, Sizes *sz) {
+    if (L <= 0 || d <= 0 || N_r <= 0 || N_c <= 0 || K <= 0 || B <= 0) return false;
+    sz->L = L; sz->d = d; sz->N_r = N_r; sz->N_c = N_c; sz->K = K; sz->B = B;
+    sz->N = (int64_t)N_r * N_c;
+    sz->M = (int64_t)L * K;
+    sz->G = (sz->N + B - 1) / B;
+    sz->Kr = K < N_r ? K : N_r;
+    sz->Kc = K < N_c ? K : N_c;
+    sz->C = merge_candidates(K, sz->Kr, sz->Kc);
+    sz->ntiles = (sz->M + kSortTile - 1) / kSortTile;
+    const int64_t gm = sz->G < sz->M ? sz->G : sz->M;
+    sz->max_items = gm + (sz->M + kItemTasks - 1) / kItemTasks;
+    return true;
+}
+
+WsLayout make_layout(const Sizes &sz, unsigned regions) {
+    WsLayout w;
+    std::memset(&w, 0, sizeof w);
+    size_t o = 0;
+    auto take = [&](size_t bytes) { const size_t at = o; o = align256(o + bytes); return at; };
+    const size_t L = (size_t)sz.L, M = (size_t)sz.M, G = (size_t)sz.G;
+    w.hdr = take(sizeof(WsHeader));
+    if (regions & kRegRouter) {
+        w.s_r = take(4 * L * sz.N_r);
+        w.s_c = take(4 * L * sz.N_c);
+        w.row_val = take(4 * L * sz.Kr);
+        w.row_idx = take(4 * L * sz.Kr);
+        w.col_val = take(4 * L * sz.Kc);
+        w.col_idx = take(4 * L * sz.Kc);
+        w.idx = take(4 * L * sz.K);
+        w.score = take(4 * L * sz.K);
+        w.gate = take(4 * L * sz.K);
+    }
+    if (regions & kRegSched) {
+        w.a_tok = take(4 * M); w.a_exp = take(4 * M); w.a_gate = take(4 * M);
+        w.b_tok = take(4 * M); w.b_exp = take(4 * M); w.b_gate = take(4 * M);
+        w.bitmap = take(4 * (size_t)((sz.N + 31) / 32));
+        w.hist = take(4 * 256 * (size_t)sz.ntiles);
+    }
+    if (regions & kRegSchedOut) {
+        w.t_tok = take(4 * M); w.t_exp = take(4 * M); w.t_gate = take(4 * M);
+        w.g_off = take(4 * (G + 1));
+        w.g_cnt = take(4 * G);
+        w.g_act = take(4 * G);
+        w.n_act = take(4);
+        w.n_dist = take(4);
+    }
+    if (regions & kRegExpert) w.items = take(16 * (size_t)sz.max_items);
+    w.total = o;
+    return w;
+}
+
+namespace {
+// One CTA waits on a barrier that never completes; the bounded wait gives up.
+__global__ void selftest_wait_kernel(int *status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_limit(&bar, 0u, status, limit_ns);
+}
+}  // namespace
+
+}  // namespace omni
+
+using namespace omni;
+
+namespace {
+
+int check_common(int L, int d, int N_r, int N_c, int K, int B, bool router, Sizes *sz) {
+    if (!make_sizes(L, d, N_r, N_c, K, B, sz)) return OMNI_ERR_INVALID_ARG;
+    if ((int64_t)K > sz->N) return OMNI_ERR_INVALID_ARG;
+    if (sz->M > INT_MAX || sz->N > INT_MAX) return OMNI_ERR_UNSUPPORTED;
+    if (K > OMNI_MAX_K || B > OMNI_MAX_B) return OMNI_ERR_UNSUPPORTED;
+    if (router && (N_r > OMNI_MAX_AXIS || N_c > OMNI_MAX_AXIS)) return OMNI_ERR_UNSUPPORTED;
+    return OMNI_OK;
+}
+
+int check_ws(const Sizes &sz, unsigned regions, void *ws, size_t ws_bytes, WsLayout *lay) {
+    if (!ws) return OMNI_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return OMNI_ERR_INVALID_ARG;
+    *lay = make_layout(sz, regions);
+    if (ws_bytes < lay->total) return OMNI_ERR_WORKSPACE;
+    return OMNI_OK;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? OMNI_OK : OMNI_ERR_CUDA; }
+
+int reset_header(void *ws, cudaStream_t st) {
+    return cuda_rc(cudaMemsetAsync(ws, 0, sizeof(WsHeader), st));
+}
+
+int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c,
+                     const Sizes &sz, float *p_r, float *p_c, int32_t *idx, float *score,
+                     float *gate, unsigned flags, void *ws, const WsLayout &lay,
+                     cudaStream_t st) {
+    int *status = ws_at<int>(ws, lay.hdr);
+    float *row_val = ws_at<float>(ws, lay.row_val), *col_val = ws_at<float>(ws, lay.col_val);
+    int *row_idx = ws_at<int>(ws, lay.row_idx), *col_idx = ws_at<int>(ws, lay.col_idx);
+    cudaError_t e;
+    if (flags & OMNI_ROUTER_LOGPROBS_IN) {
+        e = launch_axis_topk(p_r, p_c, false, nullptr, nullptr, sz.L, sz.N_r, sz.N_c, sz.K,
+                             row_val, row_idx, col_val, col_idx, status, st);
+    } else {
+        float *s_r = ws_at<float>(ws, lay.s_r), *s_c = ws_at<float>(ws, lay.s_c);
+        e = launch_router_gemm(x, W_r, W_c, sz.L, sz.d, sz.N_r, sz.N_c, s_r, s_c, status, st);
+        if (e != cudaSuccess) return OMNI_ERR_CUDA;
+        e = launch_axis_topk(s_r, s_c, true, p_r, p_c, sz.L, sz.N_r, sz.N_c, sz.K, row_val,
+                             row_idx, col_val, col_idx, status, st);
+    }
+    if (e != cudaSuccess) return OMNI_ERR_CUDA;
+    e = launch_merge_topk(row_val, row_idx, col_val, col_idx, sz.L, sz.N_c, sz.K, sz.Kr, sz.Kc,
+                          sz.C, idx, score, gate, st);
+    return cuda_rc(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int omni_version(void) { return kVersion; }
+
+const char *omni_status_string(int s) {
+    switch (s) {
+        case OMNI_OK: return "OMNI_OK";
+        case OMNI_ERR_INVALID_ARG: return "OMNI_ERR_INVALID_ARG";
+        case OMNI_ERR_UNSUPPORTED: return "OMNI_ERR_UNSUPPORTED";
+        case OMNI_ERR_WORKSPACE: return "OMNI_ERR_WORKSPACE";
+        case OMNI_ERR_CUDA: return "OMNI_ERR_CUDA";
+        case OMNI_ERR_DEVICE: return "OMNI_ERR_DEVICE";
+        default: return "unknown omni_status";
+    }
+}
+
+const char *omni_device_status_string(int s) {
+    switch (s) {
+        case OMNI_DEV_OK: return "OMNI_DEV_OK";
+        case OMNI_DEV_BAD_EXPERT: return "OMNI_DEV_BAD_EXPERT";
+        case OMNI_DEV_WAIT_TIMEOUT: return "OMNI_DEV_WAIT_TIMEOUT";
+        case OMNI_DEV_BAD_SCHEDULE: return "OMNI_DEV_BAD_SCHEDULE";
+        default: return "unknown device status";
+    }
+}
+
+size_t omni_workspace_size(int L, int d, int N_r, int N_c, int K, int B) {
+    Sizes sz;
+    if (check_common(L, d, N_r, N_c, K, B, true, &sz) != OMNI_OK) return 0;
+    return make_layout(sz, kRegAll).total;
+}
+
+size_t omni_router_workspace_size(int L, int N_r, int N_c, int K) {
+    Sizes sz;
+    if (check_common(L, 8, N_r, N_c, K, 1, true, &sz) != OMNI_OK) return 0;
+    return make_layout(sz, kRegRouter).total;
+}
+
+size_t omni_schedule_workspace_size(int L, int K, int N, int B) {
+    Sizes sz;
+    if (N <= 0 || check_common(L, 8, N, 1, K, B, false, &sz) != OMNI_OK) return 0;
+    return make_layout(sz, kRegSched).total;
+}
+
+size_t omni_expert_workspace_size(int L, int d, int K, int N, int B) {
+    Sizes sz;
+    if (N <= 0 || check_common(L, d, N, 1, K, B, false, &sz) != OMNI_OK) return 0;
+    return make_layout(sz, kRegExpert).total;
+}
+
+int omni_router_topk(const omni_bf16 *x, const omni_bf16 *W_r, const omni_bf16 *W_c, int L,
+                     int d, int N_r, int N_c, int K, float *p_r, float *p_c, int32_t *idx,
+                     float *score, float *gate, unsigned flags, void *ws, size_t ws_bytes,
+                     omni_stream_t stream) {
+    const bool lp_in = (flags & OMNI_ROUTER_LOGPROBS_IN) != 0;
+    Sizes sz;
+    int rc = check_common(L, lp_in ? 8 : d, N_r, N_c, K, 1, true, &sz);
+    if (rc) return rc;
+    if (!p_r || !p_c || !idx || !score || !gate) return OMNI_ERR_INVALID_ARG;
+    if (!lp_in) {
+        if (!x || !W_r || !W_c) return OMNI_ERR_INVALID_ARG;
+        if (d % 8 != 0) return OMNI_ERR_UNSUPPORTED;
+        if (!aligned16(x) || !aligned16(W_r) || !aligned16(W_c)) return OMNI_ERR_INVALID_ARG;
+    }
+    if (!aligned4(p_r) || !aligned4(p_c)) return OMNI_ERR_INVALID_ARG;
+    WsLayout lay;
+    if ((rc = check_ws(sz, kRegRouter, ws, ws_bytes, &lay))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = reset_header(ws, st))) return rc;
+    return router_topk_impl(x, W_r, W_c, sz, p_r, p_c, idx, score, gate, flags, ws, lay, st);
+}
+
+int omni_schedule(const int32_t *idx, const float *gate, int L, int K, int N, int B,
+                  int32_t *task_token, int32_t *task_expert, float *task_gate,
+                  int32_t *group_offsets, int32_t *group_counts, int32_t *active_groups,
+                  int32_t *num_active, int32_t *num_distinct, void *ws, size_t ws_bytes,
+                  omni_stream_t stream) {
+    if (N <= 0) return OMNI_ERR_INVALID_ARG;
+    Sizes sz;
+    int rc = check_common(L, 8, N, 1, K, B, false, &sz);   // an N x 1 grid gives the same N
+    if (rc) return rc;
+    if (!idx || !gate || !task_token || !task_expert || !task_gate || !group_offsets ||
+        !group_counts || !active_groups || !num_active || !num_distinct)
+        return OMNI_ERR_INVALID_ARG;
+    WsLayout lay;
+    if ((rc = check_ws(sz, kRegSched, ws, ws_bytes, &lay))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = reset_header(ws, st))) return rc;
+    return cuda_rc(launch_schedule(idx, gate, sz, task_token, task_expert, task_gate,
+                                   group_offsets, group_counts, active_groups, num_active,
+                                   num_distinct, ws, lay, st));
+}
+
+int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V, int L,
+                            int d, int K, int N, int B, const int32_t *task_token,
+                            const int32_t *task_expert, const float *task_gate,
+                            const int32_t *group_offsets, const int32_t *active_groups,
+                            const int32_t *num_active, float *y, unsigned flags, void *ws,
+                            size_t ws_bytes, omni_stream_t stream) {
+    if (N <= 0) return OMNI_ERR_INVALID_ARG;
+    Sizes sz;
+    int rc = check_common(L, d, N, 1, K, B, false, &sz);
+    if (rc) return rc;
+    if (!x || !W || !V || !task_token || !task_expert || !task_gate || !group_offsets ||
+        !active_groups || !num_active || !y)
+        return OMNI_ERR_INVALID_ARG;
+    if (d % 256 != 0 || d > OMNI_MAX_D) return OMNI_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(V) || !aligned16(y))
+        return OMNI_ERR_INVALID_ARG;
+    WsLayout lay;
+    if ((rc = check_ws(sz, kRegExpert, ws, ws_bytes, &lay))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = reset_header(ws, st))) return rc;
+    return cuda_rc(launch_grouped_expert(x, W, V, sz, task_token, task_expert, task_gate,
+                                         group_offsets, active_groups, num_active, y,
+                                         (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st));
+}
+
+int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
+                    const omni_bf16 *W_r, const omni_bf16 *W_c, int L, int d, int N_r, int N_c,
+                    int K, int B, float *y, int32_t *idx_out, float *gate_out, unsigned flags,
+                    void *ws, size_t ws_bytes, omni_stream_t stream) {
+    Sizes sz;
+    int rc = check_common(L, d, N_r, N_c, K, B, true, &sz);
+    if (rc) return rc;
+    if (!x || !W || !V || !W_r || !W_c || !y) return OMNI_ERR_INVALID_ARG;
+    if (d % 256 != 0 || d > OMNI_MAX_D) return OMNI_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(V) || !aligned16(W_r) || !aligned16(W_c) ||
+        !aligned16(y))
+        return OMNI_ERR_INVALID_ARG;
+    WsLayout lay;
+    if ((rc = check_ws(sz, kRegAll, ws, ws_bytes, &lay))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = reset_header(ws, st))) return rc;
+    int32_t *idx = ws_at<int32_t>(ws, lay.idx);
+    float *score = ws_at<float>(ws, lay.score), *gate = ws_at<float>(ws, lay.gate);
+    rc = router_topk_impl(x, W_r, W_c, sz, nullptr, nullptr, idx, score, gate,
+                          flags & ~OMNI_ROUTER_LOGPROBS_IN, ws, lay, st);
+    if (rc) return rc;
+    int32_t *tt = ws_at<int32_t>(ws, lay.t_tok), *te = ws_at<int32_t>(ws, lay.t_exp);
+    float *tg = ws_at<float>(ws, lay.t_gate);
+    int32_t *goff = ws_at<int32_t>(ws, lay.g_off), *gcnt = ws_at<int32_t>(ws, lay.g_cnt);
+    int32_t *gact = ws_at<int32_t>(ws, lay.g_act), *nact = ws_at<int32_t>(ws, lay.n_act);
+    int32_t *ndist = ws_at<int32_t>(ws, lay.n_dist);
+    if ((rc = cuda_rc(launch_schedule(idx, gate, sz, tt, te, tg, goff, gcnt, gact, nact, ndist,
+                                      ws, lay, st))))
+        return rc;
+    if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, tt, te, tg, goff, gact, nact, y,
+                                            (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st))))
+        return rc;
+    if (idx_out &&
+        (rc = cuda_rc(cudaMemcpyAsync(idx_out, idx, 4 * (size_t)sz.M, cudaMemcpyDeviceToDevice, st))))
+        return rc;
+    if (gate_out &&
+        (rc = cuda_rc(cudaMemcpyAsync(gate_out, gate, 4 * (size_t)sz.M, cudaMemcpyDeviceToDevice, st))))
+        return rc;
+    return OMNI_OK;
+}
+
+int omni_selftest_wait_timeout(void *ws, size_t ws_bytes, int limit_ms, omni_stream_t stream) {
+    if (!ws || ws_bytes < sizeof(WsHeader) || limit_ms < 1 || limit_ms > 10000)
+        return OMNI_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return OMNI_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int rc = reset_header(ws, st);
+    if (rc) return rc;
+    selftest_wait_kernel<<<1, 32, 0, st>>>(ws_at<int>(ws, 0), (uint64_t)limit_ms * 1000000ull);
+    return cuda_rc(cudaGetLastError());
+}
+
+int omni_get_device_status(void *ws, size_t ws_bytes, omni_stream_t stream, int *status_out) {
+    if (!ws || !status_out || ws_bytes < sizeof(WsHeader)) return OMNI_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int host = 0;
+    if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return OMNI_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return OMNI_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return OMNI_ERR_CUDA;
+    *status_out = host;
+    return host == 0 ? OMNI_OK : OMNI_ERR_DEVICE;
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// omni_internal.h -- launchers shared between the .cu files of libomni and the
+// workspace layout.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace omni {
+
+constexpr int kSortTile = 2048;        // tasks per radix-sort tile
+constexpr int kItemTasks = 256;        // max tasks per grouped-expert work item
+
+struct Sizes {
+    int L, d, N_r, N_c, K, B;
+    int64_t N, M, G;
+    int Kr, Kc;          // row / column candidates: min(K, N_r), min(K, N_c)
+    int C;               // merge candidates: cells (a, b) with (a+1)(b+1) <= K
+    int64_t ntiles;      // radix tiles
+    int64_t max_items;   // grouped-expert work items, upper bound
+};
+
+struct WsLayout {
+    size_t hdr, s_r, s_c, row_val, row_idx, col_val, col_idx, idx, score, gate;
+    size_t a_tok, a_exp, a_gate, b_tok, b_exp, b_gate, t_tok, t_exp, t_gate;
+    size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, items;
+    size_t total;
+};
+
+// Workspace regions.  Every call puts the 256-byte header at offset 0 and then
+// only the regions it uses, in this order; the whole routed forward uses all
+// of them, so omni_workspace_size (the full layout) covers every call.
+enum WsRegion : unsigned {
+    kRegRouter = 1u,      // s_r, s_c, axis candidates, idx / score / gate
+    kRegSched = 2u,       // sort buffers, expert bitmap, radix histograms
+    kRegSchedOut = 4u,    // sorted tasks and group arrays (routed forward only)
+    kRegExpert = 8u,      // work items
+    kRegAll = 15u
+};
+
+bool make_sizes(int L, int d, int N_r, int N_c, int K, int B, Sizes *sz);
+WsLayout make_layout(const Sizes &sz, unsigned regions);
+int merge_candidates(int K, int Kr, int Kc);
+
+template <typename T>
+inline T *ws_at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+// ---- router GEMM (tcgen05): s_r = x W_r^T, s_c = x W_c^T (fp32)
+cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c,
+                               int L, int d, int N_r, int N_c, float *s_r, float *s_c,
+                               int *status, cudaStream_t st);
+
+// ---- per-axis LogSoftmax (optional) + top-K; then grid merge + gates
+cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftmax,
+                             float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
+                             float *row_val, int *row_idx, float *col_val, int *col_idx,
+                             int *status, cudaStream_t st);
+cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
+                              const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
+                              int32_t *idx, float *score, float *gate, cudaStream_t st);
+
+// ---- schedule
+cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &sz,
+                            int32_t *task_token, int32_t *task_expert, float *task_gate,
+                            int32_t *group_offsets, int32_t *group_counts,
+                            int32_t *active_groups, int32_t *num_active, int32_t *num_distinct,
+                            void *ws, const WsLayout &lay, cudaStream_t st);
+
+// ---- grouped expert stage
+cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const uint16_t *V,
+                                  const Sizes &sz, const int32_t *task_token,
+                                  const int32_t *task_expert, const float *task_gate,
+                                  const int32_t *group_offsets, const int32_t *active_groups,
+                                  const int32_t *num_active, float *y, bool accumulate,
+                                  void *ws, const WsLayout &lay, cudaStream_t st);
+
+int device_sm_count();
+
+}  // namespace omni

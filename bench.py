@@ -1,0 +1,439 @@
+#!/usr/bin/env python3
+"""Benchmark of the routed-branch forward of an OmniMoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl omni|reference]
+
+One step = one pass of the whole routed branch (router GEMM, LogSoftmax,
+row/column top-K, grid merge + gates, expert-centric schedule, grouped
+expert stage) over one batch of L synthetic tokens, through the C ABI
+(omni_routed_fwd).  Inputs are resident in HBM when timing starts; L2 is
+flushed (256 MB write) between timed steps, outside the timed events.
+
+With N > 1 (launched by torchrun) every rank holds a replica of the weights
+and routes its own L tokens: the layer shards by token batch with no
+data-path collective (weak scaling); only the timing is reduced (max).
+
+Prints ONE JSON line on rank 0.  ``--impl reference`` times the CPU oracle
+(the plain C implementation under oracle/) on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from atomic_expert_layer_b200 import configs, inputs  # noqa: E402
+
+METRIC = "routed-layer tokens/s at L=4096, N≈1.7M (1×B200); % of HBM/tensor roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    """Max over ranks (timing only)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=FALLBACK_BF16_TFLOPS,
+                bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def radix_passes(G: int) -> int:
+    bits = 0
+    while bits < 31 and (1 << bits) < G:
+        bits += 1
+    return (bits + 7) // 8
+
+
+def launches_per_step(cfg) -> int:
+    # router GEMM, axis top-K, merge, schedule prepare, group scan,
+    # 3 per radix pass, build items, grouped expert kernel
+    return 3 + 2 + 3 * radix_passes(cfg.G) + 2
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [c.strip() for c in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        smax = max(float(r[2]) for r in rows)
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        # samples under load: power well above idle
+        load_idx = [i for i, r in enumerate(rows) if power and float(r[3]) > 0.5 * max(power)]
+        sm_load = [sm[i] for i in load_idx] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm_load)), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "samples_under_load": len(load_idx)}
+
+
+def traffic_from_profile(kernel_src: str) -> float | None:
+    """DRAM bytes per launch of the grouped expert kernel from the committed
+    ncu summary, if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get("grouped_expert_kernel")
+    if not d:
+        return None
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    if d.get("source_sha256") != sha:
+        return None
+    return float(d["dram_bytes_per_launch_full_size"])
+
+
+# ------------------------------------------------------------ omni arm
+def run_omni(args, cfg, world, rank, local):
+    import atomic_expert_layer_b200 as omni
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    omni.load()
+    t = inputs.make_inputs(cfg, dev, seed=0)
+    if world > 1:                                   # each rank routes its own tokens
+        t["x"] = inputs.make_inputs(cfg, dev, seed=1000 + rank, with_experts=False)["x"]
+    L, d = cfg.L, cfg.d
+    ws = omni.workspace(L, d, cfg.N_r, cfg.N_c, cfg.K, cfg.B, dev)
+    y = torch.empty((L, d), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        omni.omni_routed_fwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r, cfg.N_c,
+                             cfg.K, cfg.B, y, None, None, 0, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if omni.omni_get_device_status(ws) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # ---- timed region: K steps of omni_routed_fwd
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()                            # L2 flush, outside the events
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    clocks = clk.summary()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    ms_max = reduce_max(ms, world, dev)
+
+    # ---- staged loop: the same kernels through the three stage calls, for
+    # per-stage times and the grouped-expert kernel's duration
+    rt = omni.router_topk(t["x"], t["W_r"], t["W_c"], cfg.K)
+    sc = omni.schedule(rt["idx"], rt["gate"], cfg.N, cfg.B)
+    U = int(sc["num_distinct"].item())
+    ws_r = omni.router_workspace(L, cfg.N_r, cfg.N_c, cfg.K, dev)
+    ws_s = omni.schedule_workspace(L, cfg.K, cfg.N, cfg.B, dev)
+    ws_e = omni.expert_workspace(L, d, cfg.K, cfg.N, cfg.B, dev)
+    y2 = torch.zeros_like(y)
+
+    def staged(evs=None):
+        if evs:
+            evs[0].record(stream)
+        omni.omni_router_topk(t["x"], t["W_r"], t["W_c"], L, d, cfg.N_r, cfg.N_c, cfg.K,
+                              rt["p_r"], rt["p_c"], rt["idx"], rt["score"], rt["gate"], 0, ws_r)
+        if evs:
+            evs[1].record(stream)
+        omni.omni_schedule(rt["idx"], rt["gate"], L, cfg.K, cfg.N, cfg.B, sc["task_token"],
+                           sc["task_expert"], sc["task_gate"], sc["group_offsets"],
+                           sc["group_counts"], sc["active_groups"], sc["num_active"],
+                           sc["num_distinct"], ws_s)
+        if evs:
+            evs[2].record(stream)
+        omni.omni_grouped_expert_fwd(t["x"], t["W"], t["V"], L, d, cfg.K, cfg.N, cfg.B,
+                                     sc["task_token"], sc["task_expert"], sc["task_gate"],
+                                     sc["group_offsets"], sc["active_groups"], sc["num_active"],
+                                     y2, omni.OMNI_Y_ACCUMULATE, ws_e)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        staged()
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        staged(sev[i])
+    torch.cuda.synchronize()
+    barrier(world)
+    st_router = float(np.mean([e[0].elapsed_time(e[1]) for e in sev]))
+    st_sched = float(np.mean([e[1].elapsed_time(e[2]) for e in sev]))
+    st_expert = float(np.mean([e[2].elapsed_time(e[3]) for e in sev]))
+
+    # ---- end to end: host buffers, copies inside the timed region
+    x_host = t["x"].cpu().pin_memory()
+    y_host = torch.empty((L, d), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(t["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        omni.omni_routed_fwd(x_dev, t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r, cfg.N_c,
+                             cfg.K, cfg.B, y, None, None, 0, ws)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        eev[i][0].record(stream)
+        e2e_step()
+        eev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in eev])), world, dev)
+    if omni.omni_get_device_status(ws) != 0:
+        raise RuntimeError("device status set during timing")
+
+    peaks = measured_peaks()
+    # algorithmic bytes: the U distinct W and V rows, x read once, y written once
+    exp_bytes = 4.0 * d * U + 2.0 * L * d + 4.0 * L * d
+    layer_bytes = exp_bytes + 2.0 * d * (cfg.N_r + cfg.N_c)
+    layer_flops = 2.0 * L * d * (cfg.N_r + cfg.N_c) + 4.0 * cfg.M * d
+    achieved = exp_bytes / (st_expert * 1e-3) / 1e9
+    t_roof = max(layer_bytes / (peaks["hbm_gbs"] * 1e9),
+                 layer_flops / (peaks["bf16_tflops_sustained"] * 1e12))
+    out = {
+        "metric": METRIC,
+        "value": world * L / (ms_max * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian inputs and random-init weights of the layer's shapes)",
+        "config": {"workload": cfg.name, "L": L, "d": d, "N_r": cfg.N_r, "N_c": cfg.N_c,
+                   "N": cfg.N, "K": cfg.K, "B": cfg.B, "tokens_per_gpu": L,
+                   "parallelism": f"replicas x{world} (token batches)",
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "stages_ms": {"router_topk": st_router, "schedule": st_sched,
+                      "grouped_expert": st_expert},
+        "distinct_experts": U,
+        "roofline": {"bound": "hbm", "kernel": "grouped_expert (omni_grouped_expert_fwd)",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "peak_source": peaks["source"],
+                     "traffic": traffic_from_profile(
+                         os.path.join(ROOT, "atomic_expert_layer_b200", "csrc", "expert.cu")),
+                     "algorithmic_bytes_per_launch": exp_bytes},
+        "layer_roofline": {"t_roof_ms": t_roof * 1e3, "t_meas_ms": ms_max,
+                           "frac": t_roof * 1e3 / ms_max, "bytes": layer_bytes,
+                           "flops": layer_flops},
+        "e2e": {"value": world * L / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * L * d, "d2h_bytes_per_step": 4 * L * d,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step(cfg) * args.steps,
+        "clocks": clocks,
+    }
+    del t, ws, flush
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------- oracle (CPU) arm
+def time_oracle(cfg, n_tokens: int, seed: int = 0) -> dict:
+    """Time the CPU oracle on the first n_tokens of the workload (router,
+    top-K, gates, schedule, expert stage); inputs are made on the GPU if one
+    is present, else on the CPU, and only the expert rows the sample uses are
+    copied to the host (copying is not timed)."""
+    import oracle
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = inputs.make_inputs(cfg, dev, seed=seed)
+    x = inputs.to_u16(t["x"][:n_tokens])
+    Wr, Wc = inputs.to_u16(t["W_r"]), inputs.to_u16(t["W_c"])
+    t0 = time.perf_counter()
+    p_r, p_c = oracle.router_logprobs(x, Wr, Wc)
+    idx, score, gate = oracle.topk_from_logprobs(p_r, p_c, cfg.K)
+    t1 = time.perf_counter()
+    tok = torch.as_tensor(idx.astype(np.int64), device=dev)
+    uniq, inv = torch.unique(tok, return_inverse=True)
+    Wu, Vu = inputs.to_u16(t["W"][uniq]), inputs.to_u16(t["V"][uniq])
+    idx_local = inv.to(torch.int32).cpu().numpy()
+    t2 = time.perf_counter()
+    oracle.schedule(idx, gate, cfg.N, cfg.B)
+    oracle.expert_fwd_token_centric(x, Wu, Vu, idx_local, gate)
+    t3 = time.perf_counter()
+    del t
+    secs = (t1 - t0) + (t3 - t2)
+    return {"seconds": secs, "tokens": n_tokens, "value": n_tokens / secs,
+            "cores": oracle.max_threads()}
+
+
+def cpu_baseline(cfg, budget_s: float = 20.0) -> dict:
+    probe = min(cfg.L, 64)
+    r = time_oracle(cfg, probe)
+    per_tok = r["seconds"] / probe
+    n = int(max(probe, min(cfg.L, budget_s / max(per_tok, 1e-9))))
+    if n > probe:
+        r = time_oracle(cfg, n)
+    return {"value": r["value"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+            "sample": f"first {r['tokens']} of {cfg.L} tokens of {cfg.name}, whole routed "
+                      f"branch in the C oracle (fp64), {r['seconds']:.1f} s"}
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return None
+    n = min(cfg.L, 512)
+    for _ in range(args.warmup):
+        time_oracle(cfg, min(n, 16))
+    secs, toks, cores = 0.0, 0, 1
+    for _ in range(args.steps):
+        r = time_oracle(cfg, n)
+        secs += r["seconds"]
+        toks += r["tokens"]
+        cores = r["cores"]
+    value = toks / secs
+    sample = (f"first {n} of {cfg.L} tokens of {cfg.name} per step, whole routed branch in "
+              f"the C oracle (fp64)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * cfg.L / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "L": cfg.L, "d": cfg.d, "N_r": cfg.N_r,
+                   "N_c": cfg.N_c, "K": cfg.K, "B": cfg.B},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# -------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=configs.HEADLINE.name,
+                    help="workload name: " + ", ".join(c.name for c in configs.ALL))
+    ap.add_argument("--impl", choices=["omni", "reference"], default="omni")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = configs.BY_NAME[args.config]
+    world, rank, local = dist_env()
+    if world > 1 and args.impl == "omni":
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            out = run_reference(args, cfg, world, rank)
+        else:
+            out = run_omni(args, cfg, world, rank, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(cfg)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1 and args.impl == "omni":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

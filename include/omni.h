@@ -92,6 +92,12 @@ const char *omni_device_status_string(int dev_status);
  */
 size_t omni_workspace_size(int L, int d, int N_r, int N_c, int K, int B);
 
+/* Smaller workspaces for the three stage calls used on their own (each is at
+ * most omni_workspace_size of the same sizes).  0 for invalid sizes. */
+size_t omni_router_workspace_size(int L, int N_r, int N_c, int K);
+size_t omni_schedule_workspace_size(int L, int K, int N, int B);
+size_t omni_expert_workspace_size(int L, int d, int K, int N, int B);
+
 /*
  * Cartesian product router, [R] step 2 and [G] section 2.2.
  *   s_r = x W_r^T, s_c = x W_c^T            (bf16 inputs, fp32 accumulation)
@@ -131,8 +137,9 @@ int omni_router_topk(const omni_bf16 *x, const omni_bf16 *W_r, const omni_bf16 *
  *   num_active    [1]     int32   number of active groups
  *   num_distinct  [1]     int32   number of distinct experts among the tasks
  * idx [L, K] int32 and gate [L, K] fp32 are inputs (e.g. from omni_router_topk);
- * expert ids must lie in [0, N) and be distinct within a token (an id out of
- * range sets OMNI_DEV_BAD_EXPERT and that task is dropped from the counts).
+ * expert ids must lie in [0, N) and be distinct within a token.  An id out of
+ * range sets OMNI_DEV_BAD_EXPERT; that task is then given expert 0 and gate 0
+ * so that every later access stays in bounds.
  * Limits: M <= 2^31 - 1, B <= OMNI_MAX_B, K <= OMNI_MAX_K.
  * The output is bit-identical from run to run (the sort key is unique).
  */
@@ -180,6 +187,16 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                     int L, int d, int N_r, int N_c, int K, int B,
                     float *y, int32_t *idx_out, float *gate_out,
                     unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
+
+/*
+ * Diagnostic, not part of the layer: launches one CTA that waits on a
+ * shared-memory barrier nothing ever arrives at, through the same bounded
+ * wait the pipelined kernels use, with its limit set to `limit_ms`
+ * (1..10000).  The wait runs out, the kernel records OMNI_DEV_WAIT_TIMEOUT in
+ * the status word of `ws` and returns; the context stays usable.  Tests use
+ * it to check that a stuck wait ends with a status, not a hang.
+ */
+int omni_selftest_wait_timeout(void *ws, size_t ws_bytes, int limit_ms, omni_stream_t stream);
 
 /*
  * Synchronises `stream`, copies the status word of `ws` into *status_out

@@ -1,0 +1,105 @@
+"""The C-ABI library on the host: it loads, exports what include/omni.h
+declares, sizes workspaces and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import atomic_expert_layer_b200 as omni
+from atomic_expert_layer_b200 import _lib, build, configs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "omni.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(omni_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("omni_router_topk", "omni_schedule", "omni_grouped_expert_fwd", "omni_routed_fwd",
+              "omni_workspace_size", "omni_get_device_status"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_version_and_strings(lib):
+    assert lib.omni_version() == 1
+    assert lib.omni_status_string(-3) == b"OMNI_ERR_WORKSPACE"
+    assert lib.omni_device_status_string(2) == b"OMNI_DEV_WAIT_TIMEOUT"
+
+
+def test_workspace_sizes(lib):
+    h = configs.HEADLINE
+    full = omni.omni_workspace_size(h.L, h.d, h.N_r, h.N_c, h.K, h.B)
+    assert full > 0 and full % 256 == 0
+    r = omni.omni_router_workspace_size(h.L, h.N_r, h.N_c, h.K)
+    s = omni.omni_schedule_workspace_size(h.L, h.K, h.N, h.B)
+    e = omni.omni_expert_workspace_size(h.L, h.d, h.K, h.N, h.B)
+    assert 0 < r < full and 0 < s < full and 0 < e < full
+    # the scores s_r, s_c dominate the router part
+    assert r >= 4 * h.L * (h.N_r + h.N_c)
+    assert omni.omni_workspace_size(0, 8, 4, 4, 1, 1) == 0
+    assert omni.omni_workspace_size(4, 8, 4, 4, 17, 1) == 0         # K > N
+    assert omni.omni_workspace_size(4, 8, 4, 4, 4, 2048) == 0       # B above the limit
+    assert omni.omni_workspace_size(4, 8, 9000, 4, 4, 4) == 0       # axis above the limit
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_bad_arguments_rejected_on_host(lib):
+    """Every check below returns before any CUDA call (no GPU here)."""
+    fake = _p(1 << 20)                      # 16-byte aligned, never dereferenced
+    ws_small = 256
+    L, d, Nr, Nc, K, B = 4, 256, 4, 4, 2, 2
+    # null pointer
+    assert lib.omni_routed_fwd(None, fake, fake, fake, fake, L, d, Nr, Nc, K, B, fake, None, None,
+                               0, fake, 1 << 30, None) == -1
+    # K > N
+    assert lib.omni_routed_fwd(fake, fake, fake, fake, fake, L, d, Nr, Nc, 17, B, fake, None,
+                               None, 0, fake, 1 << 30, None) == -1
+    # d not a multiple of 256 for the expert stage
+    assert lib.omni_routed_fwd(fake, fake, fake, fake, fake, L, 264, Nr, Nc, K, B, fake, None,
+                               None, 0, fake, 1 << 30, None) == -2
+    # workspace too small
+    assert lib.omni_routed_fwd(fake, fake, fake, fake, fake, L, d, Nr, Nc, K, B, fake, None, None,
+                               0, fake, ws_small, None) == -3
+    # misaligned bf16 pointer
+    assert lib.omni_routed_fwd(_p((1 << 20) + 2), fake, fake, fake, fake, L, d, Nr, Nc, K, B,
+                               fake, None, None, 0, fake, 1 << 30, None) == -1
+    # misaligned workspace
+    assert lib.omni_schedule(fake, fake, L, K, 16, B, fake, fake, fake, fake, fake, fake, fake,
+                             fake, _p((1 << 20) + 64), 1 << 30, None) == -1
+    # N <= 0
+    assert lib.omni_grouped_expert_fwd(fake, fake, fake, L, d, K, 0, B, fake, fake, fake, fake,
+                                       fake, fake, fake, 0, fake, 1 << 30, None) == -1
+    # router: d must be a multiple of 8
+    assert lib.omni_router_topk(fake, fake, fake, L, 12, Nr, Nc, K, fake, fake, fake, fake, fake,
+                                0, fake, 1 << 30, None) == -2
+    # status query needs a workspace
+    out = ctypes.c_int(7)
+    assert lib.omni_get_device_status(None, 0, None, ctypes.byref(out)) == -1
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        _lib._ptr(x)
