@@ -54,5 +54,9 @@ def sweep(L: int) -> LayerConfig:
     return LayerConfig(f"sweep_L{L}_d2048_N1700416_K64_B128", L, 2048, 1304, 1304, 64, 128)
 
 
-ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L]
+# Headline structure at a size small enough for full profiler captures: the
+# same d, K, B and tasks per group (L*K*B/N = 20), with N = 512^2.
+PROFILE = LayerConfig("profile_L640_d1024_N262144_K64_B128", 640, 1024, 512, 512, 64, 128)
+
+ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L] + [PROFILE]
 BY_NAME = {c.name: c for c in ALL}

@@ -43,8 +43,6 @@ bool make_sizes(int L, int d, int N_r, int N_c, int K, int B, Sizes *sz) {
     sz->Kc = K < N_c ? K : N_c;
     sz->C = merge_candidates(K, sz->Kr, sz->Kc);
     sz->ntiles = (sz->M + kSortTile - 1) / kSortTile;
-    const int64_t gm = sz->G < sz->M ? sz->G : sz->M;
-    sz->max_items = gm + (sz->M + kItemTasks - 1) / kItemTasks;
     return true;
 }
 
@@ -70,7 +68,7 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.a_tok = take(4 * M); w.a_exp = take(4 * M); w.a_gate = take(4 * M);
         w.b_tok = take(4 * M); w.b_exp = take(4 * M); w.b_gate = take(4 * M);
         w.bitmap = take(4 * (size_t)((sz.N + 31) / 32));
-        w.hist = take(4 * 256 * (size_t)sz.ntiles);
+        w.hist = take(4 * 4 * 256 * (size_t)sz.ntiles);      // one per radix pass (<= 4)
     }
     if (regions & kRegSchedOut) {
         w.t_tok = take(4 * M); w.t_exp = take(4 * M); w.t_gate = take(4 * M);
@@ -80,7 +78,6 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.n_act = take(4);
         w.n_dist = take(4);
     }
-    if (regions & kRegExpert) w.items = take(16 * (size_t)sz.max_items);
     w.total = o;
     return w;
 }
@@ -266,8 +263,7 @@ int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_b
     if ((rc = check_ws(sz, kRegExpert, ws, ws_bytes, &lay))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = reset_header(ws, st))) return rc;
-    return cuda_rc(launch_grouped_expert(x, W, V, sz, task_token, task_expert, task_gate,
-                                         group_offsets, active_groups, num_active, y,
+    return cuda_rc(launch_grouped_expert(x, W, V, sz, task_token, task_expert, task_gate, y,
                                          (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st));
 }
 
@@ -300,7 +296,7 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     if ((rc = cuda_rc(launch_schedule(idx, gate, sz, tt, te, tg, goff, gcnt, gact, nact, ndist,
                                       ws, lay, st))))
         return rc;
-    if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, tt, te, tg, goff, gact, nact, y,
+    if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, tt, te, tg, y,
                                             (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st))))
         return rc;
     if (idx_out &&

@@ -9,7 +9,7 @@
 namespace omni {
 
 constexpr int kSortTile = 2048;        // tasks per radix-sort tile
-constexpr int kItemTasks = 256;        // max tasks per grouped-expert work item
+constexpr int kItemTasks = 128;        // sorted tasks per grouped-expert work item
 
 struct Sizes {
     int L, d, N_r, N_c, K, B;
@@ -17,13 +17,12 @@ struct Sizes {
     int Kr, Kc;          // row / column candidates: min(K, N_r), min(K, N_c)
     int C;               // merge candidates: cells (a, b) with (a+1)(b+1) <= K
     int64_t ntiles;      // radix tiles
-    int64_t max_items;   // grouped-expert work items, upper bound
 };
 
 struct WsLayout {
     size_t hdr, s_r, s_c, row_val, row_idx, col_val, col_idx, idx, score, gate;
     size_t a_tok, a_exp, a_gate, b_tok, b_exp, b_gate, t_tok, t_exp, t_gate;
-    size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, items;
+    size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist;
     size_t total;
 };
 
@@ -34,7 +33,7 @@ enum WsRegion : unsigned {
     kRegRouter = 1u,      // s_r, s_c, axis candidates, idx / score / gate
     kRegSched = 2u,       // sort buffers, expert bitmap, radix histograms
     kRegSchedOut = 4u,    // sorted tasks and group arrays (routed forward only)
-    kRegExpert = 8u,      // work items
+    kRegExpert = 8u,      // (the expert stage needs only the header)
     kRegAll = 15u
 };
 
@@ -72,9 +71,8 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
 cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const uint16_t *V,
                                   const Sizes &sz, const int32_t *task_token,
                                   const int32_t *task_expert, const float *task_gate,
-                                  const int32_t *group_offsets, const int32_t *active_groups,
-                                  const int32_t *num_active, float *y, bool accumulate,
-                                  void *ws, const WsLayout &lay, cudaStream_t st);
+                                  float *y, bool accumulate, void *ws, const WsLayout &lay,
+                                  cudaStream_t st);
 
 int device_sm_count();
 

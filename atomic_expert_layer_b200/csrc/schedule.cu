@@ -10,13 +10,15 @@
 //
 // Pipeline (no host synchronisation, no spin-waits):
 //   1. prepare (warp per token): sort the token's K tasks by expert id, write
-//      them in (t, e) order, count tasks per group, mark experts in a bitmap.
-//   2. group scan (1 CTA): exclusive scan of the group counts, active-group
-//      list, number of distinct experts.
-//   3. LSD radix sort of the tasks on q alone, 8-bit digits, stable.  The
-//      input is in (t, e) order, so a stable sort by q yields (q, t, e).
-//      Each pass: per-tile digit histogram, one exclusive scan, stable scatter
-//      (warps rank equal digits with __match_any_sync, in input order).
+//      them in (t, e) order, count tasks per group, mark experts in a bitmap,
+//      and count the first radix pass's digits per 2048-task tile (atomics).
+//   2. scans (one launch, two CTAs): group offsets, active-group list and
+//      distinct-expert count; the first pass's digit-major histogram.
+//   3. LSD radix sort of the tasks on q alone, digits of <= 8 bits, stable.
+//      The input is in (t, e) order, so a stable sort by q yields (q, t, e).
+//      Each pass: stable scatter (warps rank equal digits with
+//      __match_any_sync, in input order) that also counts the next pass's
+//      digits of its output, then one scan of that histogram.
 #include "omni_common.cuh"
 #include "omni_internal.h"
 
@@ -26,12 +28,21 @@ namespace {
 constexpr int kScatterThreads = 256;                       // 8 warps
 constexpr int kItemsPerWarp = kSortTile / (kScatterThreads / 32);   // 256
 
+// ------------------------------------------------------------ radix digits
+__device__ __forceinline__ uint32_t digit_of(int32_t e, int B, int shift, uint32_t dmask) {
+    return ((uint32_t)(e / B) >> shift) & dmask;
+}
+
 // ---------------------------------------------------------- 1. prepare
+// Warp per token: sort the token's K tasks by expert id, write them at
+// t*K + rank, count tasks per group, mark experts, and count the first radix
+// pass's digits per tile (so no separate histogram pass is needed).
 __global__ void sched_prepare_kernel(const int32_t *__restrict__ idx,
                                      const float *__restrict__ gate, int L, int K, int N, int B,
                                      int32_t *__restrict__ a_tok, int32_t *__restrict__ a_exp,
                                      float *__restrict__ a_gate, int32_t *__restrict__ counts,
-                                     uint32_t *__restrict__ bitmap, int *status) {
+                                     uint32_t *__restrict__ bitmap, int32_t *__restrict__ hist0,
+                                     int64_t ntiles, uint32_t dmask0, int *status) {
     extern __shared__ int32_t sh_e[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
@@ -55,131 +66,173 @@ __global__ void sched_prepare_kernel(const int32_t *__restrict__ idx,
             const int32_t ev = e_s[v];
             r += (ev < eu) | ((ev == eu) & (v < u));
         }
-        const float g = (idx[row + u] < 0 || idx[row + u] >= N) ? 0.f : gate[row + u];
-        a_tok[row + r] = t;
-        a_exp[row + r] = eu;
-        a_gate[row + r] = g;
+        const int32_t raw = idx[row + u];
+        const float g = (raw < 0 || raw >= N) ? 0.f : gate[row + u];
+        const size_t pos = row + r;
+        a_tok[pos] = t;
+        a_exp[pos] = eu;
+        a_gate[pos] = g;
         atomicAdd(&counts[eu / B], 1);
         atomicOr(&bitmap[eu >> 5], 1u << (eu & 31));
+        if (hist0) atomicAdd(&hist0[(int64_t)digit_of(eu, B, 0, dmask0) * ntiles + pos / kSortTile], 1);
     }
 }
 
-// ----------------------------------------------------- 2. group scan
-// One CTA of 1024 threads; thread t owns a contiguous chunk of groups.
-__global__ void __launch_bounds__(1024) sched_group_scan_kernel(
-    const int32_t *__restrict__ counts, int64_t G, const uint32_t *__restrict__ bitmap,
-    int64_t nwords, int32_t *__restrict__ offsets, int32_t *__restrict__ active,
-    int32_t *__restrict__ num_active, int32_t *__restrict__ num_distinct) {
-    __shared__ int sh_sum[32], sh_act[32], sh_pop[32];
-    const int tid = threadIdx.x;
-    const int64_t per = (G + 1023) / 1024;
-    const int64_t g0 = (int64_t)tid * per;
-    const int64_t g1 = g0 + per < G ? g0 + per : G;
-    int sum = 0, act = 0, pop = 0;
-    for (int64_t g = g0; g < g1; ++g) {
-        const int c = counts[g];
-        sum += c;
-        act += c > 0;
-    }
-    for (int64_t w = tid; w < nwords; w += 1024) pop += __popc(bitmap[w]);
-    // block exclusive scans of sum and act, block sum of pop
-    const int lane = tid & 31, warp = tid >> 5;
-    const int isum = warp_iscan(sum), iact = warp_iscan(act);
-    const int wpop = warp_isum(pop);
-    if (lane == 31) {
-        sh_sum[warp] = isum;
-        sh_act[warp] = iact;
-    }
-    if (lane == 0) sh_pop[warp] = wpop;
+// ------------------------------------------------ block scan (1024 threads)
+// Exclusive scan of one int per thread; returns the block total in *total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *sh32, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int incl = warp_iscan(v);
+    __syncthreads();                       // sh32 may still be read by a previous call
+    if (lane == 31) sh32[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        const int s = sh_sum[lane], a = sh_act[lane], p = sh_pop[lane];
-        const int is = warp_iscan(s), ia = warp_iscan(a), ps = warp_isum(p);
-        sh_sum[lane] = is - s;
-        sh_act[lane] = ia - a;
-        if (lane == 31) {
-            offsets[G] = is;
-            *num_active = ia;
-        }
-        if (lane == 0) *num_distinct = ps;
+        const int s = sh32[lane];
+        const int is = warp_iscan(s);
+        sh32[lane] = is - s;
+        if (lane == 31) sh32[32] = is;
     }
     __syncthreads();
-    int run = sh_sum[warp] + isum - sum;
-    int arun = sh_act[warp] + iact - act;
-    for (int64_t g = g0; g < g1; ++g) {
-        const int c = counts[g];
-        offsets[g] = run;
-        run += c;
-        if (c > 0) active[arun++] = (int32_t)g;
+    *total = sh32[32];
+    return sh32[warp] + incl - v;
+}
+
+constexpr int kScanTile = 4096;            // elements per tile: 1024 threads x 4
+
+// In-place exclusive scan of a[0..n) by one CTA of 1024 threads.  Tiles of
+// 4096 are loaded coalesced into shared memory; each thread then owns 4
+// consecutive elements.  If `tail` is non-null the total is written there.
+__device__ void cta_exclusive_scan(int32_t *a, int64_t n, int32_t *tail, int *tile, int *sh32) {
+    const int tid = threadIdx.x;
+    int carry = 0;
+    for (int64_t base = 0; base < n; base += kScanTile) {
+        __syncthreads();
+        for (int k = 0; k < 4; ++k) {
+            const int64_t i = base + k * 1024 + tid;
+            tile[k * 1024 + tid] = i < n ? a[i] : 0;
+        }
+        __syncthreads();
+        int v[4], sum = 0;
+        for (int k = 0; k < 4; ++k) {
+            v[k] = tile[4 * tid + k];
+            sum += v[k];
+        }
+        int total;
+        int run = carry + block_exclusive_scan(sum, sh32, &total);
+        for (int k = 0; k < 4; ++k) {
+            tile[4 * tid + k] = run;
+            run += v[k];
+        }
+        carry += total;
+        __syncthreads();
+        for (int k = 0; k < 4; ++k) {
+            const int64_t i = base + k * 1024 + tid;
+            if (i < n) a[i] = tile[k * 1024 + tid];
+        }
+    }
+    if (tail && tid == 0) *tail = carry;
+}
+
+// ----------------------------------------------------- 2. group scan
+// CTA 0: group offsets (exclusive scan of counts), active groups, distinct
+// experts.  CTA 1 (if a radix pass follows): exclusive scan of the first
+// pass's digit-major histogram.
+__global__ void __launch_bounds__(1024) sched_scan_kernel(
+    const int32_t *__restrict__ counts, int64_t G, const uint32_t *__restrict__ bitmap,
+    int64_t nwords, int32_t *__restrict__ offsets, int32_t *__restrict__ active,
+    int32_t *__restrict__ num_active, int32_t *__restrict__ num_distinct,
+    int32_t *__restrict__ hist0, int64_t nhist) {
+    __shared__ int tile[kScanTile];
+    __shared__ int tile2[kScanTile];
+    __shared__ int sh32[33];
+    const int tid = threadIdx.x;
+    if (blockIdx.x == 1) {
+        cta_exclusive_scan(hist0, nhist, nullptr, tile, sh32);
+        return;
+    }
+    int carry = 0, acarry = 0, pop = 0;
+    for (int64_t w = tid; w < nwords; w += 1024) pop += __popc(bitmap[w]);
+    for (int64_t base = 0; base < G; base += kScanTile) {
+        __syncthreads();
+        for (int k = 0; k < 4; ++k) {
+            const int64_t i = base + k * 1024 + tid;
+            tile[k * 1024 + tid] = i < G ? counts[i] : 0;
+        }
+        __syncthreads();
+        int v[4], sum = 0, act = 0;
+        for (int k = 0; k < 4; ++k) {
+            v[k] = tile[4 * tid + k];
+            sum += v[k];
+            act += v[k] > 0;
+        }
+        int total, atotal;
+        int run = carry + block_exclusive_scan(sum, sh32, &total);
+        int arun = acarry + block_exclusive_scan(act, sh32, &atotal);
+        for (int k = 0; k < 4; ++k) {
+            const int64_t g = base + 4 * tid + k;
+            tile2[4 * tid + k] = run;
+            run += v[k];
+            if (v[k] > 0 && g < G) active[arun++] = (int32_t)g;
+        }
+        carry += total;
+        acarry += atotal;
+        __syncthreads();
+        for (int k = 0; k < 4; ++k) {
+            const int64_t i = base + k * 1024 + tid;
+            if (i < G) offsets[i] = tile2[k * 1024 + tid];
+        }
+    }
+    int ptotal;
+    block_exclusive_scan(pop, sh32, &ptotal);
+    if (tid == 0) {
+        offsets[G] = carry;
+        *num_active = acarry;
+        *num_distinct = ptotal;
     }
 }
 
 // --------------------------------------------------- 3. radix passes
-__device__ __forceinline__ uint32_t digit_of(int32_t e, int B, int shift, uint32_t dmask) {
-    return ((uint32_t)(e / B) >> shift) & dmask;
-}
-
-__global__ void __launch_bounds__(kScatterThreads) radix_hist_kernel(
-    const int32_t *__restrict__ src_exp, int64_t M, int B, int shift, uint32_t dmask,
-    int64_t ntiles, int32_t *__restrict__ hist) {
-    __shared__ int h[256];
-    const int tid = threadIdx.x;
-    h[tid] = 0;
-    __syncthreads();
-    const int64_t base = (int64_t)blockIdx.x * kSortTile;
-    for (int i = tid; i < kSortTile; i += kScatterThreads) {
-        const int64_t m = base + i;
-        if (m < M) atomicAdd(&h[digit_of(src_exp[m], B, shift, dmask)], 1);
-    }
-    __syncthreads();
-    if ((uint32_t)tid <= dmask) hist[(int64_t)tid * ntiles + blockIdx.x] = h[tid];
-}
-
 // Exclusive scan of n ints in place, one CTA of 1024 threads.
 __global__ void __launch_bounds__(1024) exclusive_scan_kernel(int32_t *__restrict__ a,
                                                              int64_t n) {
-    __shared__ int sh[32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t per = (n + 1023) / 1024;
-    const int64_t i0 = (int64_t)tid * per;
-    const int64_t i1 = i0 + per < n ? i0 + per : n;
-    int sum = 0;
-    for (int64_t i = i0; i < i1; ++i) sum += a[i];
-    const int incl = warp_iscan(sum);
-    if (lane == 31) sh[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const int s = sh[lane];
-        sh[lane] = warp_iscan(s) - s;
-    }
-    __syncthreads();
-    int run = sh[warp] + incl - sum;
-    for (int64_t i = i0; i < i1; ++i) {
-        const int v = a[i];
-        a[i] = run;
-        run += v;
-    }
+    __shared__ int tile[kScanTile];
+    __shared__ int sh32[33];
+    cta_exclusive_scan(a, n, nullptr, tile, sh32);
 }
 
+constexpr int kRounds = kItemsPerWarp / 32;                       // 8
+
 // Stable scatter of one tile.  Warp w owns tile items [w*256, (w+1)*256) and
-// walks them in rounds of 32, so ranks follow input order.
+// walks them in rounds of 32, so ranks follow input order.  If hist_next is
+// given, the digits of the next pass are counted per output tile.
 __global__ void __launch_bounds__(kScatterThreads) radix_scatter_kernel(
     const int32_t *__restrict__ src_tok, const int32_t *__restrict__ src_exp,
     const float *__restrict__ src_gate, int64_t M, int B, int shift, uint32_t dmask,
     int64_t ntiles, const int32_t *__restrict__ hist_scanned, int32_t *__restrict__ dst_tok,
-    int32_t *__restrict__ dst_exp, float *__restrict__ dst_gate) {
+    int32_t *__restrict__ dst_exp, float *__restrict__ dst_gate,
+    int32_t *__restrict__ hist_next, int next_shift, uint32_t next_dmask) {
     __shared__ int wcount[kScatterThreads / 32][256];
     const int tid = threadIdx.x, warp = tid >> 5;
     const unsigned lane = lane_id();
     for (int i = tid; i < (kScatterThreads / 32) * 256; i += kScatterThreads)
         (&wcount[0][0])[i] = 0;
-    __syncthreads();
     const int64_t wbase = (int64_t)blockIdx.x * kSortTile + (int64_t)warp * kItemsPerWarp;
-    // per-warp digit counts
-    for (int j = 0; j < kItemsPerWarp; j += 32) {
-        const int64_t m = wbase + j + lane;
+    int32_t e[kRounds], tk[kRounds];
+    float g[kRounds];
+#pragma unroll
+    for (int j = 0; j < kRounds; ++j) {
+        const int64_t m = wbase + j * 32 + lane;
         const bool valid = m < M;
-        const uint32_t dg = valid ? digit_of(src_exp[m], B, shift, dmask) : 0xffffffffu;
+        e[j] = valid ? src_exp[m] : -1;
+        tk[j] = valid ? src_tok[m] : 0;
+        g[j] = valid ? src_gate[m] : 0.f;
+    }
+    __syncthreads();
+    // per-warp digit counts
+#pragma unroll
+    for (int j = 0; j < kRounds; ++j) {
+        const bool valid = e[j] >= 0;
+        const uint32_t dg = valid ? digit_of(e[j], B, shift, dmask) : 0xffffffffu;
         const unsigned peers = __match_any_sync(0xffffffffu, dg);
         if (valid && (lanemask_lt() & peers) == 0) wcount[warp][dg] += __popc(peers);
         __syncwarp();
@@ -195,23 +248,19 @@ __global__ void __launch_bounds__(kScatterThreads) radix_scatter_kernel(
         }
     }
     __syncthreads();
-    for (int j = 0; j < kItemsPerWarp; j += 32) {
-        const int64_t m = wbase + j + lane;
-        const bool valid = m < M;
-        int32_t e = 0, tk = 0;
-        float g = 0.f;
-        if (valid) {
-            e = src_exp[m];
-            tk = src_tok[m];
-            g = src_gate[m];
-        }
-        const uint32_t dg = valid ? digit_of(e, B, shift, dmask) : 0xffffffffu;
+#pragma unroll
+    for (int j = 0; j < kRounds; ++j) {
+        const bool valid = e[j] >= 0;
+        const uint32_t dg = valid ? digit_of(e[j], B, shift, dmask) : 0xffffffffu;
         const unsigned peers = __match_any_sync(0xffffffffu, dg);
         if (valid) {
             const int pos = wcount[warp][dg] + __popc(peers & lanemask_lt());
-            dst_tok[pos] = tk;
-            dst_exp[pos] = e;
-            dst_gate[pos] = g;
+            dst_tok[pos] = tk[j];
+            dst_exp[pos] = e[j];
+            dst_gate[pos] = g[j];
+            if (hist_next)
+                atomicAdd(&hist_next[(int64_t)digit_of(e[j], B, next_shift, next_dmask) * ntiles +
+                                     pos / kSortTile], 1);
         }
         __syncwarp();
         if (valid && (lanemask_lt() & peers) == 0) wcount[warp][dg] += __popc(peers);
@@ -235,40 +284,55 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
     uint32_t *bitmap = ws_at<uint32_t>(ws, lay.bitmap);
     int32_t *hist = ws_at<int32_t>(ws, lay.hist);
     const int64_t nwords = (sz.N + 31) / 32;
+    const int64_t ntiles = sz.ntiles;
+    const int64_t hstride = 256 * ntiles;                // one histogram per pass
     cudaError_t e;
-
-    if ((e = cudaMemsetAsync(group_counts, 0, sizeof(int32_t) * G, st)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(bitmap, 0, sizeof(uint32_t) * nwords, st)) != cudaSuccess) return e;
-    {
-        const int wpb = 8;
-        const size_t smem = sizeof(int32_t) * (size_t)sz.K * wpb;
-        sched_prepare_kernel<<<(unsigned)((sz.L + wpb - 1) / wpb), 32 * wpb, smem, st>>>(
-            idx, gate, sz.L, sz.K, (int)sz.N, sz.B, a_tok, a_exp, a_gate, group_counts, bitmap,
-            status);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    sched_group_scan_kernel<<<1, 1024, 0, st>>>(group_counts, G, bitmap, nwords, group_offsets,
-                                                 active_groups, num_active, num_distinct);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // radix passes over q = e / B
     int nbits = 0;
     while (nbits < 31 && ((int64_t)1 << nbits) < G) ++nbits;       // bits of G - 1
     const int passes = (nbits + 7) / 8;
+    const int width = passes ? (nbits + passes - 1) / passes : 0;
+    auto pass_mask = [&](int p) -> uint32_t {
+        const int shift = p * width;
+        const int w = (nbits - shift) < width ? (nbits - shift) : width;
+        return (1u << w) - 1u;
+    };
+
+    if ((e = cudaMemsetAsync(group_counts, 0, sizeof(int32_t) * G, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(bitmap, 0, sizeof(uint32_t) * nwords, st)) != cudaSuccess) return e;
+    if (passes > 0 &&
+        (e = cudaMemsetAsync(hist, 0, sizeof(int32_t) * hstride * passes, st)) != cudaSuccess)
+        return e;
+    {
+        const int wpb = 8;
+        const size_t smem = sizeof(int32_t) * (size_t)sz.K * wpb;
+        sched_prepare_kernel<<<(unsigned)((sz.L + wpb - 1) / wpb), 32 * wpb, smem, st>>>(
+            idx, gate, sz.L, sz.K, (int)sz.N, sz.B, a_tok, a_exp, a_gate, group_counts, bitmap,
+            passes ? hist : nullptr, ntiles, passes ? pass_mask(0) : 0u, status);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    sched_scan_kernel<<<passes ? 2 : 1, 1024, 0, st>>>(
+        group_counts, G, bitmap, nwords, group_offsets, active_groups, num_active, num_distinct,
+        hist, passes ? (int64_t)(pass_mask(0) + 1) * ntiles : 0);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
     if (passes == 0) {
         if ((e = cudaMemcpyAsync(task_token, a_tok, 4 * M, cudaMemcpyDeviceToDevice, st))) return e;
         if ((e = cudaMemcpyAsync(task_expert, a_exp, 4 * M, cudaMemcpyDeviceToDevice, st))) return e;
         return cudaMemcpyAsync(task_gate, a_gate, 4 * M, cudaMemcpyDeviceToDevice, st);
     }
-    const int width = (nbits + passes - 1) / passes;
-    const int64_t ntiles = sz.ntiles;
     const int32_t *s_tok = a_tok, *s_exp = a_exp;
     const float *s_gate = a_gate;
     for (int p = 0; p < passes; ++p) {
         const int shift = p * width;
-        const int w = (nbits - shift) < width ? (nbits - shift) : width;
-        const uint32_t dmask = (1u << w) - 1u;
+        const uint32_t dmask = pass_mask(p);
         const bool last = p == passes - 1;
+        int32_t *h = hist + hstride * p;
+        if (p > 0) {
+            exclusive_scan_kernel<<<1, 1024, 0, st>>>(h, (int64_t)(dmask + 1) * ntiles);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
         // ping-pong: the last pass writes the caller's arrays
         int32_t *d_tok, *d_exp;
         float *d_gate;
@@ -279,13 +343,10 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
         } else {
             d_tok = a_tok; d_exp = a_exp; d_gate = a_gate;
         }
-        radix_hist_kernel<<<(unsigned)ntiles, kScatterThreads, 0, st>>>(s_exp, M, sz.B, shift,
-                                                                         dmask, ntiles, hist);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        exclusive_scan_kernel<<<1, 1024, 0, st>>>(hist, (int64_t)(dmask + 1) * ntiles);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
         radix_scatter_kernel<<<(unsigned)ntiles, kScatterThreads, 0, st>>>(
-            s_tok, s_exp, s_gate, M, sz.B, shift, dmask, ntiles, hist, d_tok, d_exp, d_gate);
+            s_tok, s_exp, s_gate, M, sz.B, shift, dmask, ntiles, h, d_tok, d_exp, d_gate,
+            last ? nullptr : hist + hstride * (p + 1), (p + 1) * width,
+            last ? 0u : pass_mask(p + 1));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         s_tok = d_tok; s_exp = d_exp; s_gate = d_gate;
     }

@@ -330,6 +330,42 @@ def run_omni(args, cfg, world, rank, local):
     return out
 
 
+def profile_stage(args, cfg):
+    """Run one stage (or the whole layer) W + K times, synchronising at the end."""
+    import atomic_expert_layer_b200 as omni
+    dev = torch.device("cuda", 0)
+    omni.load()
+    t = inputs.make_inputs(cfg, dev, seed=0,
+                           with_experts=args.profile_stage in ("expert", "all"))
+    L, d = cfg.L, cfg.d
+    rt = omni.router_topk(t["x"], t["W_r"], t["W_c"], cfg.K)
+    sc = omni.schedule(rt["idx"], rt["gate"], cfg.N, cfg.B)
+    ws = omni.workspace(L, d, cfg.N_r, cfg.N_c, cfg.K, cfg.B, dev)
+    y = torch.zeros((L, d), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup + args.steps):
+        if args.profile_stage == "router":
+            omni.omni_router_topk(t["x"], t["W_r"], t["W_c"], L, d, cfg.N_r, cfg.N_c, cfg.K,
+                                  rt["p_r"], rt["p_c"], rt["idx"], rt["score"], rt["gate"], 0, ws)
+        elif args.profile_stage == "schedule":
+            omni.omni_schedule(rt["idx"], rt["gate"], L, cfg.K, cfg.N, cfg.B, sc["task_token"],
+                               sc["task_expert"], sc["task_gate"], sc["group_offsets"],
+                               sc["group_counts"], sc["active_groups"], sc["num_active"],
+                               sc["num_distinct"], ws)
+        elif args.profile_stage == "expert":
+            omni.omni_grouped_expert_fwd(t["x"], t["W"], t["V"], L, d, cfg.K, cfg.N, cfg.B,
+                                         sc["task_token"], sc["task_expert"], sc["task_gate"],
+                                         sc["group_offsets"], sc["active_groups"],
+                                         sc["num_active"], y, omni.OMNI_Y_ACCUMULATE, ws)
+        else:
+            omni.omni_routed_fwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r,
+                                 cfg.N_c, cfg.K, cfg.B, y, None, None, 0, ws)
+    torch.cuda.synchronize()
+    status = omni.omni_get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    print(f"profile-stage {args.profile_stage} {cfg.name}: {args.warmup + args.steps} runs ok")
+
+
 # ------------------------------------------------------- oracle (CPU) arm
 def time_oracle(cfg, n_tokens: int, seed: int = 0) -> dict:
     """Time the CPU oracle on the first n_tokens of the workload (router,
@@ -410,6 +446,8 @@ def main():
                     help="workload name: " + ", ".join(c.name for c in configs.ALL))
     ap.add_argument("--impl", choices=["omni", "reference"], default="omni")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-stage", choices=["router", "schedule", "expert", "all"],
+                    help="run only this stage W + K times (for profiler captures; no JSON)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -421,6 +459,9 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     try:
+        if args.profile_stage:
+            profile_stage(args, cfg)
+            return
         if args.impl == "reference":
             out = run_reference(args, cfg, world, rank)
         else:
