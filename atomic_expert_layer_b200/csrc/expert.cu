@@ -81,13 +81,19 @@ struct ExpertCfg {
     static constexpr int kSlotBytes = 2 * kRowBytes;     // W row + V row
     static constexpr int kConsumers = VPL <= 2 ? 16 : (VPL <= 4 ? 12 : 6);  // consumer warps
     static constexpr int kThreads = 32 * (1 + kConsumers);
-    static constexpr int kFixed = ((int)(sizeof(ChunkMeta) * kNChunk + sizeof(ProducerScratch) +
-                                         24 * kNChunk + 1023) / 1024) * 1024;
+    // after the slots: chunk metadata, producer scratch, then the barriers on
+    // a 16-byte boundary (mbarriers need 8-byte alignment)
+    static constexpr int kMetaBytes = (int)(sizeof(ChunkMeta) * kNChunk);
+    static constexpr int kBarOff = ((kMetaBytes + (int)sizeof(ProducerScratch) + 15) / 16) * 16;
+    static constexpr int kFixed = ((kBarOff + 3 * 8 * kNChunk + 1023) / 1024) * 1024;
     static constexpr int kNSlot = (kSmemBudget - kFixed) / kSlotBytes;
     static constexpr int kMaxChunk = kNSlot / 2;         // experts per chunk
     static constexpr int kSmem = kFixed + kNSlot * kSlotBytes;
     static_assert(kNSlot >= 8, "ring too small");
+    static_assert((kNSlot * kSlotBytes) % 1024 == 0, "slots keep 1 KB alignment");
+    static_assert((kNSlot * kSlotBytes + kBarOff) % 16 == 0, "barriers 16-byte aligned");
 };
+static_assert(sizeof(ChunkMeta) % 4 == 0, "metadata entries stay 4-byte aligned");
 
 constexpr int kTPL = kItemTasks / 32;                    // tasks per producer lane
 
@@ -106,9 +112,10 @@ grouped_expert_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict
     extern __shared__ __align__(1024) uint8_t smem[];
     // slots first, then chunk metadata, producer scratch and barriers
     uint8_t *slots = smem;
-    ChunkMeta *meta = reinterpret_cast<ChunkMeta *>(smem + (size_t)NSLOT * Cfg::kSlotBytes);
-    ProducerScratch *ps = reinterpret_cast<ProducerScratch *>(meta + kNChunk);
-    uint64_t *meta_full = reinterpret_cast<uint64_t *>(ps + 1);   // chunk described
+    uint8_t *fixed = smem + (size_t)NSLOT * Cfg::kSlotBytes;
+    ChunkMeta *meta = reinterpret_cast<ChunkMeta *>(fixed);
+    ProducerScratch *ps = reinterpret_cast<ProducerScratch *>(fixed + Cfg::kMetaBytes);
+    uint64_t *meta_full = reinterpret_cast<uint64_t *>(fixed + Cfg::kBarOff);   // chunk described
     uint64_t *data_full = meta_full + kNChunk;                    // its rows have landed
     uint64_t *empty = data_full + kNChunk;                        // consumers are done
 
