@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/omni.h"
+#include "omni.h"
 
 namespace omni {
 
