@@ -54,9 +54,10 @@ def sweep(L: int) -> LayerConfig:
     return LayerConfig(f"sweep_L{L}_d2048_N1700416_K64_B128", L, 2048, 1304, 1304, 64, 128)
 
 
-# Headline structure at a size small enough for full profiler captures: the
-# same d, K, B and tasks per group (L*K*B/N = 20), with N = 512^2.
-PROFILE = LayerConfig("profile_L640_d1024_N262144_K64_B128", 640, 1024, 512, 512, 64, 128)
+# Headline task structure at a size small enough for full profiler captures:
+# the same L, d, K, tasks (M = 262,144) and tasks per group (L*K*B/N = 20),
+# with W and V of 512 MB each (N = 512^2) instead of 3.5 GB.
+PROFILE = LayerConfig("profile_L4096_d1024_N262144_K64_B20", 4096, 1024, 512, 512, 64, 20)
 
 ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L] + [PROFILE]
 BY_NAME = {c.name: c for c in ALL}

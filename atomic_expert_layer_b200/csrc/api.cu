@@ -78,6 +78,10 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.n_act = take(4);
         w.n_dist = take(4);
     }
+    if (regions & kRegExpert) {
+        w.tok_count = take(4 * L);
+        w.tok_slots = take(8 * M);
+    }
     w.total = o;
     return w;
 }

@@ -8,25 +8,26 @@
 // its tokens and G_q the gate of each (token, expert) task, 0 elsewhere.
 // sigma is read as SiLU (each atomic expert has a single w_in).
 //
-// Design.  The cost is the gather of the active expert rows (2*d bytes each
-// for W and V) from HBM; G_q is sparse (about 8% dense for 4096 tokens over
-// 1.7M experts), so only the task pairs are computed, on CUDA cores, and the
-// kernel is built to keep many independent row loads in flight:
-//   - every warp owns a contiguous share of the sorted task array (no work
-//     list, no claiming); it cuts its share where the group changes;
-//   - inside a group segment the warp goes expert by expert (expert-major):
-//     the W and V rows of an expert are loaded once and used for every token
-//     of the segment that chose it.  Rows are prefetched kStages-1 experts
-//     ahead with cp.async (16 bytes per lane) into the warp's own shared-
-//     memory ring, so each warp keeps several rows in flight without
-//     spending registers on them;
-//   - per task the warp computes h = x_t . w_e (warp reduction),
-//     p = g * SiLU(h) and adds p * v_e into y[t] with vector reductions
-//     (red.global.add.v4.f32); y is L2-resident for typical L.  The x row of
-//     the next task is loaded while the current one is computed.
+// Two kernels, no atomics on y:
+//   1. group pass (expert-centric, per group as the pages have it):
+//      P_q = G_q . SiLU(X_q W_q^T) for the task pairs only (G_q is about 8%
+//      dense for 4096 tokens over 1.7M experts).  Every warp owns a
+//      contiguous share of the sorted tasks and cuts it where the group
+//      changes; inside a group segment it goes expert by expert, loading each
+//      W row once (cp.async, 16 bytes per lane, kStages-1 experts ahead into
+//      the warp's own shared-memory ring) and using it for every token of
+//      the segment that chose it.  Each task's p = g * SiLU(x_t . w_e) is
+//      written with its expert id into a slot of its token.
+//   2. token pass: y[t] = sum over the token's slots of p * V[e], one warp
+//      per token, V rows prefetched the same way; y is written once per
+//      token.  This is O_q = P_q V_q plus the scatter-add, regrouped by
+//      token: on B200 the fp32 reductions of per-group partial rows into y
+//      (16-byte red.global.add.v4.f32, one L2 sector operation each) ran at
+//      about 3 TB/s and cost more than the HBM gather they were meant to
+//      follow, while V rows are used about 1.1 times per group at this scale.
 // A warp that shares a group with its neighbour reloads the experts common
-// to both halves (about one row per warp boundary).  No waits on other warps
-// or other CTAs exist in this kernel.
+// to both halves (about one row per warp boundary).  No kernel here waits on
+// another warp or CTA.
 #include "omni_common.cuh"
 #include "omni_internal.h"
 
@@ -42,10 +43,10 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float *f) {
     }
 }
 
-// ---------------------------------------------------------- main kernel
+// ---------------------------------------------------------- common parts
 constexpr int kSub = 256;                 // tasks staged per sub-range
 
-// Per-warp scratch for one sub-range of tasks.
+// Per-warp scratch of the group pass for one sub-range of tasks.
 struct WarpScratch {
     int tok[kSub];
     int exp[kSub];
@@ -71,54 +72,59 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// copy one bf16 row of 256*VPL elements into shared memory, 16 bytes per lane
 template <int VPL>
-struct ExpertCfg {
-    static constexpr int kD = 256 * VPL;                 // d
-    static constexpr int kRowBytes = 2 * kD;             // one bf16 row
-    static constexpr int kPairBytes = 2 * kRowBytes;     // W row + V row
-    static constexpr int kStages = VPL <= 1 ? 6 : (VPL <= 2 ? 5 : (VPL <= 4 ? 4 : 3));
-    static constexpr int kWarpBytes = kStages * kPairBytes + (int)sizeof(WarpScratch);
-    static constexpr int kWarpsFit = (227 * 1024) / kWarpBytes;
-    static constexpr int kWarps = kWarpsFit > 16 ? 16 : kWarpsFit;
-    static constexpr int kThreads = 32 * kWarps;
-    static constexpr int kSmem = kWarps * kWarpBytes;
+__device__ __forceinline__ void row_async(uint8_t *dst, const uint16_t *src, unsigned lane) {
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) cp_async16(dst + (size_t)(v * 32 + lane) * 16, s4 + v * 32 + lane);
+}
+
+template <int VPL, int STAGES, int EXTRA>
+struct WarpSmem {
+    static constexpr int kRowBytes = 512 * VPL;
+    static constexpr int kWarpBytes = STAGES * kRowBytes + EXTRA;
+    static constexpr int kFit = (227 * 1024) / kWarpBytes;
+    static constexpr int kWarps = kFit > 16 ? 16 : kFit;
     static_assert(kWarps >= 2, "too little shared memory per warp");
-    static_assert(kPairBytes % 16 == 0, "ring slots stay 16-byte aligned");
+    static_assert(kWarpBytes % 16 == 0, "per-warp areas stay 16-byte aligned");
 };
 
 template <int VPL>
-__global__ void __launch_bounds__(ExpertCfg<VPL>::kThreads, 1)
-grouped_expert_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W,
-                      const uint16_t *__restrict__ V, int L, int N, int B, int M, int per_warp,
-                      const int32_t *__restrict__ task_token,
-                      const int32_t *__restrict__ task_expert,
-                      const float *__restrict__ task_gate, float *__restrict__ y, int *status) {
-    using Cfg = ExpertCfg<VPL>;
-    constexpr int D = Cfg::kD;
+struct GateCfg {
+    static constexpr int kStages = VPL <= 2 ? 8 : (VPL <= 4 ? 6 : 4);
+    using Smem = WarpSmem<VPL, kStages, (int)sizeof(WarpScratch)>;
+};
+template <int VPL>
+struct CombineCfg {
+    static constexpr int kStages = VPL <= 2 ? 10 : (VPL <= 4 ? 8 : 5);
+    static constexpr int kWarps = 4;                      // per CTA; several CTAs per SM
+    static constexpr int kRowBytes = 512 * VPL;
+    static constexpr int kSmem = kWarps * kStages * kRowBytes;
+};
+
+// ------------------------------------------------------- 1. group pass
+template <int VPL>
+__global__ void __launch_bounds__(32 * GateCfg<VPL>::Smem::kWarps, 1)
+group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W, int L, int N,
+                  int B, int K, int M, int per_warp, const int32_t *__restrict__ task_token,
+                  const int32_t *__restrict__ task_expert, const float *__restrict__ task_gate,
+                  int *__restrict__ tok_count, int2 *__restrict__ tok_slots, int *status) {
+    using Cfg = GateCfg<VPL>;
+    using Sm = typename Cfg::Smem;
+    constexpr int D = 256 * VPL;
     constexpr int S = Cfg::kStages;
-    constexpr int RB = Cfg::kRowBytes;
+    constexpr int RB = Sm::kRowBytes;
     extern __shared__ __align__(16) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
-    uint8_t *ring = smem + (size_t)warp * Cfg::kWarpBytes;
-    WarpScratch &sc = *reinterpret_cast<WarpScratch *>(ring + S * Cfg::kPairBytes);
+    uint8_t *ring = smem + (size_t)warp * Sm::kWarpBytes;
+    WarpScratch &sc = *reinterpret_cast<WarpScratch *>(ring + S * RB);
     const int nwords = (B + 31) >> 5;
 
-    const int64_t gw = (int64_t)blockIdx.x * Cfg::kWarps + warp;
+    const int64_t gw = (int64_t)blockIdx.x * Sm::kWarps + warp;
     const int64_t a0 = gw * per_warp;
     const int64_t a1 = a0 + per_warp < M ? a0 + per_warp : M;
-
-    // issue the cp.async copies of one expert's W and V rows into ring slot k % S
-    auto issue = [&](int k, int64_t e) {
-        uint8_t *slot = ring + (k % S) * Cfg::kPairBytes;
-        const uint4 *wsrc = reinterpret_cast<const uint4 *>(W + e * D);
-        const uint4 *vsrc = reinterpret_cast<const uint4 *>(V + e * D);
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-            cp_async16(slot + (size_t)(v * 32 + lane) * 16, wsrc + v * 32 + lane);
-            cp_async16(slot + RB + (size_t)(v * 32 + lane) * 16, vsrc + v * 32 + lane);
-        }
-    };
 
     for (int64_t sub = a0; sub < a1; sub += kSub) {
         const int n = (int)(a1 - sub < kSub ? a1 - sub : kSub);
@@ -177,11 +183,10 @@ grouped_expert_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict
             // start the first S-1 experts' rows while the ordering is built
 #pragma unroll
             for (int k = 0; k < S - 1; ++k) {
-                if (k < n_e) issue(k, ebase + sc.rlist[k]);
+                if (k < n_e) row_async<VPL>(ring + (k % S) * RB, W + (ebase + sc.rlist[k]) * D, lane);
                 cp_async_commit();
             }
-            // per task: expert rank; per expert: task count (deterministic,
-            // in task order)
+            // per task: expert rank; per expert: task count (in task order)
             for (int j0 = js; j0 < je; j0 += 32) {
                 const int j = j0 + (int)lane;
                 const bool in = j < je;
@@ -221,9 +226,8 @@ grouped_expert_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict
                 if (in && (peers & lanemask_lt()) == 0) sc.start[rk] += __popc(peers);
                 __syncwarp();
             }
-            // start[] now holds each expert's end; the tasks are order[0 .. je-js)
             const int ns = je - js;
-            // ---- expert-major pass
+            // ---- expert-major pass: p for every task of the segment
             uint4 xr[VPL], xn[VPL];
             {
                 const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)sc.tok[sc.order[0]] * D);
@@ -235,13 +239,13 @@ grouped_expert_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict
                 const int j = sc.order[i];
                 const int k = sc.rank[j];
                 if (k != cur) {
-                    // expert k's rows: its group is the (k+1)-th committed;
-                    // allow S-2 newer groups to stay in flight
+                    // expert k's row is the (k+1)-th committed group; allow the
+                    // S-2 newer groups to stay in flight
                     cp_async_wait<S - 2>();
                     __syncwarp();
                     cur = k;
                     const int kn = k + S - 1;
-                    if (kn < n_e) issue(kn, ebase + sc.rlist[kn]);
+                    if (kn < n_e) row_async<VPL>(ring + (kn % S) * RB, W + (ebase + sc.rlist[kn]) * D, lane);
                     cp_async_commit();
                 }
                 if (i + 1 < ns) {
@@ -250,9 +254,7 @@ grouped_expert_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict
 #pragma unroll
                     for (int v = 0; v < VPL; ++v) xn[v] = __ldg(src + v * 32 + lane);
                 }
-                const uint8_t *slot = ring + (k % S) * Cfg::kPairBytes;
-                const uint4 *wr = reinterpret_cast<const uint4 *>(slot);
-                const uint4 *vr = reinterpret_cast<const uint4 *>(slot + RB);
+                const uint4 *wr = reinterpret_cast<const uint4 *>(ring + (k % S) * RB);
                 float h = 0.f;
 #pragma unroll
                 for (int v = 0; v < VPL; ++v) {
@@ -263,15 +265,14 @@ grouped_expert_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict
                     for (int c = 0; c < 8; ++c) h = fmaf(xf[c], wf[c], h);
                 }
                 h = warp_sum(h);
-                const float p = sc.gate[j] * (h / (1.f + __expf(-h)));
-                float *yr = y + (size_t)sc.tok[j] * D;
-#pragma unroll
-                for (int v = 0; v < VPL; ++v) {
-                    float vf[8];
-                    bf16x8_to_f32(vr[v * 32 + lane], vf);
-                    float *dst = yr + (size_t)(v * 32 + lane) * 8;
-                    red_add_v4(dst, p * vf[0], p * vf[1], p * vf[2], p * vf[3]);
-                    red_add_v4(dst + 4, p * vf[4], p * vf[5], p * vf[6], p * vf[7]);
+                if (lane == 0) {
+                    const float p = sc.gate[j] * (h / (1.f + __expf(-h)));
+                    const int t = sc.tok[j];
+                    const int slot = atomicAdd(&tok_count[t], 1);
+                    if (slot < K)
+                        tok_slots[(size_t)t * K + slot] = make_int2(sc.exp[j], __float_as_int(p));
+                    else
+                        set_status(status, OMNI_DEV_BAD_SCHEDULE);
                 }
                 if (i + 1 < ns) {
 #pragma unroll
@@ -286,22 +287,131 @@ grouped_expert_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict
     }
 }
 
+// ------------------------------------------------------- 2. token pass
+// One warp per token (grid-stride): y[t] (+)= sum_s p_s * V[e_s].
+template <int VPL>
+__global__ void __launch_bounds__(32 * CombineCfg<VPL>::kWarps)
+token_combine_kernel(const uint16_t *__restrict__ V, int L, int N, int K,
+                     const int *__restrict__ tok_count, const int2 *__restrict__ tok_slots,
+                     float *__restrict__ y, int accumulate, int *status) {
+    using Cfg = CombineCfg<VPL>;
+    constexpr int D = 256 * VPL;
+    constexpr int S = Cfg::kStages;
+    constexpr int RB = Cfg::kRowBytes;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const unsigned lane = lane_id();
+    uint8_t *ring = smem + (size_t)warp * S * RB;
+    const int nwarps = gridDim.x * Cfg::kWarps;
+    for (int t = blockIdx.x * Cfg::kWarps + warp; t < L; t += nwarps) {
+        int n = tok_count[t];
+        if (n > K) {
+            set_status(status, OMNI_DEV_BAD_SCHEDULE);
+            n = K;
+        }
+        const int2 *sl = tok_slots + (size_t)t * K;
+        // expert ids of the token's first 32 slots, one per lane
+        int2 mine = lane < (unsigned)n ? sl[lane] : make_int2(0, 0);
+        if (mine.x < 0 || mine.x >= N) mine.x = 0;
+        auto expert_of = [&](int s) -> int {
+            // slot s lives in lane s % 32 of the block of 32 slots holding it
+            return __shfl_sync(0xffffffffu, mine.x, s & 31);
+        };
+        float acc[VPL * 8];
+#pragma unroll
+        for (int c = 0; c < VPL * 8; ++c) acc[c] = 0.f;
+#pragma unroll
+        for (int s = 0; s < S - 1; ++s) {
+            if (s < n) row_async<VPL>(ring + (s % S) * RB, V + (size_t)expert_of(s) * D, lane);
+            cp_async_commit();
+        }
+        for (int s = 0; s < n; ++s) {
+            cp_async_wait<S - 2>();
+            __syncwarp();
+            const float p = __int_as_float(__shfl_sync(0xffffffffu, mine.y, s & 31));
+            const int sn = s + S - 1;
+            int en = 0;
+            if (sn < n) {
+                if ((sn >> 5) == (s >> 5)) {
+                    en = expert_of(sn);                // held by the lanes of this block
+                } else {
+                    const int2 nx = sl[sn];            // next block: same address in every lane
+                    en = (nx.x < 0 || nx.x >= N) ? 0 : nx.x;
+                }
+                row_async<VPL>(ring + (sn % S) * RB, V + (size_t)en * D, lane);
+            }
+            cp_async_commit();
+            const uint4 *vr = reinterpret_cast<const uint4 *>(ring + (s % S) * RB);
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                float vf[8];
+                bf16x8_to_f32(vr[v * 32 + lane], vf);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[8 * v + c] = fmaf(p, vf[c], acc[8 * v + c]);
+            }
+            if (((s + 1) & 31) == 0 && s + 1 < n) {
+                // next block of 32 slots
+                mine = (s + 1 + (int)lane) < n ? sl[s + 1 + lane] : make_int2(0, 0);
+                if (mine.x < 0 || mine.x >= N) mine.x = 0;
+            }
+        }
+        cp_async_wait<0>();
+        __syncwarp();
+        float *yr = y + (size_t)t * D;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+            float4 *dst = reinterpret_cast<float4 *>(yr + (size_t)(v * 32 + lane) * 8);
+            float4 a = make_float4(acc[8 * v], acc[8 * v + 1], acc[8 * v + 2], acc[8 * v + 3]);
+            float4 b = make_float4(acc[8 * v + 4], acc[8 * v + 5], acc[8 * v + 6], acc[8 * v + 7]);
+            if (accumulate) {
+                const float4 oa = dst[0], ob = dst[1];
+                a.x += oa.x; a.y += oa.y; a.z += oa.z; a.w += oa.w;
+                b.x += ob.x; b.y += ob.y; b.z += ob.z; b.w += ob.w;
+            }
+            dst[0] = a;
+            dst[1] = b;
+        }
+    }
+}
+
 template <int VPL>
 cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, const Sizes &sz,
                        const int32_t *tt, const int32_t *te, const float *tg, float *y,
-                       int *status, cudaStream_t st) {
-    using Cfg = ExpertCfg<VPL>;
-    cudaError_t e = cudaFuncSetAttribute(grouped_expert_kernel<VPL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+                       bool accumulate, int *tok_count, int2 *tok_slots, int *status,
+                       cudaStream_t st) {
+    using G = GateCfg<VPL>;
+    using C = CombineCfg<VPL>;
+    constexpr int gwarps = G::Smem::kWarps;
+    constexpr int gsmem = gwarps * G::Smem::kWarpBytes;
+    cudaError_t e = cudaFuncSetAttribute(group_gate_kernel<VPL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, gsmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(token_combine_kernel<VPL>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     const int sms = device_sm_count();
-    const int64_t warps = (int64_t)sms * Cfg::kWarps;
-    int64_t per_warp = (sz.M + warps - 1) / warps;
-    if (per_warp < 32) per_warp = 32;
-    const int64_t needed = (sz.M + per_warp - 1) / per_warp;          // warps with work
-    const int grid = (int)((needed + Cfg::kWarps - 1) / Cfg::kWarps);
-    grouped_expert_kernel<VPL><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(
-        x, W, V, sz.L, (int)sz.N, sz.B, (int)sz.M, (int)per_warp, tt, te, tg, y, status);
+    if ((e = cudaMemsetAsync(tok_count, 0, sizeof(int) * (size_t)sz.L, st)) != cudaSuccess) return e;
+    {
+        const int64_t warps = (int64_t)sms * gwarps;
+        int64_t per_warp = (sz.M + warps - 1) / warps;
+        if (per_warp < 32) per_warp = 32;
+        const int64_t needed = (sz.M + per_warp - 1) / per_warp;      // warps with work
+        const int grid = (int)((needed + gwarps - 1) / gwarps);
+        group_gate_kernel<VPL><<<grid, 32 * gwarps, gsmem, st>>>(
+            x, W, sz.L, (int)sz.N, sz.B, sz.K, (int)sz.M, (int)per_warp, tt, te, tg, tok_count,
+            tok_slots, status);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        int per_sm = (227 * 1024) / C::kSmem;
+        if (per_sm < 1) per_sm = 1;
+        if (per_sm > 8) per_sm = 8;
+        int64_t grid = (int64_t)sms * per_sm;
+        const int64_t need = (sz.L + C::kWarps - 1) / C::kWarps;
+        if (grid > need) grid = need;
+        token_combine_kernel<VPL><<<(unsigned)grid, 32 * C::kWarps, C::kSmem, st>>>(
+            V, sz.L, (int)sz.N, sz.K, tok_count, tok_slots, y, accumulate ? 1 : 0, status);
+    }
     return cudaGetLastError();
 }
 
@@ -313,20 +423,15 @@ cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const ui
                                   float *y, bool accumulate, void *ws, const WsLayout &lay,
                                   cudaStream_t st) {
     int *status = ws_at<int>(ws, lay.hdr);
-    cudaError_t e;
-    if (!accumulate) {
-        if ((e = cudaMemsetAsync(y, 0, sizeof(float) * (size_t)sz.L * sz.d, st)) != cudaSuccess)
-            return e;
-    }
+    int *tok_count = ws_at<int>(ws, lay.tok_count);
+    int2 *tok_slots = ws_at<int2>(ws, lay.tok_slots);
     switch (sz.d / 256) {
-        case 1: return launch_vpl<1>(x, W, V, sz, task_token, task_expert, task_gate, y, status, st);
-        case 2: return launch_vpl<2>(x, W, V, sz, task_token, task_expert, task_gate, y, status, st);
-        case 3: return launch_vpl<3>(x, W, V, sz, task_token, task_expert, task_gate, y, status, st);
-        case 4: return launch_vpl<4>(x, W, V, sz, task_token, task_expert, task_gate, y, status, st);
-        case 5: return launch_vpl<5>(x, W, V, sz, task_token, task_expert, task_gate, y, status, st);
-        case 6: return launch_vpl<6>(x, W, V, sz, task_token, task_expert, task_gate, y, status, st);
-        case 7: return launch_vpl<7>(x, W, V, sz, task_token, task_expert, task_gate, y, status, st);
-        case 8: return launch_vpl<8>(x, W, V, sz, task_token, task_expert, task_gate, y, status, st);
+#define OMNI_CASE(n) \
+        case n: return launch_vpl<n>(x, W, V, sz, task_token, task_expert, task_gate, y, accumulate, \
+                                     tok_count, tok_slots, status, st);
+        OMNI_CASE(1) OMNI_CASE(2) OMNI_CASE(3) OMNI_CASE(4)
+        OMNI_CASE(5) OMNI_CASE(6) OMNI_CASE(7) OMNI_CASE(8)
+#undef OMNI_CASE
         default: return cudaErrorInvalidValue;
     }
 }

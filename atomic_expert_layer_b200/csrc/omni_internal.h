@@ -22,7 +22,7 @@ struct Sizes {
 struct WsLayout {
     size_t hdr, s_r, s_c, row_val, row_idx, col_val, col_idx, idx, score, gate;
     size_t a_tok, a_exp, a_gate, b_tok, b_exp, b_gate, t_tok, t_exp, t_gate;
-    size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist;
+    size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, tok_count, tok_slots;
     size_t total;
 };
 
@@ -33,7 +33,7 @@ enum WsRegion : unsigned {
     kRegRouter = 1u,      // s_r, s_c, axis candidates, idx / score / gate
     kRegSched = 2u,       // sort buffers, expert bitmap, radix histograms
     kRegSchedOut = 4u,    // sorted tasks and group arrays (routed forward only)
-    kRegExpert = 8u,      // (the expert stage needs only the header)
+    kRegExpert = 8u,      // per-token slots of (expert, p) between the two expert kernels
     kRegAll = 15u
 };
 
