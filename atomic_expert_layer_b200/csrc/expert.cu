@@ -13,10 +13,11 @@
 //      P_q = G_q . SiLU(X_q W_q^T) for the task pairs only (G_q is about 8%
 //      dense for 4096 tokens over 1.7M experts).  Every warp owns a
 //      contiguous share of the sorted tasks and cuts it where the group
-//      changes; inside a group segment it goes expert by expert, loading each
-//      W row once (cp.async, 16 bytes per lane, kStages-1 experts ahead into
-//      the warp's own shared-memory ring) and using it for every token of
-//      the segment that chose it.  Each task's p = g * SiLU(x_t . w_e) is
+//      changes; it orders its tasks by expert id (a counting sort inside
+//      each group) and goes expert by expert, loading each W row once
+//      (cp.async, 16 bytes per lane, kStages-1 experts ahead into the warp's
+//      own shared-memory ring, one continuous stream across groups) and
+//      using it for every token of the group that chose it.  Each task's p = g * SiLU(x_t . w_e) is
 //      written with its expert id into a slot of its token.
 //   2. token pass: y[t] = sum over the token's slots of p * V[e], one warp
 //      per token, V rows prefetched the same way; y is written once per
@@ -51,10 +52,11 @@ struct WarpScratch {
     int tok[kSub];
     int exp[kSub];
     float gate[kSub];
-    uint16_t rank[kSub];          // rank of the task's expert within its segment
+    uint16_t rank[kSub];          // rank of the task's expert in the sub-range's expert list
     uint16_t order[kSub];         // segment tasks, expert-major
+    int slot[kSub];               // the task's slot among its token's K slots
     int start[kSub + 4];          // per expert rank: first position in order[] (+ padding)
-    uint16_t rlist[kSub];         // distinct experts of the segment (r = e - q*B)
+    int elist[kSub];              // distinct experts of the sub-range, ascending
     uint32_t bitmap[OMNI_MAX_B / 32];
     int word_prefix[OMNI_MAX_B / 32];
 };
@@ -139,11 +141,17 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
             sc.tok[j] = t;
             sc.exp[j] = e;
             sc.gate[j] = task_gate[sub + j];
+            // claim the task's slot now, 32 tasks per round trip
+            sc.slot[j] = atomicAdd(&tok_count[t], 1);
         }
         __syncwarp();
-        int js = 0;
-        while (js < n) {
-            // ---- segment [js, je): the run of tasks of one group
+        // ---- setup for the whole sub-range: tasks sorted by expert id (the
+        // sub-range is in (group, token, expert) order, so this is a per-group
+        // counting sort on e - q*B), expert list, expert-major task order
+        for (int k = lane; k <= n; k += 32) sc.start[k] = 0;
+        __syncwarp();
+        int n_e = 0;
+        for (int js = 0; js < n;) {
             const int q = sc.exp[js] / B;
             int je = n;
             for (int j0 = js + 1; j0 < n; j0 += 32) {
@@ -156,7 +164,6 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
                 }
             }
             const int64_t ebase = (int64_t)q * B;
-            // distinct experts, ranked by expert id
             for (int w = lane; w < nwords; w += 32) sc.bitmap[w] = 0u;
             __syncwarp();
             for (int j = js + lane; j < je; j += 32) {
@@ -167,26 +174,18 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
             const uint32_t wbits = lane < (unsigned)nwords ? sc.bitmap[lane] : 0u;
             const int cnt = __popc(wbits);
             const int incl = warp_iscan(cnt);
-            const int n_e = __shfl_sync(0xffffffffu, incl, 31);
             if (lane < (unsigned)nwords) {
                 sc.word_prefix[lane] = incl - cnt;
                 uint32_t bits = wbits;
-                int pos = incl - cnt;
+                int pos = n_e + incl - cnt;
                 while (bits) {
                     const int b = __ffs(bits) - 1;
-                    sc.rlist[pos++] = (uint16_t)(lane * 32 + b);
+                    sc.elist[pos++] = (int)(ebase + lane * 32 + b);
                     bits &= bits - 1;
                 }
             }
-            for (int k = lane; k <= n_e; k += 32) sc.start[k] = 0;
             __syncwarp();
-            // start the first S-1 experts' rows while the ordering is built
-#pragma unroll
-            for (int k = 0; k < S - 1; ++k) {
-                if (k < n_e) row_async<VPL>(ring + (k % S) * RB, W + (ebase + sc.rlist[k]) * D, lane);
-                cp_async_commit();
-            }
-            // per task: expert rank; per expert: task count (in task order)
+            // per task: global expert rank; per expert: task count (task order)
             for (int j0 = js; j0 < je; j0 += 32) {
                 const int j = j0 + (int)lane;
                 const bool in = j < je;
@@ -194,96 +193,100 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
                 if (in) {
                     const int r = (int)(sc.exp[j] - ebase);
                     const int wd = r >> 5;
-                    rk = sc.word_prefix[wd] + __popc(sc.bitmap[wd] & ((1u << (r & 31)) - 1u));
+                    rk = n_e + sc.word_prefix[wd] + __popc(sc.bitmap[wd] & ((1u << (r & 31)) - 1u));
                     sc.rank[j] = (uint16_t)rk;
                 }
                 const unsigned peers = __match_any_sync(0xffffffffu, rk);
                 if (in && (peers & lanemask_lt()) == 0) sc.start[rk + 1] += __popc(peers);
                 __syncwarp();
             }
-            // exclusive scan of the counts -> start[k]
-            {
-                int carry = 0;
-                for (int k0 = 0; k0 <= n_e; k0 += 32) {
-                    const int k = k0 + (int)lane;
-                    const int v = k <= n_e ? sc.start[k] : 0;
-                    const int inc = warp_iscan(v);
-                    if (k <= n_e) sc.start[k] = carry + inc;
-                    carry += __shfl_sync(0xffffffffu, inc, 31);
-                }
-            }
-            __syncwarp();
-            // place tasks expert-major, keeping task order inside an expert
-            for (int j0 = js; j0 < je; j0 += 32) {
-                const int j = j0 + (int)lane;
-                const bool in = j < je;
-                const int rk = in ? (int)sc.rank[j] : 0x7fffffff;
-                const unsigned peers = __match_any_sync(0xffffffffu, rk);
-                int base = 0;
-                if (in) base = sc.start[rk];
-                if (in) sc.order[base + __popc(peers & lanemask_lt())] = (uint16_t)j;
-                __syncwarp();
-                if (in && (peers & lanemask_lt()) == 0) sc.start[rk] += __popc(peers);
-                __syncwarp();
-            }
-            const int ns = je - js;
-            // ---- expert-major pass: p for every task of the segment
-            uint4 xr[VPL], xn[VPL];
-            {
-                const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)sc.tok[sc.order[0]] * D);
-#pragma unroll
-                for (int v = 0; v < VPL; ++v) xr[v] = __ldg(src + v * 32 + lane);
-            }
-            int cur = -1;
-            for (int i = 0; i < ns; ++i) {
-                const int j = sc.order[i];
-                const int k = sc.rank[j];
-                if (k != cur) {
-                    // expert k's row is the (k+1)-th committed group; allow the
-                    // S-2 newer groups to stay in flight
-                    cp_async_wait<S - 2>();
-                    __syncwarp();
-                    cur = k;
-                    const int kn = k + S - 1;
-                    if (kn < n_e) row_async<VPL>(ring + (kn % S) * RB, W + (ebase + sc.rlist[kn]) * D, lane);
-                    cp_async_commit();
-                }
-                if (i + 1 < ns) {
-                    const uint4 *src =
-                        reinterpret_cast<const uint4 *>(x + (size_t)sc.tok[sc.order[i + 1]] * D);
-#pragma unroll
-                    for (int v = 0; v < VPL; ++v) xn[v] = __ldg(src + v * 32 + lane);
-                }
-                const uint4 *wr = reinterpret_cast<const uint4 *>(ring + (k % S) * RB);
-                float h = 0.f;
-#pragma unroll
-                for (int v = 0; v < VPL; ++v) {
-                    float xf[8], wf[8];
-                    bf16x8_to_f32(xr[v], xf);
-                    bf16x8_to_f32(wr[v * 32 + lane], wf);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) h = fmaf(xf[c], wf[c], h);
-                }
-                h = warp_sum(h);
-                if (lane == 0) {
-                    const float p = sc.gate[j] * (h / (1.f + __expf(-h)));
-                    const int t = sc.tok[j];
-                    const int slot = atomicAdd(&tok_count[t], 1);
-                    if (slot < K)
-                        tok_slots[(size_t)t * K + slot] = make_int2(sc.exp[j], __float_as_int(p));
-                    else
-                        set_status(status, OMNI_DEV_BAD_SCHEDULE);
-                }
-                if (i + 1 < ns) {
-#pragma unroll
-                    for (int v = 0; v < VPL; ++v) xr[v] = xn[v];
-                }
-            }
-            // drain this segment's remaining copies before the ring is reused
-            cp_async_wait<0>();
-            __syncwarp();
+            n_e += __shfl_sync(0xffffffffu, incl, 31);
             js = je;
         }
+        // start the first S-1 experts' rows while the order is built
+#pragma unroll
+        for (int k = 0; k < S - 1; ++k) {
+            if (k < n_e) row_async<VPL>(ring + (k % S) * RB, W + (size_t)sc.elist[k] * D, lane);
+            cp_async_commit();
+        }
+        // exclusive scan of the counts -> start[k]
+        {
+            int carry = 0;
+            for (int k0 = 0; k0 <= n_e; k0 += 32) {
+                const int k = k0 + (int)lane;
+                const int v = k <= n_e ? sc.start[k] : 0;
+                const int inc = warp_iscan(v);
+                if (k <= n_e) sc.start[k] = carry + inc;
+                carry += __shfl_sync(0xffffffffu, inc, 31);
+            }
+        }
+        __syncwarp();
+        // place tasks expert-major, keeping task order inside an expert
+        for (int j0 = 0; j0 < n; j0 += 32) {
+            const int j = j0 + (int)lane;
+            const bool in = j < n;
+            const int rk = in ? (int)sc.rank[j] : 0x7fffffff;
+            const unsigned peers = __match_any_sync(0xffffffffu, rk);
+            int base = 0;
+            if (in) base = sc.start[rk];
+            if (in) sc.order[base + __popc(peers & lanemask_lt())] = (uint16_t)j;
+            __syncwarp();
+            if (in && (peers & lanemask_lt()) == 0) sc.start[rk] += __popc(peers);
+            __syncwarp();
+        }
+        // ---- expert-major pass over the sub-range: p for every task
+        uint4 xr[VPL], xn[VPL];
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)sc.tok[sc.order[0]] * D);
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) xr[v] = __ldg(src + v * 32 + lane);
+        }
+        int cur = -1;
+        for (int i = 0; i < n; ++i) {
+            const int j = sc.order[i];
+            const int k = sc.rank[j];
+            if (k != cur) {
+                // expert k's row is the (k+1)-th committed group; allow the
+                // S-2 newer groups to stay in flight
+                cp_async_wait<S - 2>();
+                __syncwarp();
+                cur = k;
+                const int kn = k + S - 1;
+                if (kn < n_e) row_async<VPL>(ring + (kn % S) * RB, W + (size_t)sc.elist[kn] * D, lane);
+                cp_async_commit();
+            }
+            if (i + 1 < n) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)sc.tok[sc.order[i + 1]] * D);
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) xn[v] = __ldg(src + v * 32 + lane);
+            }
+            const uint4 *wr = reinterpret_cast<const uint4 *>(ring + (k % S) * RB);
+            float h = 0.f;
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                float xf[8], wf[8];
+                bf16x8_to_f32(xr[v], xf);
+                bf16x8_to_f32(wr[v * 32 + lane], wf);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) h = fmaf(xf[c], wf[c], h);
+            }
+            h = warp_sum(h);
+            if (lane == 0) {
+                const float p = sc.gate[j] * (h / (1.f + __expf(-h)));
+                const int slot = sc.slot[j];
+                if (slot < K)
+                    tok_slots[(size_t)sc.tok[j] * K + slot] = make_int2(sc.exp[j], __float_as_int(p));
+                else
+                    set_status(status, OMNI_DEV_BAD_SCHEDULE);
+            }
+            if (i + 1 < n) {
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) xr[v] = xn[v];
+            }
+        }
+        // drain the remaining copies before the ring is reused
+        cp_async_wait<0>();
+        __syncwarp();
     }
 }
 
