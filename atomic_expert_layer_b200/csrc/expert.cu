@@ -15,9 +15,9 @@
 //      contiguous share of the sorted tasks and cuts it where the group
 //      changes; it orders its tasks by expert id (a counting sort inside
 //      each group) and goes expert by expert, loading each W row once
-//      (cp.async, 16 bytes per lane, kStages-1 experts ahead into the warp's
-//      own shared-memory ring, one continuous stream across groups) and
-//      using it for every token of the group that chose it.  Each task's p = g * SiLU(x_t . w_e) is
+//      (cp.async, 16 bytes per lane, into the warp's own shared-memory ring)
+//      and using it for every token of the group that chose it.  The x rows
+//      of the tasks stream through a second ring, kStages-1 tasks ahead.  Each task's p = g * SiLU(x_t . w_e) is
 //      written with its expert id into a slot of its token.
 //   2. token pass: y[t] = sum over the token's slots of p * V[e], one warp
 //      per token, V rows prefetched the same way; y is written once per
@@ -94,8 +94,9 @@ struct WarpSmem {
 
 template <int VPL>
 struct GateCfg {
-    static constexpr int kStages = VPL <= 2 ? 8 : (VPL <= 4 ? 6 : 4);
-    using Smem = WarpSmem<VPL, kStages, (int)sizeof(WarpScratch)>;
+    // tasks in flight per warp; each stage holds a W row and an x row
+    static constexpr int kStages = VPL <= 1 ? 10 : (VPL <= 2 ? 8 : (VPL <= 4 ? 6 : 4));
+    using Smem = WarpSmem<VPL, 2 * kStages, (int)sizeof(WarpScratch)>;
 };
 template <int VPL>
 struct CombineCfg {
@@ -120,8 +121,9 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
     extern __shared__ __align__(16) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
-    uint8_t *ring = smem + (size_t)warp * Sm::kWarpBytes;
-    WarpScratch &sc = *reinterpret_cast<WarpScratch *>(ring + S * RB);
+    uint8_t *ring = smem + (size_t)warp * Sm::kWarpBytes;          // S W rows, then S x rows
+    WarpScratch &sc = *reinterpret_cast<WarpScratch *>(ring + 2 * S * RB);
+    static_assert(Sm::kWarpBytes == 2 * S * RB + (int)sizeof(WarpScratch), "per-warp layout");
     const int nwords = (B + 31) >> 5;
 
     const int64_t gw = (int64_t)blockIdx.x * Sm::kWarps + warp;
@@ -203,12 +205,6 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
             n_e += __shfl_sync(0xffffffffu, incl, 31);
             js = je;
         }
-        // start the first S-1 experts' rows while the order is built
-#pragma unroll
-        for (int k = 0; k < S - 1; ++k) {
-            if (k < n_e) row_async<VPL>(ring + (k % S) * RB, W + (size_t)sc.elist[k] * D, lane);
-            cp_async_commit();
-        }
         // exclusive scan of the counts -> start[k]
         {
             int carry = 0;
@@ -234,38 +230,39 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
             if (in && (peers & lanemask_lt()) == 0) sc.start[rk] += __popc(peers);
             __syncwarp();
         }
-        // ---- expert-major pass over the sub-range: p for every task
-        uint4 xr[VPL], xn[VPL];
-        {
-            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)sc.tok[sc.order[0]] * D);
-#pragma unroll
-            for (int v = 0; v < VPL; ++v) xr[v] = __ldg(src + v * 32 + lane);
-        }
-        int cur = -1;
-        for (int i = 0; i < n; ++i) {
+        // ---- expert-major pass over the sub-range: p for every task.
+        // Stream unit = one task: its x row (x ring slot i % S) and, for the
+        // first task of an expert, the expert's W row (W ring slot k % S).
+        // Tasks i .. i+S-1 span at most S experts, so a W slot is refilled only
+        // after every task of its previous expert has been computed.
+        uint8_t *wring = ring;
+        uint8_t *xring = ring + S * RB;
+        auto issue = [&](int i) {
             const int j = sc.order[i];
             const int k = sc.rank[j];
-            if (k != cur) {
-                // expert k's row is the (k+1)-th committed group; allow the
-                // S-2 newer groups to stay in flight
-                cp_async_wait<S - 2>();
-                __syncwarp();
-                cur = k;
-                const int kn = k + S - 1;
-                if (kn < n_e) row_async<VPL>(ring + (kn % S) * RB, W + (size_t)sc.elist[kn] * D, lane);
-                cp_async_commit();
-            }
-            if (i + 1 < n) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)sc.tok[sc.order[i + 1]] * D);
-#pragma unroll
-                for (int v = 0; v < VPL; ++v) xn[v] = __ldg(src + v * 32 + lane);
-            }
-            const uint4 *wr = reinterpret_cast<const uint4 *>(ring + (k % S) * RB);
+            if (i == 0 || sc.rank[sc.order[i - 1]] != k)
+                row_async<VPL>(wring + (k % S) * RB, W + (size_t)sc.elist[k] * D, lane);
+            row_async<VPL>(xring + (i % S) * RB, x + (size_t)sc.tok[j] * D, lane);
+        };
+#pragma unroll 1
+        for (int i = 0; i < S - 1; ++i) {
+            if (i < n) issue(i);
+            cp_async_commit();
+        }
+        for (int i = 0; i < n; ++i) {
+            cp_async_wait<S - 2>();                // task i's rows have landed
+            __syncwarp();
+            if (i + S - 1 < n) issue(i + S - 1);
+            cp_async_commit();
+            const int j = sc.order[i];
+            const int k = sc.rank[j];
+            const uint4 *wr = reinterpret_cast<const uint4 *>(wring + (k % S) * RB);
+            const uint4 *xr = reinterpret_cast<const uint4 *>(xring + (i % S) * RB);
             float h = 0.f;
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
                 float xf[8], wf[8];
-                bf16x8_to_f32(xr[v], xf);
+                bf16x8_to_f32(xr[v * 32 + lane], xf);
                 bf16x8_to_f32(wr[v * 32 + lane], wf);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) h = fmaf(xf[c], wf[c], h);
@@ -278,10 +275,6 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
                     tok_slots[(size_t)sc.tok[j] * K + slot] = make_int2(sc.exp[j], __float_as_int(p));
                 else
                     set_status(status, OMNI_DEV_BAD_SCHEDULE);
-            }
-            if (i + 1 < n) {
-#pragma unroll
-                for (int v = 0; v < VPL; ++v) xr[v] = xn[v];
             }
         }
         // drain the remaining copies before the ring is reused
