@@ -9,26 +9,22 @@
 // sigma is read as SiLU (each atomic expert has a single w_in).
 //
 // Two kernels, no atomics on y:
-//   1. group pass (expert-centric, per group as the pages have it):
-//      P_q = G_q . SiLU(X_q W_q^T) for the task pairs only (G_q is about 8%
-//      dense for 4096 tokens over 1.7M experts).  Every warp owns a
-//      contiguous share of the sorted tasks and cuts it where the group
-//      changes; it orders its tasks by expert id (a counting sort inside
-//      each group) and goes expert by expert, loading each W row once
-//      (cp.async, 16 bytes per lane, into the warp's own shared-memory ring)
-//      and using it for every token of the group that chose it.  The x rows
-//      of the tasks stream through a second ring, kStages-1 tasks ahead.  Each task's p = g * SiLU(x_t . w_e) is
-//      written with its expert id into a slot of its token.
+//   1. group pass: P_q = G_q . SiLU(X_q W_q^T) for the task pairs only (G_q is
+//      about 8% dense for 4096 tokens over 1.7M experts).  Every warp streams
+//      a contiguous share of the sorted tasks (group, token, expert order):
+//      per task the expert's W row and the token's x row go through the
+//      warp's own cp.async ring (16 bytes per lane, several tasks ahead), and
+//      p = g * SiLU(x . w) is written with the expert id into a slot of its
+//      token.  A group's experts form one contiguous block of W rows and its
+//      tasks are adjacent in the stream, so an expert used by several tokens
+//      of the group is read from HBM once and then served by L2.
 //   2. token pass: y[t] = sum over the token's slots of p * V[e], one warp
-//      per token, V rows prefetched the same way; y is written once per
-//      token.  This is O_q = P_q V_q plus the scatter-add, regrouped by
-//      token: on B200 the fp32 reductions of per-group partial rows into y
+//      per token, V rows through the same kind of ring; y is written once
+//      per token.  This is O_q = P_q V_q plus the scatter-add, regrouped by
+//      token: on B200 fp32 reductions of per-group partial rows into y
 //      (16-byte red.global.add.v4.f32, one L2 sector operation each) ran at
-//      about 3 TB/s and cost more than the HBM gather they were meant to
-//      follow, while V rows are used about 1.1 times per group at this scale.
-// A warp that shares a group with its neighbour reloads the experts common
-// to both halves (about one row per warp boundary).  No kernel here waits on
-// another warp or CTA.
+//      about 3 TB/s and cost more than the HBM gather of the rows.
+// No kernel here waits on another warp or CTA.
 #include "omni_common.cuh"
 #include "omni_internal.h"
 
@@ -45,23 +41,6 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float *f) {
 }
 
 // ---------------------------------------------------------- common parts
-constexpr int kSub = 256;                 // tasks staged per sub-range
-
-// Per-warp scratch of the group pass for one sub-range of tasks.
-struct WarpScratch {
-    int tok[kSub];
-    int exp[kSub];
-    float gate[kSub];
-    uint16_t rank[kSub];          // rank of the task's expert in the sub-range's expert list
-    uint16_t order[kSub];         // segment tasks, expert-major
-    int slot[kSub];               // the task's slot among its token's K slots
-    int start[kSub + 4];          // per expert rank: first position in order[] (+ padding)
-    int elist[kSub];              // distinct experts of the sub-range, ascending
-    uint32_t bitmap[OMNI_MAX_B / 32];
-    int word_prefix[OMNI_MAX_B / 32];
-};
-static_assert(sizeof(WarpScratch) % 16 == 0, "scratch keeps 16-byte alignment");
-
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
                  ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
@@ -82,21 +61,15 @@ __device__ __forceinline__ void row_async(uint8_t *dst, const uint16_t *src, uns
     for (int v = 0; v < VPL; ++v) cp_async16(dst + (size_t)(v * 32 + lane) * 16, s4 + v * 32 + lane);
 }
 
-template <int VPL, int STAGES, int EXTRA>
-struct WarpSmem {
-    static constexpr int kRowBytes = 512 * VPL;
-    static constexpr int kWarpBytes = STAGES * kRowBytes + EXTRA;
-    static constexpr int kFit = (227 * 1024) / kWarpBytes;
-    static constexpr int kWarps = kFit > 16 ? 16 : kFit;
-    static_assert(kWarps >= 2, "too little shared memory per warp");
-    static_assert(kWarpBytes % 16 == 0, "per-warp areas stay 16-byte aligned");
-};
+constexpr int kChunk = 32;                // tasks whose metadata a warp holds at once
 
 template <int VPL>
 struct GateCfg {
-    // tasks in flight per warp; each stage holds a W row and an x row
-    static constexpr int kStages = VPL <= 1 ? 10 : (VPL <= 2 ? 8 : (VPL <= 4 ? 6 : 4));
-    using Smem = WarpSmem<VPL, 2 * kStages, (int)sizeof(WarpScratch)>;
+    // tasks in flight per warp; a stage holds the task's W row and x row
+    static constexpr int kStages = VPL <= 1 ? 12 : (VPL <= 2 ? 8 : (VPL <= 4 ? 6 : 4));
+    static constexpr int kWarps = 4;                      // per CTA; several CTAs per SM
+    static constexpr int kRowBytes = 512 * VPL;
+    static constexpr int kSmem = kWarps * 2 * kStages * kRowBytes;
 };
 template <int VPL>
 struct CombineCfg {
@@ -107,180 +80,108 @@ struct CombineCfg {
 };
 
 // ------------------------------------------------------- 1. group pass
+// Warp gw streams the sorted tasks [gw*per_warp, (gw+1)*per_warp): for each
+// task the W row of its expert and the x row of its token go through the
+// warp's cp.async ring, kStages-1 tasks ahead; p = g * SiLU(x . w) is written
+// with the expert id into the token's slot.  Inside a group the tasks of one
+// expert are close together, so a repeated W row is normally served by L2.
 template <int VPL>
-__global__ void __launch_bounds__(32 * GateCfg<VPL>::Smem::kWarps, 1)
+__global__ void __launch_bounds__(32 * GateCfg<VPL>::kWarps)
 group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W, int L, int N,
-                  int B, int K, int M, int per_warp, const int32_t *__restrict__ task_token,
+                  int K, int M, int per_warp, const int32_t *__restrict__ task_token,
                   const int32_t *__restrict__ task_expert, const float *__restrict__ task_gate,
                   int *__restrict__ tok_count, int2 *__restrict__ tok_slots, int *status) {
     using Cfg = GateCfg<VPL>;
-    using Sm = typename Cfg::Smem;
     constexpr int D = 256 * VPL;
     constexpr int S = Cfg::kStages;
-    constexpr int RB = Sm::kRowBytes;
+    constexpr int RB = Cfg::kRowBytes;
+    static_assert(S - 1 <= kChunk, "prefetch stays within two metadata chunks");
     extern __shared__ __align__(16) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
-    uint8_t *ring = smem + (size_t)warp * Sm::kWarpBytes;          // S W rows, then S x rows
-    WarpScratch &sc = *reinterpret_cast<WarpScratch *>(ring + 2 * S * RB);
-    static_assert(Sm::kWarpBytes == 2 * S * RB + (int)sizeof(WarpScratch), "per-warp layout");
-    const int nwords = (B + 31) >> 5;
+    uint8_t *wring = smem + (size_t)warp * 2 * S * RB;
+    uint8_t *xring = wring + S * RB;
 
-    const int64_t gw = (int64_t)blockIdx.x * Sm::kWarps + warp;
+    const int64_t gw = (int64_t)blockIdx.x * Cfg::kWarps + warp;
     const int64_t a0 = gw * per_warp;
     const int64_t a1 = a0 + per_warp < M ? a0 + per_warp : M;
+    if (a0 >= a1) return;
+    const int n = (int)(a1 - a0);
 
-    for (int64_t sub = a0; sub < a1; sub += kSub) {
-        const int n = (int)(a1 - sub < kSub ? a1 - sub : kSub);
-        __syncwarp();
-        for (int j = lane; j < n; j += 32) {
-            int t = task_token[sub + j], e = task_expert[sub + j];
+    // task metadata of the current chunk of 32 tasks, one task per lane; the
+    // slot of each task is claimed here, 32 tasks per atomic round trip
+    auto load_meta = [&](int c0, int &t, int &e, float &g, int &slot) {
+        const int i = c0 + (int)lane;
+        t = 0; e = 0; g = 0.f; slot = K;
+        if (i < n) {
+            t = task_token[a0 + i];
+            e = task_expert[a0 + i];
+            g = task_gate[a0 + i];
             if (e < 0 || e >= N || t < 0 || t >= L) {
                 set_status(status, OMNI_DEV_BAD_SCHEDULE);
                 e = e < 0 || e >= N ? 0 : e;
                 t = t < 0 || t >= L ? 0 : t;
             }
-            sc.tok[j] = t;
-            sc.exp[j] = e;
-            sc.gate[j] = task_gate[sub + j];
-            // claim the task's slot now, 32 tasks per round trip
-            sc.slot[j] = atomicAdd(&tok_count[t], 1);
+            slot = atomicAdd(&tok_count[t], 1);
         }
-        __syncwarp();
-        // ---- setup for the whole sub-range: tasks sorted by expert id (the
-        // sub-range is in (group, token, expert) order, so this is a per-group
-        // counting sort on e - q*B), expert list, expert-major task order
-        for (int k = lane; k <= n; k += 32) sc.start[k] = 0;
-        __syncwarp();
-        int n_e = 0;
-        for (int js = 0; js < n;) {
-            const int q = sc.exp[js] / B;
-            int je = n;
-            for (int j0 = js + 1; j0 < n; j0 += 32) {
-                const int j = j0 + (int)lane;
-                const bool brk = j < n && sc.exp[j] / B != q;
-                const unsigned bal = __ballot_sync(0xffffffffu, brk);
-                if (bal) {
-                    je = j0 + __ffs(bal) - 1;
-                    break;
-                }
-            }
-            const int64_t ebase = (int64_t)q * B;
-            for (int w = lane; w < nwords; w += 32) sc.bitmap[w] = 0u;
-            __syncwarp();
-            for (int j = js + lane; j < je; j += 32) {
-                const int r = (int)(sc.exp[j] - ebase);
-                atomicOr(&sc.bitmap[r >> 5], 1u << (r & 31));
-            }
-            __syncwarp();
-            const uint32_t wbits = lane < (unsigned)nwords ? sc.bitmap[lane] : 0u;
-            const int cnt = __popc(wbits);
-            const int incl = warp_iscan(cnt);
-            if (lane < (unsigned)nwords) {
-                sc.word_prefix[lane] = incl - cnt;
-                uint32_t bits = wbits;
-                int pos = n_e + incl - cnt;
-                while (bits) {
-                    const int b = __ffs(bits) - 1;
-                    sc.elist[pos++] = (int)(ebase + lane * 32 + b);
-                    bits &= bits - 1;
-                }
-            }
-            __syncwarp();
-            // per task: global expert rank; per expert: task count (task order)
-            for (int j0 = js; j0 < je; j0 += 32) {
-                const int j = j0 + (int)lane;
-                const bool in = j < je;
-                int rk = 0x7fffffff;
-                if (in) {
-                    const int r = (int)(sc.exp[j] - ebase);
-                    const int wd = r >> 5;
-                    rk = n_e + sc.word_prefix[wd] + __popc(sc.bitmap[wd] & ((1u << (r & 31)) - 1u));
-                    sc.rank[j] = (uint16_t)rk;
-                }
-                const unsigned peers = __match_any_sync(0xffffffffu, rk);
-                if (in && (peers & lanemask_lt()) == 0) sc.start[rk + 1] += __popc(peers);
-                __syncwarp();
-            }
-            n_e += __shfl_sync(0xffffffffu, incl, 31);
-            js = je;
-        }
-        // exclusive scan of the counts -> start[k]
-        {
-            int carry = 0;
-            for (int k0 = 0; k0 <= n_e; k0 += 32) {
-                const int k = k0 + (int)lane;
-                const int v = k <= n_e ? sc.start[k] : 0;
-                const int inc = warp_iscan(v);
-                if (k <= n_e) sc.start[k] = carry + inc;
-                carry += __shfl_sync(0xffffffffu, inc, 31);
-            }
-        }
-        __syncwarp();
-        // place tasks expert-major, keeping task order inside an expert
-        for (int j0 = 0; j0 < n; j0 += 32) {
-            const int j = j0 + (int)lane;
-            const bool in = j < n;
-            const int rk = in ? (int)sc.rank[j] : 0x7fffffff;
-            const unsigned peers = __match_any_sync(0xffffffffu, rk);
-            int base = 0;
-            if (in) base = sc.start[rk];
-            if (in) sc.order[base + __popc(peers & lanemask_lt())] = (uint16_t)j;
-            __syncwarp();
-            if (in && (peers & lanemask_lt()) == 0) sc.start[rk] += __popc(peers);
-            __syncwarp();
-        }
-        // ---- expert-major pass over the sub-range: p for every task.
-        // Stream unit = one task: its x row (x ring slot i % S) and, for the
-        // first task of an expert, the expert's W row (W ring slot k % S).
-        // Tasks i .. i+S-1 span at most S experts, so a W slot is refilled only
-        // after every task of its previous expert has been computed.
-        uint8_t *wring = ring;
-        uint8_t *xring = ring + S * RB;
-        auto issue = [&](int i) {
-            const int j = sc.order[i];
-            const int k = sc.rank[j];
-            if (i == 0 || sc.rank[sc.order[i - 1]] != k)
-                row_async<VPL>(wring + (k % S) * RB, W + (size_t)sc.elist[k] * D, lane);
-            row_async<VPL>(xring + (i % S) * RB, x + (size_t)sc.tok[j] * D, lane);
-        };
+    };
+    int ct, ce, cs, nt, ne, ns;     // current and next chunk (token, expert, slot)
+    float cg, ng;
+    load_meta(0, ct, ce, cg, cs);
+    load_meta(kChunk, nt, ne, ng, ns);
+    // task i (ring slot i % S) whose metadata is entry rel of the current
+    // (rel < 32) or the next (32 <= rel < 64) chunk
+    auto issue = [&](int i, int rel) {
+        const bool same = rel < kChunk;
+        const int src = rel % kChunk;
+        const int t = __shfl_sync(0xffffffffu, same ? ct : nt, src);
+        const int e = __shfl_sync(0xffffffffu, same ? ce : ne, src);
+        row_async<VPL>(wring + (i % S) * RB, W + (size_t)e * D, lane);
+        row_async<VPL>(xring + (i % S) * RB, x + (size_t)t * D, lane);
+    };
 #pragma unroll 1
-        for (int i = 0; i < S - 1; ++i) {
-            if (i < n) issue(i);
-            cp_async_commit();
-        }
-        for (int i = 0; i < n; ++i) {
-            cp_async_wait<S - 2>();                // task i's rows have landed
-            __syncwarp();
-            if (i + S - 1 < n) issue(i + S - 1);
-            cp_async_commit();
-            const int j = sc.order[i];
-            const int k = sc.rank[j];
-            const uint4 *wr = reinterpret_cast<const uint4 *>(wring + (k % S) * RB);
-            const uint4 *xr = reinterpret_cast<const uint4 *>(xring + (i % S) * RB);
-            float h = 0.f;
-#pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                float xf[8], wf[8];
-                bf16x8_to_f32(xr[v * 32 + lane], xf);
-                bf16x8_to_f32(wr[v * 32 + lane], wf);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) h = fmaf(xf[c], wf[c], h);
-            }
-            h = warp_sum(h);
-            if (lane == 0) {
-                const float p = sc.gate[j] * (h / (1.f + __expf(-h)));
-                const int slot = sc.slot[j];
-                if (slot < K)
-                    tok_slots[(size_t)sc.tok[j] * K + slot] = make_int2(sc.exp[j], __float_as_int(p));
-                else
-                    set_status(status, OMNI_DEV_BAD_SCHEDULE);
-            }
-        }
-        // drain the remaining copies before the ring is reused
-        cp_async_wait<0>();
-        __syncwarp();
+    for (int i = 0; i < S - 1; ++i) {
+        if (i < n) issue(i, i);
+        cp_async_commit();
     }
+    int base = 0;                   // first task of the current chunk
+    for (int i = 0; i < n; ++i) {
+        if (i - base == kChunk) {   // move to the next chunk of metadata
+            base += kChunk;
+            ct = nt; ce = ne; cg = ng; cs = ns;
+            load_meta(base + kChunk, nt, ne, ng, ns);
+        }
+        cp_async_wait<S - 2>();     // task i's rows have landed
+        __syncwarp();
+        const int ip = i + S - 1;
+        if (ip < n) issue(ip, ip - base);
+        cp_async_commit();
+        const uint4 *wr = reinterpret_cast<const uint4 *>(wring + (i % S) * RB);
+        const uint4 *xr = reinterpret_cast<const uint4 *>(xring + (i % S) * RB);
+        float h = 0.f;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+            float xf[8], wf[8];
+            bf16x8_to_f32(xr[v * 32 + lane], xf);
+            bf16x8_to_f32(wr[v * 32 + lane], wf);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) h = fmaf(xf[c], wf[c], h);
+        }
+        h = warp_sum(h);
+        const int src = i - base;
+        const int t = __shfl_sync(0xffffffffu, ct, src);
+        const int e = __shfl_sync(0xffffffffu, ce, src);
+        const float g = __shfl_sync(0xffffffffu, cg, src);
+        const int slot = __shfl_sync(0xffffffffu, cs, src);
+        if (lane == 0) {
+            const float p = g * (h / (1.f + __expf(-h)));
+            if (slot < K)
+                tok_slots[(size_t)t * K + slot] = make_int2(e, __float_as_int(p));
+            else
+                set_status(status, OMNI_DEV_BAD_SCHEDULE);
+        }
+    }
+    cp_async_wait<0>();
 }
 
 // ------------------------------------------------------- 2. token pass
@@ -377,10 +278,8 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
                        cudaStream_t st) {
     using G = GateCfg<VPL>;
     using C = CombineCfg<VPL>;
-    constexpr int gwarps = G::Smem::kWarps;
-    constexpr int gsmem = gwarps * G::Smem::kWarpBytes;
     cudaError_t e = cudaFuncSetAttribute(group_gate_kernel<VPL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, gsmem);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(token_combine_kernel<VPL>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
@@ -388,13 +287,16 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
     const int sms = device_sm_count();
     if ((e = cudaMemsetAsync(tok_count, 0, sizeof(int) * (size_t)sz.L, st)) != cudaSuccess) return e;
     {
-        const int64_t warps = (int64_t)sms * gwarps;
+        int per_sm = (227 * 1024) / G::kSmem;
+        if (per_sm < 1) per_sm = 1;
+        if (per_sm > 8) per_sm = 8;
+        const int64_t warps = (int64_t)sms * per_sm * G::kWarps;
         int64_t per_warp = (sz.M + warps - 1) / warps;
         if (per_warp < 32) per_warp = 32;
         const int64_t needed = (sz.M + per_warp - 1) / per_warp;      // warps with work
-        const int grid = (int)((needed + gwarps - 1) / gwarps);
-        group_gate_kernel<VPL><<<grid, 32 * gwarps, gsmem, st>>>(
-            x, W, sz.L, (int)sz.N, sz.B, sz.K, (int)sz.M, (int)per_warp, tt, te, tg, tok_count,
+        const int grid = (int)((needed + G::kWarps - 1) / G::kWarps);
+        group_gate_kernel<VPL><<<grid, 32 * G::kWarps, G::kSmem, st>>>(
+            x, W, sz.L, (int)sz.N, sz.K, (int)sz.M, (int)per_warp, tt, te, tg, tok_count,
             tok_slots, status);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
