@@ -65,15 +65,16 @@ constexpr int kChunk = 32;                // tasks whose metadata a warp holds a
 
 template <int VPL>
 struct GateCfg {
-    // tasks in flight per warp; a stage holds the task's W row and x row
-    static constexpr int kStages = VPL <= 1 ? 12 : (VPL <= 2 ? 8 : (VPL <= 4 ? 6 : 4));
+    // stages per warp (a stage holds a task's W row and x row).  Measured at
+    // d = 1024: many warps with shallow rings beat few warps with deep ones.
+    static constexpr int kStages = VPL <= 2 ? 4 : (VPL <= 4 ? 3 : 2);
     static constexpr int kWarps = 4;                      // per CTA; several CTAs per SM
     static constexpr int kRowBytes = 512 * VPL;
     static constexpr int kSmem = kWarps * 2 * kStages * kRowBytes;
 };
 template <int VPL>
 struct CombineCfg {
-    static constexpr int kStages = VPL <= 2 ? 10 : (VPL <= 4 ? 8 : 5);
+    static constexpr int kStages = VPL <= 2 ? 4 : 3;
     static constexpr int kWarps = 4;                      // per CTA; several CTAs per SM
     static constexpr int kRowBytes = 512 * VPL;
     static constexpr int kSmem = kWarps * kStages * kRowBytes;
@@ -289,7 +290,7 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
     {
         int per_sm = (227 * 1024) / G::kSmem;
         if (per_sm < 1) per_sm = 1;
-        if (per_sm > 8) per_sm = 8;
+        if (per_sm > 16) per_sm = 16;
         const int64_t warps = (int64_t)sms * per_sm * G::kWarps;
         int64_t per_warp = (sz.M + warps - 1) / warps;
         if (per_warp < 32) per_warp = 32;
@@ -303,7 +304,7 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
     {
         int per_sm = (227 * 1024) / C::kSmem;
         if (per_sm < 1) per_sm = 1;
-        if (per_sm > 8) per_sm = 8;
+        if (per_sm > 16) per_sm = 16;
         int64_t grid = (int64_t)sms * per_sm;
         const int64_t need = (sz.L + C::kWarps - 1) / C::kWarps;
         if (grid > need) grid = need;
