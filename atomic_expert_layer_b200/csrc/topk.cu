@@ -9,20 +9,34 @@
 // softmax over the K selected scores.
 //
 // Kernel 1 (axis_topk): one warp per (token, axis).  Optional LogSoftmax,
-//   then an exact radix select (4 passes of 8 bits over order-preserving
-//   keys) of the axis' top min(K, n) entries, then a rank sort of those.
+//   then the axis' top min(K, n) entries.
 // Kernel 2 (merge_topk): one warp per token.  Because fp32 addition is
 //   monotone, a cell with row rank a and column rank b is dominated by every
 //   cell (a', b') with a' <= a, b' <= b, and the key above ranks a dominating
 //   cell first even on equal S; so the K best cells all satisfy
 //   (a+1)(b+1) <= K.  Those C candidates (C = sum_a min(Kc, K/(a+1))) are
-//   scored, radix-selected on S and rank-sorted by the full key.
+//   scored and the K best taken.
+//
+// Selection (both kernels, exact): values are bucketed by
+//   b(v) = floor((vmax - v) * 128)      (fp32, monotone non-increasing in v)
+// over 1024 buckets (8 units below the maximum).  Any value in a lower
+// bucket is strictly larger than any value in a higher one, so with b* the
+// bucket holding the k-th value, the top k are all values with b < b* plus
+// the best of bucket b*.  Those candidates (about k + 1 for Gaussian-like
+// rows) are sorted by the full key with a warp bitonic sort.  If fewer than k
+// values lie within 8 units of the maximum, or the candidates exceed the
+// sort's capacity, an exact radix select (4 passes of 8 bits over
+// order-preserving keys) followed by a rank sort is used instead.
 #include "omni_common.cuh"
 #include "omni_internal.h"
 
 namespace omni {
 namespace {
 
+constexpr int kNB = 1024;              // value buckets
+constexpr float kBucketScale = 128.f;  // buckets per unit
+
+// ----------------------------------------------------------- radix select
 // Exact k-th largest key of keys[0..n) (a warp, smem histogram `hist` of 256).
 // Returns the threshold key T and sets *take_eq to how many keys equal to T
 // belong to the top k (the rest of the top k is every key > T).
@@ -75,14 +89,111 @@ __device__ uint32_t warp_radix_select(const uint32_t *keys, int n, int k, uint32
     return prefix;
 }
 
+// ------------------------------------------------------------ value buckets
+__device__ __forceinline__ int bucket_of(float vmax, float v) {
+    const float dv = __fmul_rn(__fsub_rn(vmax, v), kBucketScale);
+    return dv < (float)kNB ? (int)dv : kNB;           // kNB = beyond the range
+}
+
+// Zero the histogram, count vals[0..n) (optionally through `get`) into it and
+// find the bucket b* holding the k-th largest value.  Returns the number of
+// values in buckets <= b*, or -1 if fewer than k values are in range.
+template <typename Get>
+__device__ int bucket_threshold(Get get, int n, int k, float vmax, uint32_t *hist, int *bstar) {
+    const unsigned lane = lane_id();
+    for (int b = lane; b < kNB; b += 32) hist[b] = 0u;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+        const int b = bucket_of(vmax, get(i));
+        if (b < kNB) atomicAdd(&hist[b], 1u);
+    }
+    __syncwarp();
+    // lane l owns buckets [32l, 32l + 32)
+    int tot = 0;
+    for (int j = 0; j < kNB / 32; ++j) tot += (int)hist[lane * (kNB / 32) + j];
+    const int incl = warp_iscan(tot);
+    const int excl = incl - tot;
+    const bool mine = excl < k && k <= incl;
+    const unsigned bal = __ballot_sync(0xffffffffu, mine);
+    if (bal == 0u) return -1;
+    int bs = 0, through = 0;
+    if (mine) {
+        int run = excl;
+        for (int j = 0; j < kNB / 32; ++j) {
+            run += (int)hist[lane * (kNB / 32) + j];
+            if (run >= k) {
+                bs = lane * (kNB / 32) + j;
+                through = run;
+                break;
+            }
+        }
+    }
+    const int src = __ffs(bal) - 1;
+    *bstar = __shfl_sync(0xffffffffu, bs, src);
+    return __shfl_sync(0xffffffffu, through, src);
+}
+
+// -------------------------------------------------------- warp bitonic sort
+// Sort 32*E keys held as v[i] of lane l (element id l + 32 i) in descending
+// order of (hi, lo).  With ONE_WORD only hi is compared.
+template <int E, bool ONE_WORD>
+__device__ __forceinline__ void bitonic_desc(uint64_t (&hi)[E], uint64_t (&lo)[E]) {
+    const unsigned lane = lane_id();
+#pragma unroll
+    for (int k = 2; k <= 32 * E; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j >= 32) {
+#pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    const int p = i ^ (j >> 5);
+                    if (p > i) {
+                        const bool desc = (((int)lane + 32 * i) & k) == 0;
+                        const bool gt = ONE_WORD ? hi[i] > hi[p]
+                                                 : (hi[i] > hi[p] || (hi[i] == hi[p] && lo[i] > lo[p]));
+                        if (desc != gt) {            // swap so the segment runs the right way
+                            const uint64_t th = hi[i], tl = lo[i];
+                            hi[i] = hi[p];
+                            lo[i] = lo[p];
+                            hi[p] = th;
+                            lo[p] = tl;
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    const int id = (int)lane + 32 * i;
+                    const uint64_t oh = __shfl_xor_sync(0xffffffffu, hi[i], j);
+                    const uint64_t ol = ONE_WORD ? 0ull : __shfl_xor_sync(0xffffffffu, lo[i], j);
+                    const bool low = (id & j) == 0;
+                    const bool desc = (id & k) == 0;
+                    const bool other_gt = ONE_WORD ? oh > hi[i]
+                                                   : (oh > hi[i] || (oh == hi[i] && ol > lo[i]));
+                    const bool other_lt = ONE_WORD ? oh < hi[i]
+                                                   : (oh < hi[i] || (oh == hi[i] && ol < lo[i]));
+                    // the low element keeps the larger key in a descending segment
+                    const bool take = (low == desc) ? other_gt : other_lt;
+                    if (take) {
+                        hi[i] = oh;
+                        lo[i] = ol;
+                    }
+                }
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------ axis top-K
-// Dynamic smem per warp: keys[nmax] + hist[256] + sel_key[kmax] + sel_idx[kmax].
+// Dynamic smem per warp (words): vals[nmax] | hist[kNB] | sel_key[kmax] | sel_idx[kmax]
+//                                | stage[2 * 32E] (bitonic staging, u64)
+template <int E>
 __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__restrict__ in_c,
                                  int logsoftmax, float *__restrict__ p_r_out,
                                  float *__restrict__ p_c_out, int L, int N_r, int N_c, int K,
                                  float *__restrict__ row_val, int *__restrict__ row_idx,
                                  float *__restrict__ col_val, int *__restrict__ col_idx,
-                                 int nmax, int kmax) {
+                                 int nmax, int kmax, size_t warp_words) {
     extern __shared__ __align__(16) uint32_t smem_u[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
@@ -98,37 +209,87 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     float *oval = (axis ? col_val : row_val) + (size_t)t * kx;
     int *oidx = (axis ? col_idx : row_idx) + (size_t)t * kx;
 
-    uint32_t *keys = smem_u + (size_t)warp * (nmax + 256 + 2 * kmax);
-    uint32_t *hist = keys + nmax;
-    uint32_t *sel_key = hist + 256;
+    uint32_t *base = smem_u + (size_t)warp * warp_words;
+    float *vals = reinterpret_cast<float *>(base);
+    uint32_t *hist = base + nmax;
+    uint32_t *sel_key = hist + kNB;
     int *sel_idx = reinterpret_cast<int *>(sel_key + kmax);
+    const size_t stage_off = ((size_t)nmax + kNB + 2 * (size_t)kmax + 1) & ~(size_t)1;
+    uint64_t *stage = reinterpret_cast<uint64_t *>(base + stage_off);
 
+    float vmax = -INFINITY;
     if (logsoftmax) {
         float mx = -INFINITY;
         for (int i = lane; i < n; i += 32) {
             const float v = in[i];
-            keys[i] = __float_as_uint(v);
+            vals[i] = v;
             mx = fmaxf(mx, v);
         }
         mx = warp_max(mx);
         float sum = 0.f;
-        for (int i = lane; i < n; i += 32) sum += expf(__uint_as_float(keys[i]) - mx);
+        for (int i = lane; i < n; i += 32) sum += __expf(vals[i] - mx);
         sum = warp_sum(sum);
-        const float lse = mx + logf(sum);
+        const float lse = mx + __logf(sum);
         for (int i = lane; i < n; i += 32) {
-            const float p = __uint_as_float(keys[i]) - lse;
+            const float p = vals[i] - lse;
             if (pout) pout[(size_t)t * n + i] = p;
-            keys[i] = f2key(p);
+            vals[i] = p;
         }
+        vmax = mx - lse;                   // the p of the largest logit, same rounding
     } else {
-        for (int i = lane; i < n; i += 32) keys[i] = f2key(in[i]);
+        for (int i = lane; i < n; i += 32) {
+            const float v = in[i];
+            vals[i] = v;
+            vmax = fmaxf(vmax, v);
+        }
+        vmax = warp_max(vmax);
     }
     __syncwarp();
 
+    if (E > 0) {
+        int bs = 0;
+        const int ncand =
+            bucket_threshold([&](int i) { return vals[i]; }, n, kx, vmax, hist, &bs);
+        if (ncand >= kx && ncand <= 32 * E) {
+            // candidates in index order -> 64-bit keys (key(p), ~index)
+            int taken = 0;
+            for (int i0 = 0; i0 < n; i0 += 32) {
+                const int i = i0 + (int)lane;
+                const bool in_c = i < n && bucket_of(vmax, vals[i]) <= bs;
+                const unsigned bal = __ballot_sync(0xffffffffu, in_c);
+                if (in_c) {
+                    const int pos = taken + __popc(bal & lanemask_lt());
+                    stage[pos] = ((uint64_t)f2key(vals[i]) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
+                }
+                taken += __popc(bal);
+            }
+            for (int i = taken + (int)lane; i < 32 * E; i += 32) stage[i] = 0ull;
+            __syncwarp();
+            uint64_t hi[E > 0 ? E : 1], lo[E > 0 ? E : 1];
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                hi[i] = stage[lane + 32 * i];
+                lo[i] = 0ull;
+            }
+            bitonic_desc<(E > 0 ? E : 1), true>(hi, lo);
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const int r = (int)lane + 32 * i;
+                if (r < kx) {
+                    oval[r] = key2f((uint32_t)(hi[i] >> 32));
+                    oidx[r] = (int)(0xffffffffu - (uint32_t)hi[i]);
+                }
+            }
+            return;
+        }
+    }
+
+    // ---- exact fallback: radix select on keys, rank sort
+    uint32_t *keys = reinterpret_cast<uint32_t *>(vals);
+    for (int i = lane; i < n; i += 32) keys[i] = f2key(vals[i]);
+    __syncwarp();
     int take_eq;
     const uint32_t T = warp_radix_select(keys, n, kx, hist, &take_eq);
-
-    // collect the top kx in index order: every key > T, and the first take_eq keys == T
     int taken = 0, eq_seen = 0;
     for (int i0 = 0; i0 < n; i0 += 32) {
         const int i = i0 + (int)lane;
@@ -148,7 +309,6 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
         eq_seen += __popc(beq);
     }
     __syncwarp();
-    // rank sort by (key desc, index asc); sel is in index order
     for (int u = lane; u < kx; u += 32) {
         const uint32_t ku = sel_key[u];
         int r = 0;
@@ -177,32 +337,86 @@ __device__ __forceinline__ bool better(const Cand &u, const Cand &v) {
     return u.n < v.n;
 }
 
-// Dynamic smem per warp:
-//   rv[Kr] f32, ri[Kr] i32, cv[Kc] f32, ci[Kc] i32, ckey[C] u32, cab[C] u32,
-//   hist[256] u32, q[C] Cand, out_S[K] f32, out_n[K] u32
+struct MergeLayout {   // offsets (words) inside one warp's region
+    size_t rv, ri, cv, ci, sval, cab, hist, q, out_s, out_n, words;
+};
+
+__host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C) {
+    MergeLayout m;
+    size_t o = 0;
+    m.rv = o; o += Kr;
+    m.ri = o; o += Kr;
+    m.cv = o; o += Kc;
+    m.ci = o; o += Kc;
+    m.sval = o; o += C;
+    m.cab = o; o += C;
+    m.hist = o; o += kNB;
+    o = (o + 3) & ~(size_t)3;                 // 16-byte alignment for Cand / u64
+    m.q = o; o += 4 * (size_t)C;               // Cand[C], also the bitonic staging
+    m.out_s = o; o += K;
+    m.out_n = o; o += K;
+    m.words = (o + 3) & ~(size_t)3;
+    return m;
+}
+
+// Shared by the CTA: table[c] = (a << 16) | b for the c-th candidate, a-major.
+template <int E>
 __global__ void merge_topk_kernel(const float *__restrict__ row_val,
                                   const int *__restrict__ row_idx,
                                   const float *__restrict__ col_val,
                                   const int *__restrict__ col_idx, int L, int N_c, int K, int Kr,
-                                  int Kc, int C, size_t warp_words, int32_t *__restrict__ idx,
+                                  int Kc, int C, int32_t *__restrict__ idx,
                                   float *__restrict__ score, float *__restrict__ gate) {
     extern __shared__ __align__(16) uint32_t smem_u[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
-    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+    const int wpb = blockDim.x >> 5;
+    const MergeLayout ml = merge_layout(K, Kr, Kc, C);
+    uint32_t *table = smem_u;                                   // C entries
+    int *off = reinterpret_cast<int *>(table + C);               // Kr + 1 entries
+    const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
+
+    // ---- candidate table (once per CTA): off[a] = sum_{a' < a} nb(a')
+    if (warp == 0) {
+        int carry = 0;
+        for (int a0 = 0; a0 < Kr; a0 += 32) {
+            const int a = a0 + (int)lane;
+            int nb = 0;
+            if (a < Kr) {
+                nb = K / (a + 1);
+                if (nb > Kc) nb = Kc;
+            }
+            const int inc = warp_iscan(nb);
+            if (a < Kr) off[a] = carry + inc - nb;
+            carry += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) off[Kr] = carry;
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        int lo = 0, hi = Kr - 1;                 // last a with off[a] <= c
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (off[mid] <= c) lo = mid; else hi = mid - 1;
+        }
+        table[c] = ((uint32_t)lo << 16) | (uint32_t)(c - off[lo]);
+    }
+    __syncthreads();
+
+    const int t = blockIdx.x * wpb + warp;
     if (t >= L) return;
-    uint32_t *base = smem_u + (size_t)warp * warp_words;
-    float *rv = reinterpret_cast<float *>(base);
-    uint32_t *ri = base + Kr;
-    float *cv = reinterpret_cast<float *>(ri + Kr);
-    uint32_t *ci = reinterpret_cast<uint32_t *>(cv + Kc);
-    uint32_t *ckey = ci + Kc;
-    uint32_t *cab = ckey + C;
-    uint32_t *hist = cab + C;
-    const size_t q_off = ((size_t)(2 * Kr + 2 * Kc + 2 * C + 256) + 3) & ~(size_t)3;
-    Cand *q = reinterpret_cast<Cand *>(base + q_off);
-    float *out_S = reinterpret_cast<float *>(q + C);
-    uint32_t *out_n = reinterpret_cast<uint32_t *>(out_S + K);
+    uint32_t *base = smem_u + head + (size_t)warp * ml.words;
+    float *rv = reinterpret_cast<float *>(base + ml.rv);
+    uint32_t *ri = base + ml.ri;
+    float *cv = reinterpret_cast<float *>(base + ml.cv);
+    uint32_t *ci = base + ml.ci;
+    float *sval = reinterpret_cast<float *>(base + ml.sval);
+    uint32_t *cab = base + ml.cab;
+    uint32_t *hist = base + ml.hist;
+    Cand *q = reinterpret_cast<Cand *>(base + ml.q);
+    uint64_t *stage = reinterpret_cast<uint64_t *>(base + ml.q);
+    float *out_S = reinterpret_cast<float *>(base + ml.out_s);
+    uint32_t *out_n = base + ml.out_n;
 
     for (int a = lane; a < Kr; a += 32) {
         rv[a] = row_val[(size_t)t * Kr + a];
@@ -213,67 +427,116 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
         ci[b] = (uint32_t)col_idx[(size_t)t * Kc + b];
     }
     __syncwarp();
-    // candidate block: a-major, b < min(Kc, K / (a+1))
-    int off = 0;
-    for (int a = 0; a < Kr; ++a) {
-        int nb = K / (a + 1);
-        if (nb > Kc) nb = Kc;
-        if (nb <= 0) break;
-        const float pr = rv[a];
-        for (int b = lane; b < nb; b += 32) {
-            const float S = __fadd_rn(pr, cv[b]);
-            ckey[off + b] = f2key(S);
-            cab[off + b] = ((uint32_t)a << 16) | (uint32_t)b;
-        }
-        off += nb;
+    for (int c = lane; c < C; c += 32) {
+        const uint32_t ab = table[c];
+        sval[c] = __fadd_rn(rv[ab >> 16], cv[ab & 0xffffu]);
     }
+    const float smax = __fadd_rn(rv[0], cv[0]);           // cell (0, 0) is the largest
     __syncwarp();
 
-    int take_eq;
-    const uint32_t T = warp_radix_select(ckey, C, K, hist, &take_eq);
-
-    // Q = all candidates with key(S) >= T, in candidate order
-    int nq = 0;
-    for (int c0 = 0; c0 < C; c0 += 32) {
-        const int c = c0 + (int)lane;
-        const bool in = c < C && ckey[c] >= T;
-        const unsigned bal = __ballot_sync(0xffffffffu, in);
-        if (in) {
-            const int pos = nq + __popc(bal & lanemask_lt());
-            const uint32_t ab = cab[c];
-            const int a = (int)(ab >> 16), b = (int)(ab & 0xffffu);
-            Cand cd;
-            cd.skey = ckey[c];
-            cd.prkey = f2key(rv[a]);
-            cd.pckey = f2key(cv[b]);
-            cd.n = ri[a] * (uint32_t)N_c + ci[b];
-            q[pos] = cd;
+    bool done = false;
+    if (E > 0) {
+        int bs = 0;
+        const int ncand =
+            bucket_threshold([&](int c) { return sval[c]; }, C, K, smax, hist, &bs);
+        if (ncand >= K && ncand <= 32 * E) {
+            int taken = 0;
+            for (int c0 = 0; c0 < C; c0 += 32) {
+                const int c = c0 + (int)lane;
+                const bool in_c = c < C && bucket_of(smax, sval[c]) <= bs;
+                const unsigned bal = __ballot_sync(0xffffffffu, in_c);
+                if (in_c) {
+                    const int pos = taken + __popc(bal & lanemask_lt());
+                    const uint32_t ab = table[c];
+                    const int a = (int)(ab >> 16), b = (int)(ab & 0xffffu);
+                    const uint32_t nn = ri[a] * (uint32_t)N_c + ci[b];
+                    stage[2 * pos] = ((uint64_t)f2key(sval[c]) << 32) | f2key(rv[a]);
+                    stage[2 * pos + 1] = ((uint64_t)f2key(cv[b]) << 32) | (uint64_t)(0xffffffffu - nn);
+                }
+                taken += __popc(bal);
+            }
+            for (int i = taken + (int)lane; i < 32 * E; i += 32) {
+                stage[2 * i] = 0ull;
+                stage[2 * i + 1] = 0ull;
+            }
+            __syncwarp();
+            uint64_t hi[E > 0 ? E : 1], lo[E > 0 ? E : 1];
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                hi[i] = stage[2 * (lane + 32 * i)];
+                lo[i] = stage[2 * (lane + 32 * i) + 1];
+            }
+            bitonic_desc<(E > 0 ? E : 1), false>(hi, lo);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const int r = (int)lane + 32 * i;
+                if (r < K) {
+                    out_S[r] = key2f((uint32_t)(hi[i] >> 32));
+                    out_n[r] = 0xffffffffu - (uint32_t)lo[i];
+                }
+            }
+            done = true;
         }
-        nq += __popc(bal);
     }
-    __syncwarp();
-    // rank by the full key; the K best go to out[rank]
-    for (int u = lane; u < nq; u += 32) {
-        const Cand cu = q[u];
-        int r = 0;
-        for (int v = 0; v < nq; ++v) r += better(q[v], cu) ? 1 : 0;
-        if (r < K) {
-            out_S[r] = key2f(cu.skey);
-            out_n[r] = cu.n;
+    if (!done) {
+        // ---- exact fallback: radix select on key(S), rank sort by the full key
+        uint32_t *ckey = reinterpret_cast<uint32_t *>(sval);
+        for (int c = lane; c < C; c += 32) {
+            ckey[c] = f2key(sval[c]);
+            cab[c] = table[c];
+        }
+        __syncwarp();
+        int take_eq;
+        const uint32_t T = warp_radix_select(ckey, C, K, hist, &take_eq);
+        int nq = 0;
+        for (int c0 = 0; c0 < C; c0 += 32) {
+            const int c = c0 + (int)lane;
+            const bool in_q = c < C && ckey[c] >= T;
+            const unsigned bal = __ballot_sync(0xffffffffu, in_q);
+            if (in_q) {
+                const int pos = nq + __popc(bal & lanemask_lt());
+                const uint32_t ab = cab[c];
+                const int a = (int)(ab >> 16), b = (int)(ab & 0xffffu);
+                Cand cd;
+                cd.skey = ckey[c];
+                cd.prkey = f2key(rv[a]);
+                cd.pckey = f2key(cv[b]);
+                cd.n = ri[a] * (uint32_t)N_c + ci[b];
+                q[pos] = cd;
+            }
+            nq += __popc(bal);
+        }
+        __syncwarp();
+        for (int u = lane; u < nq; u += 32) {
+            const Cand cu = q[u];
+            int r = 0;
+            for (int v = 0; v < nq; ++v) r += better(q[v], cu) ? 1 : 0;
+            if (r < K) {
+                out_S[r] = key2f(cu.skey);
+                out_n[r] = cu.n;
+            }
         }
     }
     __syncwarp();
     // gates: softmax over the K selected S (S sorted, out_S[0] is the max)
-    const float smax = out_S[0];
+    const float smx = out_S[0];
     float part = 0.f;
-    for (int k = lane; k < K; k += 32) part += expf(out_S[k] - smax);
+    for (int k = lane; k < K; k += 32) part += expf(out_S[k] - smx);
     const float den = warp_sum(part);
     for (int k = lane; k < K; k += 32) {
         const float S = out_S[k];
         idx[(size_t)t * K + k] = (int32_t)out_n[k];
         score[(size_t)t * K + k] = S;
-        gate[(size_t)t * K + k] = expf(S - smax) / den;
+        gate[(size_t)t * K + k] = expf(S - smx) / den;
     }
+}
+
+int sort_capacity(int k) {
+    // warp bitonic capacity 32*E with room for the boundary bucket; 0 = none
+    int e = 1;
+    while (32 * e < k + 16) e <<= 1;
+    return e <= 8 ? e : 0;
 }
 
 }  // namespace
@@ -289,40 +552,14 @@ int merge_candidates(int K, int Kr, int Kc) {
     return C;
 }
 
-cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftmax,
-                             float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
-                             float *row_val, int *row_idx, float *col_val, int *col_idx,
-                             int *status, cudaStream_t st) {
-    (void)status;
+template <int E>
+static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logsoftmax,
+                                 float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
+                                 float *row_val, int *row_idx, float *col_val, int *col_idx,
+                                 cudaStream_t st) {
     const int nmax = N_r > N_c ? N_r : N_c;
     const int kmax = K < nmax ? K : nmax;
-    const size_t per_warp = (size_t)(nmax + 256 + 2 * kmax) * 4;
-    int wpb = (int)((96 * 1024) / per_warp);
-    if (wpb > 8) wpb = 8;
-    if (wpb < 1) wpb = 1;
-    const size_t smem = per_warp * wpb;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(axis_topk_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    const int64_t probs = 2 * (int64_t)L;
-    const unsigned grid = (unsigned)((probs + wpb - 1) / wpb);
-    axis_topk_kernel<<<grid, 32 * wpb, smem, st>>>(in_r, in_c, logsoftmax ? 1 : 0, p_r_out,
-                                                   p_c_out, L, N_r, N_c, K, row_val, row_idx,
-                                                   col_val, col_idx, nmax, kmax);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
-                              const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
-                              int32_t *idx, float *score, float *gate, cudaStream_t st) {
-    // words per warp: rv, ri (Kr each), cv, ci (Kc each), ckey, cab (C each),
-    // hist 256, q (4 words per cand), out_S, out_n (K each); pad to 4 words
-    size_t words = 2 * (size_t)Kr + 2 * (size_t)Kc + 2 * (size_t)C + 256;
-    words = (words + 3) & ~(size_t)3;                 // 16-byte alignment for Cand
-    words += 4 * (size_t)C + 2 * (size_t)K;
+    size_t words = (((size_t)nmax + kNB + 2 * (size_t)kmax + 1) & ~(size_t)1) + 2 * 32 * (size_t)(E > 0 ? E : 0);
     words = (words + 3) & ~(size_t)3;
     const size_t per_warp = words * 4;
     int wpb = (int)((96 * 1024) / per_warp);
@@ -330,15 +567,69 @@ cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const fl
     if (wpb < 1) wpb = 1;
     const size_t smem = per_warp * wpb;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel,
+        cudaError_t e = cudaFuncSetAttribute(axis_topk_kernel<E>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t probs = 2 * (int64_t)L;
+    const unsigned grid = (unsigned)((probs + wpb - 1) / wpb);
+    axis_topk_kernel<E><<<grid, 32 * wpb, smem, st>>>(in_r, in_c, logsoftmax ? 1 : 0, p_r_out,
+                                                      p_c_out, L, N_r, N_c, K, row_val, row_idx,
+                                                      col_val, col_idx, nmax, kmax, words);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftmax,
+                             float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
+                             float *row_val, int *row_idx, float *col_val, int *col_idx,
+                             int *status, cudaStream_t st) {
+    (void)status;
+    const int nmax = N_r > N_c ? N_r : N_c;
+    const int kmax = K < nmax ? K : nmax;
+    switch (sort_capacity(kmax)) {
+#define OMNI_AX(e) case e: return launch_axis_e<e>(in_r, in_c, logsoftmax, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
+        OMNI_AX(1) OMNI_AX(2) OMNI_AX(4) OMNI_AX(8)
+        default: OMNI_AX(0)
+#undef OMNI_AX
+    }
+}
+
+template <int E>
+static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, const float *col_val,
+                                  const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
+                                  int32_t *idx, float *score, float *gate, cudaStream_t st) {
+    const MergeLayout ml = merge_layout(K, Kr, Kc, C);
+    const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
+    const size_t per_warp = ml.words * 4;
+    int wpb = (int)((96 * 1024 - head * 4) / per_warp);
+    if (wpb > 8) wpb = 8;
+    if (wpb < 1) wpb = 1;
+    const size_t smem = head * 4 + per_warp * wpb;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel<E>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
     }
     const unsigned grid = (unsigned)((L + wpb - 1) / wpb);
-    merge_topk_kernel<<<grid, 32 * wpb, smem, st>>>(row_val, row_idx, col_val, col_idx, L, N_c, K,
-                                                    Kr, Kc, C, words, idx, score, gate);
+    merge_topk_kernel<E><<<grid, 32 * wpb, smem, st>>>(row_val, row_idx, col_val, col_idx, L, N_c,
+                                                       K, Kr, Kc, C, idx, score, gate);
     return cudaGetLastError();
+}
+
+cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
+                              const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
+                              int32_t *idx, float *score, float *gate, cudaStream_t st) {
+    // the bitonic staging lives in the Cand area (4 words per candidate)
+    int e = sort_capacity(K);
+    if (e > 0 && 32 * e > C) e = 0;
+    switch (e) {
+#define OMNI_MG(e) case e: return launch_merge_e<e>(row_val, row_idx, col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, st);
+        OMNI_MG(1) OMNI_MG(2) OMNI_MG(4) OMNI_MG(8)
+        default: OMNI_MG(0)
+#undef OMNI_MG
+    }
 }
 
 }  // namespace omni
