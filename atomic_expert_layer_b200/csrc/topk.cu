@@ -18,8 +18,8 @@
 //   scored and the K best taken.
 //
 // Selection (both kernels, exact): values are bucketed by
-//   b(v) = floor((vmax - v) * 128)      (fp32, monotone non-increasing in v)
-// over 1024 buckets (8 units below the maximum).  Any value in a lower
+//   b(v) = floor((vmax - v) * 32)       (fp32, monotone non-increasing in v)
+// over 256 buckets (8 units below the maximum).  Any value in a lower
 // bucket is strictly larger than any value in a higher one, so with b* the
 // bucket holding the k-th value, the top k are all values with b < b* plus
 // the best of bucket b*.  Those candidates (about k + 1 for Gaussian-like
@@ -33,8 +33,8 @@
 namespace omni {
 namespace {
 
-constexpr int kNB = 1024;              // value buckets
-constexpr float kBucketScale = 128.f;  // buckets per unit
+constexpr int kNB = 256;               // value buckets (also the radix histogram)
+constexpr float kBucketScale = 32.f;   // buckets per unit: 8 units below the maximum
 
 // ----------------------------------------------------------- radix select
 // Exact k-th largest key of keys[0..n) (a warp, smem histogram `hist` of 256).
@@ -108,7 +108,7 @@ __device__ int bucket_threshold(Get get, int n, int k, float vmax, uint32_t *his
         if (b < kNB) atomicAdd(&hist[b], 1u);
     }
     __syncwarp();
-    // lane l owns buckets [32l, 32l + 32)
+    // lane l owns buckets [l * kNB/32, (l + 1) * kNB/32)
     int tot = 0;
     for (int j = 0; j < kNB / 32; ++j) tot += (int)hist[lane * (kNB / 32) + j];
     const int incl = warp_iscan(tot);
@@ -185,8 +185,8 @@ __device__ __forceinline__ void bitonic_desc(uint64_t (&hi)[E], uint64_t (&lo)[E
 }
 
 // ------------------------------------------------------------ axis top-K
-// Dynamic smem per warp (words): vals[nmax] | hist[kNB] | sel_key[kmax] | sel_idx[kmax]
-//                                | stage[2 * 32E] (bitonic staging, u64)
+// Dynamic smem per warp (words): vals[nmax] | hist[kNB] | area[max(2 kmax, 64 E)], where
+// area is either sel_key[kmax] + sel_idx[kmax] (fallback) or the bitonic staging (u64)
 template <int E>
 __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__restrict__ in_c,
                                  int logsoftmax, float *__restrict__ p_r_out,
@@ -212,10 +212,10 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     uint32_t *base = smem_u + (size_t)warp * warp_words;
     float *vals = reinterpret_cast<float *>(base);
     uint32_t *hist = base + nmax;
-    uint32_t *sel_key = hist + kNB;
+    const size_t area_off = ((size_t)nmax + kNB + 1) & ~(size_t)1;      // 8-byte aligned
+    uint32_t *sel_key = base + area_off;
     int *sel_idx = reinterpret_cast<int *>(sel_key + kmax);
-    const size_t stage_off = ((size_t)nmax + kNB + 2 * (size_t)kmax + 1) & ~(size_t)1;
-    uint64_t *stage = reinterpret_cast<uint64_t *>(base + stage_off);
+    uint64_t *stage = reinterpret_cast<uint64_t *>(base + area_off);
 
     float vmax = -INFINITY;
     if (logsoftmax) {
@@ -338,7 +338,7 @@ __device__ __forceinline__ bool better(const Cand &u, const Cand &v) {
 }
 
 struct MergeLayout {   // offsets (words) inside one warp's region
-    size_t rv, ri, cv, ci, sval, cab, hist, q, out_s, out_n, words;
+    size_t rv, ri, cv, ci, sval, hist, q, out_s, out_n, words;
 };
 
 __host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C) {
@@ -349,7 +349,6 @@ __host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C
     m.cv = o; o += Kc;
     m.ci = o; o += Kc;
     m.sval = o; o += C;
-    m.cab = o; o += C;
     m.hist = o; o += kNB;
     o = (o + 3) & ~(size_t)3;                 // 16-byte alignment for Cand / u64
     m.q = o; o += 4 * (size_t)C;               // Cand[C], also the bitonic staging
@@ -411,7 +410,6 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     float *cv = reinterpret_cast<float *>(base + ml.cv);
     uint32_t *ci = base + ml.ci;
     float *sval = reinterpret_cast<float *>(base + ml.sval);
-    uint32_t *cab = base + ml.cab;
     uint32_t *hist = base + ml.hist;
     Cand *q = reinterpret_cast<Cand *>(base + ml.q);
     uint64_t *stage = reinterpret_cast<uint64_t *>(base + ml.q);
@@ -482,10 +480,7 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     if (!done) {
         // ---- exact fallback: radix select on key(S), rank sort by the full key
         uint32_t *ckey = reinterpret_cast<uint32_t *>(sval);
-        for (int c = lane; c < C; c += 32) {
-            ckey[c] = f2key(sval[c]);
-            cab[c] = table[c];
-        }
+        for (int c = lane; c < C; c += 32) ckey[c] = f2key(sval[c]);
         __syncwarp();
         int take_eq;
         const uint32_t T = warp_radix_select(ckey, C, K, hist, &take_eq);
@@ -496,7 +491,7 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
             const unsigned bal = __ballot_sync(0xffffffffu, in_q);
             if (in_q) {
                 const int pos = nq + __popc(bal & lanemask_lt());
-                const uint32_t ab = cab[c];
+                const uint32_t ab = table[c];
                 const int a = (int)(ab >> 16), b = (int)(ab & 0xffffu);
                 Cand cd;
                 cd.skey = ckey[c];
@@ -559,10 +554,11 @@ static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logs
                                  cudaStream_t st) {
     const int nmax = N_r > N_c ? N_r : N_c;
     const int kmax = K < nmax ? K : nmax;
-    size_t words = (((size_t)nmax + kNB + 2 * (size_t)kmax + 1) & ~(size_t)1) + 2 * 32 * (size_t)(E > 0 ? E : 0);
+    const size_t area = 2 * (size_t)kmax > 64 * (size_t)E ? 2 * (size_t)kmax : 64 * (size_t)E;
+    size_t words = (((size_t)nmax + kNB + 1) & ~(size_t)1) + area;
     words = (words + 3) & ~(size_t)3;
     const size_t per_warp = words * 4;
-    int wpb = (int)((96 * 1024) / per_warp);
+    int wpb = (int)((64 * 1024) / per_warp);
     if (wpb > 8) wpb = 8;
     if (wpb < 1) wpb = 1;
     const size_t smem = per_warp * wpb;
@@ -602,7 +598,7 @@ static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, cons
     const MergeLayout ml = merge_layout(K, Kr, Kc, C);
     const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
     const size_t per_warp = ml.words * 4;
-    int wpb = (int)((96 * 1024 - head * 4) / per_warp);
+    int wpb = (int)((64 * 1024 - head * 4) / per_warp);
     if (wpb > 8) wpb = 8;
     if (wpb < 1) wpb = 1;
     const size_t smem = head * 4 + per_warp * wpb;
