@@ -56,6 +56,8 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
     if (regions & kRegRouter) {
         w.s_r = take(4 * L * sz.N_r);
         w.s_c = take(4 * L * sz.N_c);
+        w.part_r = take(8 * L * (size_t)((sz.N_r + kGemmTileN - 1) / kGemmTileN));
+        w.part_c = take(8 * L * (size_t)((sz.N_c + kGemmTileN - 1) / kGemmTileN));
         w.row_val = take(4 * L * sz.Kr);
         w.row_idx = take(4 * L * sz.Kr);
         w.col_val = take(4 * L * sz.Kc);
@@ -137,14 +139,16 @@ int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c
     int *row_idx = ws_at<int>(ws, lay.row_idx), *col_idx = ws_at<int>(ws, lay.col_idx);
     cudaError_t e;
     if (flags & OMNI_ROUTER_LOGPROBS_IN) {
-        e = launch_axis_topk(p_r, p_c, false, nullptr, nullptr, sz.L, sz.N_r, sz.N_c, sz.K,
-                             row_val, row_idx, col_val, col_idx, status, st);
+        e = launch_axis_topk(p_r, p_c, false, nullptr, nullptr, nullptr, nullptr, sz.L, sz.N_r,
+                             sz.N_c, sz.K, row_val, row_idx, col_val, col_idx, status, st);
     } else {
         float *s_r = ws_at<float>(ws, lay.s_r), *s_c = ws_at<float>(ws, lay.s_c);
-        e = launch_router_gemm(x, W_r, W_c, sz.L, sz.d, sz.N_r, sz.N_c, s_r, s_c, status, st);
+        float *part_r = ws_at<float>(ws, lay.part_r), *part_c = ws_at<float>(ws, lay.part_c);
+        e = launch_router_gemm(x, W_r, W_c, sz.L, sz.d, sz.N_r, sz.N_c, s_r, s_c, part_r, part_c,
+                               status, st);
         if (e != cudaSuccess) return OMNI_ERR_CUDA;
-        e = launch_axis_topk(s_r, s_c, true, p_r, p_c, sz.L, sz.N_r, sz.N_c, sz.K, row_val,
-                             row_idx, col_val, col_idx, status, st);
+        e = launch_axis_topk(s_r, s_c, true, part_r, part_c, p_r, p_c, sz.L, sz.N_r, sz.N_c,
+                             sz.K, row_val, row_idx, col_val, col_idx, status, st);
     }
     if (e != cudaSuccess) return OMNI_ERR_CUDA;
     e = launch_merge_topk(row_val, row_idx, col_val, col_idx, sz.L, sz.N_c, sz.K, sz.Kr, sz.Kc,

@@ -20,7 +20,7 @@ struct Sizes {
 };
 
 struct WsLayout {
-    size_t hdr, s_r, s_c, row_val, row_idx, col_val, col_idx, idx, score, gate;
+    size_t hdr, s_r, s_c, part_r, part_c, row_val, row_idx, col_val, col_idx, idx, score, gate;
     size_t a_tok, a_exp, a_gate, b_tok, b_exp, b_gate, t_tok, t_exp, t_gate;
     size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, tok_count, tok_slots;
     size_t total;
@@ -47,12 +47,18 @@ inline T *ws_at(void *ws, size_t off) {
 }
 
 // ---- router GEMM (tcgen05): s_r = x W_r^T, s_c = x W_c^T (fp32)
+// part_r [L, ceil(N_r/128)] and part_c: per (token, 128-column tile) the max
+// of s and the sum of exp(s - max), as float pairs.
 cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c,
                                int L, int d, int N_r, int N_c, float *s_r, float *s_c,
-                               int *status, cudaStream_t st);
+                               float *part_r, float *part_c, int *status, cudaStream_t st);
+constexpr int kGemmTileN = 128;
 
 // ---- per-axis LogSoftmax (optional) + top-K; then grid merge + gates
+// With part_r / part_c (from the router GEMM) the LogSoftmax uses the
+// per-tile partials; without them it computes max and sum itself.
 cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftmax,
+                             const float *part_r, const float *part_c,
                              float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
                              float *row_val, int *row_idx, float *col_val, int *col_idx,
                              int *status, cudaStream_t st);

@@ -6,14 +6,17 @@
 // two d x sqrt(N) projections instead of one d x N.  W_r / W_c are stored as
 // N_r / N_c rows of d, so both operands are K-major.
 //
-// One launch computes both: CTA (n-tile, m-tile) with n-tiles of W_r first,
-// then those of W_c.  Tile 128 x 128, K step 64 (one 128-byte swizzle atom of
-// bf16), 3-stage TMA -> shared memory pipeline (tile loads, no multicast),
-// tcgen05.mma kind::f16 (bf16 in, fp32 accumulate) issued by one thread into
-// a 128-column TMEM accumulator, tcgen05.ld epilogue by 4 warps (one TMEM lane
-// quarter each) writing fp32 s rows.  Ragged edges (L, N_r, N_c, d not
-// multiples of the tile) read as zeros through TMA out-of-bounds fill and are
-// masked on store.
+// One persistent launch computes both.  Tiles are 128 x 128 (n-tiles of W_r
+// first, then those of W_c), K step 64 (one 128-byte swizzle atom of bf16).
+// Warp roles: warp 0 issues TMA tile loads (no multicast) into a 6-stage
+// shared-memory ring; warp 1 issues tcgen05.mma kind::f16 (bf16 in, fp32
+// accumulate) into one of two 128-column TMEM accumulators; warps 2-5 drain
+// the other accumulator with tcgen05.ld (one TMEM lane quarter each), write
+// the fp32 logits and, per (token, tile), the maximum and the sum of
+// exp(s - max) over the tile's columns -- the LogSoftmax partials -- so the
+// epilogue of one tile overlaps the main loop of the next.  Ragged edges (L,
+// N_r, N_c, d not multiples of the tile) read as zeros through TMA
+// out-of-bounds fill and are masked on store.
 #include <cuda.h>
 
 #include "omni_common.cuh"
@@ -22,17 +25,19 @@
 namespace omni {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 64, STAGES = 3;
+constexpr int BM = 128, BN = 128, BK = 64, STAGES = 6;
 constexpr int kTileBytesA = BM * BK * 2;     // 16 KB
 constexpr int kTileBytesB = BN * BK * 2;     // 16 KB
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemCols = 2 * BN;       // two fp32 accumulators
+constexpr int kThreads = 192;                // producer, MMA, 4 epilogue warps
 
 struct __align__(1024) GemmSmem {
     uint8_t a[STAGES][kTileBytesA];
     uint8_t b[STAGES][kTileBytesB];
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    uint64_t accum;
+    uint64_t tfull[2];                       // accumulator ready for the epilogue
+    uint64_t tempty[2];                      // accumulator drained
     uint32_t tmem_base;
     int abort;
 };
@@ -104,31 +109,32 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_wr,
                    const __grid_constant__ CUtensorMap tm_wc, float *__restrict__ s_r,
-                   float *__restrict__ s_c, int L, int d, int N_r, int N_c, int ntile_r,
-                   int *status) {
+                   float *__restrict__ s_c, float2 *__restrict__ part_r,
+                   float2 *__restrict__ part_c, int L, int d, int N_r, int N_c, int ntile_r,
+                   int ntile_c, int *status) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment of the tiles is required by the swizzled layout
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     GemmSmem &sm = *reinterpret_cast<GemmSmem *>(smem_raw + pad);
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
-    const bool col_axis = (int)blockIdx.x >= ntile_r;
-    const int n0 = (col_axis ? (int)blockIdx.x - ntile_r : (int)blockIdx.x) * BN;
-    const int m0 = (int)blockIdx.y * BM;
-    const int n_axis = col_axis ? N_c : N_r;
-    const CUtensorMap *tm_b = col_axis ? &tm_wc : &tm_wr;
     const int nk = (d + BK - 1) / BK;
+    const int nnt = ntile_r + ntile_c;
+    const int ntiles = ((L + BM - 1) / BM) * nnt;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        mbar_init(&sm.accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.tfull[b], 1);
+            mbar_init(&sm.tempty[b], 4);
+        }
         sm.abort = 0;
         fence_barrier_init();
     }
@@ -142,76 +148,133 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0 && lane == 0) {
-        // TMA producer
-        int issued = 0;
-        for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % STAGES;
-            if (kb >= STAGES &&
-                !mbar_wait(&sm.empty[s], (uint32_t)(((kb / STAGES) - 1) & 1), status)) {
-                sm.abort = 1;
-                break;
-            }
-            mbar_arrive_expect_tx(&sm.full[s], kTileBytesA + kTileBytesB);
-            tma_load_2d(sm.a[s], &tm_x, kb * BK, m0, &sm.full[s]);
-            tma_load_2d(sm.b[s], tm_b, kb * BK, n0, &sm.full[s]);
-            ++issued;
-        }
-        if (sm.abort) {
-            // let the loads already issued land before the CTA can exit
-            const int first = issued > STAGES ? issued - STAGES : 0;
-            for (int kb = first; kb < issued; ++kb)
-                mbar_wait(&sm.full[kb % STAGES], (uint32_t)((kb / STAGES) & 1), status);
-        }
-    } else if (warp == 1 && lane == 0) {
-        // MMA issuer
-        bool ok = true;
-        for (int kb = 0; kb < nk && ok; ++kb) {
-            const int s = kb % STAGES;
-            if (!mbar_wait(&sm.full[s], (uint32_t)((kb / STAGES) & 1), status)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint64_t ad = sw128_desc(sm.a[s]);
-            const uint64_t bd = sw128_desc(sm.b[s]);
-#pragma unroll
-            for (int k = 0; k < BK / 16; ++k) {
-                // advance 16 bf16 = 32 bytes along K inside the swizzle atom
-                umma_bf16(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k),
-                          (kb > 0 || k > 0) ? 1u : 0u);
-            }
-            umma_commit(&sm.empty[s]);
-        }
-        if (!ok) sm.abort = 1;
-        umma_commit(&sm.accum);      // arrives once every issued MMA has finished
-    }
-    __syncwarp();
-
-    // epilogue: warp w owns accumulator rows 32w..32w+31 (TMEM lanes)
-    const bool acc_ok = mbar_wait(&sm.accum, 0u, status);
-    tc_fence_after();
-    if (acc_ok && !*(volatile int *)&sm.abort) {
-        const int row = m0 + warp * 32 + (int)lane;
-        float *out = (col_axis ? s_c : s_r) + (size_t)row * n_axis;
-        const bool vec = (n_axis & 3) == 0;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, r);
-            if (row < L) {
-                const int col = n0 + c0;
-                if (vec && col + 32 <= n_axis) {
-                    float4 *o4 = reinterpret_cast<float4 *>(out + col);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        o4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                            __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (col + j < n_axis) out[col + j] = __uint_as_float(r[j]);
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- TMA producer
+            int it = 0, issued_from = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !sm.abort; tile += gridDim.x) {
+                const int m0 = (tile / nnt) * BM;
+                const int nt = tile % nnt;
+                const bool col_axis = nt >= ntile_r;
+                const int n0 = (col_axis ? nt - ntile_r : nt) * BN;
+                const CUtensorMap *tm_b = col_axis ? &tm_wc : &tm_wr;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (it >= STAGES &&
+                        !mbar_wait(&sm.empty[s], (uint32_t)(((it / STAGES) - 1) & 1), status)) {
+                        sm.abort = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sm.full[s], kTileBytesA + kTileBytesB);
+                    tma_load_2d(sm.a[s], &tm_x, kb * BK, m0, &sm.full[s]);
+                    tma_load_2d(sm.b[s], tm_b, kb * BK, n0, &sm.full[s]);
+                    issued_from = it + 1 > STAGES ? it + 1 - STAGES : 0;
                 }
+            }
+            if (sm.abort) {
+                // let the loads already issued land before the CTA can exit
+                for (int k = issued_from; k < it; ++k)
+                    mbar_wait(&sm.full[k % STAGES], (uint32_t)((k / STAGES) & 1), status);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---- MMA issuer
+            int it = 0, lt = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                if (lt >= 2 && !mbar_wait(&sm.tempty[buf], (uint32_t)(((lt >> 1) - 1) & 1), status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t acc = tmem + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&sm.full[s], (uint32_t)((it / STAGES) & 1), status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(sm.a[s]);
+                    const uint64_t bd = sw128_desc(sm.b[s]);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        // advance 16 bf16 = 32 bytes along K inside the swizzle atom
+                        umma_bf16(acc, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k),
+                                  (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&sm.empty[s]);
+                }
+                umma_commit(&sm.tfull[buf]);      // arrives once this tile's MMAs are done
+            }
+            if (!ok) sm.abort = 1;
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (accumulator rows)
+        const int quarter = warp & 3;
+        int lt = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+            const int buf = lt & 1;
+            if (!mbar_wait(&sm.tfull[buf], (uint32_t)((lt >> 1) & 1), status)) break;
+            tc_fence_after();
+            const int m0 = (tile / nnt) * BM;
+            const int nt = tile % nnt;
+            const bool col_axis = nt >= ntile_r;
+            const int tn = col_axis ? nt - ntile_r : nt;
+            const int n0 = tn * BN;
+            const int n_axis = col_axis ? N_c : N_r;
+            const int row = m0 + quarter * 32 + (int)lane;
+            float *out = (col_axis ? s_c : s_r) + (size_t)row * n_axis;
+            const bool vec = (n_axis & 3) == 0;
+            float cm[BN / 32], cs[BN / 32];
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
+                const int col = n0 + c * 32;
+                float mx = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (col + j < n_axis) mx = fmaxf(mx, __uint_as_float(r[j]));
+                float sm_ = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (col + j < n_axis) sm_ += __expf(__uint_as_float(r[j]) - mx);
+                cm[c] = mx;
+                cs[c] = sm_;
+                if (row < L) {
+                    if (vec && col + 32 <= n_axis) {
+                        float4 *o4 = reinterpret_cast<float4 *>(out + col);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            o4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (col + j < n_axis) out[col + j] = __uint_as_float(r[j]);
+                    }
+                }
+            }
+            // this accumulator may be overwritten once every epilogue warp is done
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+            if (row < L) {
+                float M = cm[0];
+#pragma unroll
+                for (int c = 1; c < BN / 32; ++c) M = fmaxf(M, cm[c]);
+                float S = 0.f;
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c)
+                    if (cm[c] > -INFINITY) S += cs[c] * __expf(cm[c] - M);
+                float2 *part = col_axis ? part_c : part_r;
+                const int nta = col_axis ? ntile_c : ntile_r;
+                part[(size_t)row * nta + tn] = make_float2(M, S);
             }
         }
     }
@@ -262,7 +325,7 @@ bool make_map(CUtensorMap *tm, const uint16_t *ptr, int rows, int d, int box_row
 
 cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c,
                                int L, int d, int N_r, int N_c, float *s_r, float *s_c,
-                               int *status, cudaStream_t st) {
+                               float *part_r, float *part_c, int *status, cudaStream_t st) {
     CUtensorMap tm_x, tm_wr, tm_wc;
     if (!make_map(&tm_x, x, L, d, BM) || !make_map(&tm_wr, W_r, N_r, d, BN) ||
         !make_map(&tm_wc, W_c, N_c, d, BN))
@@ -272,9 +335,12 @@ cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *W_r, const uin
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int ntile_r = (N_r + BN - 1) / BN, ntile_c = (N_c + BN - 1) / BN;
-    dim3 grid(ntile_r + ntile_c, (L + BM - 1) / BM);
-    router_gemm_kernel<<<grid, 128, smem, st>>>(tm_x, tm_wr, tm_wc, s_r, s_c, L, d, N_r, N_c,
-                                                ntile_r, status);
+    const int ntiles = ((L + BM - 1) / BM) * (ntile_r + ntile_c);
+    const int sms = device_sm_count();
+    const int grid = ntiles < sms ? ntiles : sms;
+    router_gemm_kernel<<<grid, kThreads, smem, st>>>(
+        tm_x, tm_wr, tm_wc, s_r, s_c, reinterpret_cast<float2 *>(part_r),
+        reinterpret_cast<float2 *>(part_c), L, d, N_r, N_c, ntile_r, ntile_c, status);
     return cudaGetLastError();
 }
 

@@ -8,7 +8,8 @@
 // n = i * N_c + j, and axis ranks use (p desc, index asc).  Gates are the
 // softmax over the K selected scores.
 //
-// Kernel 1 (axis_topk): one warp per (token, axis).  Optional LogSoftmax,
+// Kernel 1 (axis_topk): one warp per (token, axis).  Optional LogSoftmax
+//   (from the router GEMM's per-tile max / sum-exp partials when given),
 //   then the axis' top min(K, n) entries.
 // Kernel 2 (merge_topk): one warp per token.  Because fp32 addition is
 //   monotone, a cell with row rank a and column rank b is dominated by every
@@ -189,7 +190,8 @@ __device__ __forceinline__ void bitonic_desc(uint64_t (&hi)[E], uint64_t (&lo)[E
 // area is either sel_key[kmax] + sel_idx[kmax] (fallback) or the bitonic staging (u64)
 template <int E>
 __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__restrict__ in_c,
-                                 int logsoftmax, float *__restrict__ p_r_out,
+                                 int logsoftmax, const float2 *__restrict__ part_r,
+                                 const float2 *__restrict__ part_c, float *__restrict__ p_r_out,
                                  float *__restrict__ p_c_out, int L, int N_r, int N_c, int K,
                                  float *__restrict__ row_val, int *__restrict__ row_idx,
                                  float *__restrict__ col_val, int *__restrict__ col_idx,
@@ -218,7 +220,28 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     uint64_t *stage = reinterpret_cast<uint64_t *>(base + area_off);
 
     float vmax = -INFINITY;
-    if (logsoftmax) {
+    const float2 *part = axis ? part_c : part_r;
+    if (logsoftmax && part) {
+        // per 128-column tile: (max, sum exp(s - max)) from the router GEMM
+        const int nt = (n + kGemmTileN - 1) / kGemmTileN;
+        float m = -INFINITY, sm_ = 0.f;
+        for (int u = lane; u < nt; u += 32) {
+            const float2 pt = part[(size_t)t * nt + u];
+            const float mn = fmaxf(m, pt.x);
+            sm_ = sm_ * __expf(m - mn) + pt.y * __expf(pt.x - mn);
+            m = mn;
+        }
+        const float mx = warp_max(m);
+        float sum = (m > -INFINITY) ? sm_ * __expf(m - mx) : 0.f;
+        sum = warp_sum(sum);
+        const float lse = mx + __logf(sum);
+        for (int i = lane; i < n; i += 32) {
+            const float p = in[i] - lse;
+            if (pout) pout[(size_t)t * n + i] = p;
+            vals[i] = p;
+        }
+        vmax = mx - lse;                   // the p of the largest logit, same rounding
+    } else if (logsoftmax) {
         float mx = -INFINITY;
         for (int i = lane; i < n; i += 32) {
             const float v = in[i];
@@ -549,6 +572,7 @@ int merge_candidates(int K, int Kr, int Kc) {
 
 template <int E>
 static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logsoftmax,
+                                 const float *part_r, const float *part_c,
                                  float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
                                  float *row_val, int *row_idx, float *col_val, int *col_idx,
                                  cudaStream_t st) {
@@ -570,13 +594,17 @@ static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logs
     }
     const int64_t probs = 2 * (int64_t)L;
     const unsigned grid = (unsigned)((probs + wpb - 1) / wpb);
-    axis_topk_kernel<E><<<grid, 32 * wpb, smem, st>>>(in_r, in_c, logsoftmax ? 1 : 0, p_r_out,
+    axis_topk_kernel<E><<<grid, 32 * wpb, smem, st>>>(in_r, in_c, logsoftmax ? 1 : 0,
+                                                      reinterpret_cast<const float2 *>(part_r),
+                                                      reinterpret_cast<const float2 *>(part_c),
+                                                      p_r_out,
                                                       p_c_out, L, N_r, N_c, K, row_val, row_idx,
                                                       col_val, col_idx, nmax, kmax, words);
     return cudaGetLastError();
 }
 
 cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftmax,
+                             const float *part_r, const float *part_c,
                              float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
                              float *row_val, int *row_idx, float *col_val, int *col_idx,
                              int *status, cudaStream_t st) {
@@ -584,7 +612,7 @@ cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftm
     const int nmax = N_r > N_c ? N_r : N_c;
     const int kmax = K < nmax ? K : nmax;
     switch (sort_capacity(kmax)) {
-#define OMNI_AX(e) case e: return launch_axis_e<e>(in_r, in_c, logsoftmax, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
+#define OMNI_AX(e) case e: return launch_axis_e<e>(in_r, in_c, logsoftmax, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
         OMNI_AX(1) OMNI_AX(2) OMNI_AX(4) OMNI_AX(8)
         default: OMNI_AX(0)
 #undef OMNI_AX
