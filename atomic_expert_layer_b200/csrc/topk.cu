@@ -24,10 +24,12 @@
 // bucket is strictly larger than any value in a higher one, so with b* the
 // bucket holding the k-th value, the top k are all values with b < b* plus
 // the best of bucket b*.  Those candidates (about k + 1 for Gaussian-like
-// rows) are sorted by the full key with a warp bitonic sort.  If fewer than k
-// values lie within 8 units of the maximum, or the candidates exceed the
-// sort's capacity, an exact radix select (4 passes of 8 bits over
-// order-preserving keys) followed by a rank sort is used instead.
+// rows) are placed by a counting sort on the bucket (buckets are in value
+// order) and ranked by the full key only among the peers of their bucket.
+// If fewer than k values lie within 8 units of the maximum, or there are
+// more candidates than the kernel's capacity, an exact radix select (4
+// passes of 8 bits over order-preserving keys) followed by a rank sort is
+// used instead.
 #include "omni_common.cuh"
 #include "omni_internal.h"
 
@@ -134,61 +136,34 @@ __device__ int bucket_threshold(Get get, int n, int k, float vmax, uint32_t *his
     return __shfl_sync(0xffffffffu, through, src);
 }
 
-// -------------------------------------------------------- warp bitonic sort
-// Sort 32*E keys held as v[i] of lane l (element id l + 32 i) in descending
-// order of (hi, lo).  With ONE_WORD only hi is compared.
-template <int E, bool ONE_WORD>
-__device__ __forceinline__ void bitonic_desc(uint64_t (&hi)[E], uint64_t (&lo)[E]) {
+// --------------------------------------------------- bucket counting sort
+// After bucket_threshold: turn the counts of buckets [0, kNB) into starting
+// positions (exclusive prefix, written back into hist) and copy them to cur.
+__device__ __forceinline__ void bucket_starts(uint32_t *hist, uint32_t *cur) {
     const unsigned lane = lane_id();
+    constexpr int per = kNB / 32;
+    uint32_t c[per];
+    int tot = 0;
 #pragma unroll
-    for (int k = 2; k <= 32 * E; k <<= 1) {
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            if (j >= 32) {
-#pragma unroll
-                for (int i = 0; i < E; ++i) {
-                    const int p = i ^ (j >> 5);
-                    if (p > i) {
-                        const bool desc = (((int)lane + 32 * i) & k) == 0;
-                        const bool gt = ONE_WORD ? hi[i] > hi[p]
-                                                 : (hi[i] > hi[p] || (hi[i] == hi[p] && lo[i] > lo[p]));
-                        if (desc != gt) {            // swap so the segment runs the right way
-                            const uint64_t th = hi[i], tl = lo[i];
-                            hi[i] = hi[p];
-                            lo[i] = lo[p];
-                            hi[p] = th;
-                            lo[p] = tl;
-                        }
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < E; ++i) {
-                    const int id = (int)lane + 32 * i;
-                    const uint64_t oh = __shfl_xor_sync(0xffffffffu, hi[i], j);
-                    const uint64_t ol = ONE_WORD ? 0ull : __shfl_xor_sync(0xffffffffu, lo[i], j);
-                    const bool low = (id & j) == 0;
-                    const bool desc = (id & k) == 0;
-                    const bool other_gt = ONE_WORD ? oh > hi[i]
-                                                   : (oh > hi[i] || (oh == hi[i] && ol > lo[i]));
-                    const bool other_lt = ONE_WORD ? oh < hi[i]
-                                                   : (oh < hi[i] || (oh == hi[i] && ol < lo[i]));
-                    // the low element keeps the larger key in a descending segment
-                    const bool take = (low == desc) ? other_gt : other_lt;
-                    if (take) {
-                        hi[i] = oh;
-                        lo[i] = ol;
-                    }
-                }
-            }
-        }
+    for (int j = 0; j < per; ++j) {
+        c[j] = hist[lane * per + j];
+        tot += (int)c[j];
     }
+    int run = warp_iscan(tot) - tot;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+        hist[lane * per + j] = (uint32_t)run;
+        cur[lane * per + j] = (uint32_t)run;
+        run += (int)c[j];
+    }
+    __syncwarp();
 }
 
 // ------------------------------------------------------------ axis top-K
-// Dynamic smem per warp (words): vals[nmax] | hist[kNB] | area[max(2 kmax, 64 E)], where
-// area is either sel_key[kmax] + sel_idx[kmax] (fallback) or the bitonic staging (u64)
-template <int E>
+// Dynamic smem per warp (words): vals[nmax] | hist[kNB] | cur[kNB] |
+// area[max(2 kmax, 2 CAP)], where area is either sel_key[kmax] + sel_idx[kmax]
+// (fallback) or the candidate keys tmp[CAP] (u64)
+template <int CAP>
 __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__restrict__ in_c,
                                  int logsoftmax, const float2 *__restrict__ part_r,
                                  const float2 *__restrict__ part_c, float *__restrict__ p_r_out,
@@ -214,10 +189,11 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     uint32_t *base = smem_u + (size_t)warp * warp_words;
     float *vals = reinterpret_cast<float *>(base);
     uint32_t *hist = base + nmax;
-    const size_t area_off = ((size_t)nmax + kNB + 1) & ~(size_t)1;      // 8-byte aligned
+    uint32_t *cur = hist + kNB;
+    const size_t area_off = ((size_t)nmax + 2 * kNB + 1) & ~(size_t)1;  // 8-byte aligned
     uint32_t *sel_key = base + area_off;
     int *sel_idx = reinterpret_cast<int *>(sel_key + kmax);
-    uint64_t *stage = reinterpret_cast<uint64_t *>(base + area_off);
+    uint64_t *tmp = reinterpret_cast<uint64_t *>(base + area_off);
 
     float vmax = -INFINITY;
     const float2 *part = axis ? part_c : part_r;
@@ -269,38 +245,33 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     }
     __syncwarp();
 
-    if (E > 0) {
+    if (CAP > 0) {
         int bs = 0;
         const int ncand =
             bucket_threshold([&](int i) { return vals[i]; }, n, kx, vmax, hist, &bs);
-        if (ncand >= kx && ncand <= 32 * E) {
-            // candidates in index order -> 64-bit keys (key(p), ~index)
-            int taken = 0;
-            for (int i0 = 0; i0 < n; i0 += 32) {
-                const int i = i0 + (int)lane;
-                const bool in_c = i < n && bucket_of(vmax, vals[i]) <= bs;
-                const unsigned bal = __ballot_sync(0xffffffffu, in_c);
-                if (in_c) {
-                    const int pos = taken + __popc(bal & lanemask_lt());
-                    stage[pos] = ((uint64_t)f2key(vals[i]) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
+        if (ncand >= kx && ncand <= CAP) {
+            // candidates go to their bucket's range; buckets are in value order
+            bucket_starts(hist, cur);
+            for (int i = lane; i < n; i += 32) {
+                const float v = vals[i];
+                if (bucket_of(vmax, v) <= bs) {
+                    const uint32_t pos = atomicAdd(&cur[bucket_of(vmax, v)], 1u);
+                    tmp[pos] = ((uint64_t)f2key(v) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
                 }
-                taken += __popc(bal);
             }
-            for (int i = taken + (int)lane; i < 32 * E; i += 32) stage[i] = 0ull;
             __syncwarp();
-            uint64_t hi[E > 0 ? E : 1], lo[E > 0 ? E : 1];
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                hi[i] = stage[lane + 32 * i];
-                lo[i] = 0ull;
-            }
-            bitonic_desc<(E > 0 ? E : 1), true>(hi, lo);
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const int r = (int)lane + 32 * i;
-                if (r < kx) {
-                    oval[r] = key2f((uint32_t)(hi[i] >> 32));
-                    oidx[r] = (int)(0xffffffffu - (uint32_t)hi[i]);
+            // inside a bucket, order by (key desc, index asc): rank among its peers
+            for (int pos = lane; pos < ncand; pos += 32) {
+                const uint64_t k = tmp[pos];
+                const int b = bucket_of(vmax, key2f((uint32_t)(k >> 32)));
+                const int s0 = (int)hist[b];
+                const int s1 = b < bs ? (int)hist[b + 1] : ncand;
+                int r = 0;
+                for (int q = s0; q < s1; ++q) r += tmp[q] > k ? 1 : 0;
+                const int fp = s0 + r;
+                if (fp < kx) {
+                    oval[fp] = key2f((uint32_t)(k >> 32));
+                    oidx[fp] = (int)(0xffffffffu - (uint32_t)k);
                 }
             }
             return;
@@ -361,7 +332,7 @@ __device__ __forceinline__ bool better(const Cand &u, const Cand &v) {
 }
 
 struct MergeLayout {   // offsets (words) inside one warp's region
-    size_t rv, ri, cv, ci, sval, hist, q, out_s, out_n, words;
+    size_t rv, ri, cv, ci, sval, hist, cur, q, out_s, out_n, words;
 };
 
 __host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C) {
@@ -373,8 +344,9 @@ __host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C
     m.ci = o; o += Kc;
     m.sval = o; o += C;
     m.hist = o; o += kNB;
+    m.cur = o; o += kNB;
     o = (o + 3) & ~(size_t)3;                 // 16-byte alignment for Cand / u64
-    m.q = o; o += 4 * (size_t)C;               // Cand[C], also the bitonic staging
+    m.q = o; o += 4 * (size_t)C;               // Cand[C] (fallback) or the candidate keys
     m.out_s = o; o += K;
     m.out_n = o; o += K;
     m.words = (o + 3) & ~(size_t)3;
@@ -382,7 +354,7 @@ __host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C
 }
 
 // Shared by the CTA: table[c] = (a << 16) | b for the c-th candidate, a-major.
-template <int E>
+template <int CAP>
 __global__ void merge_topk_kernel(const float *__restrict__ row_val,
                                   const int *__restrict__ row_idx,
                                   const float *__restrict__ col_val,
@@ -434,8 +406,9 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     uint32_t *ci = base + ml.ci;
     float *sval = reinterpret_cast<float *>(base + ml.sval);
     uint32_t *hist = base + ml.hist;
+    uint32_t *cur = base + ml.cur;
     Cand *q = reinterpret_cast<Cand *>(base + ml.q);
-    uint64_t *stage = reinterpret_cast<uint64_t *>(base + ml.q);
+    uint64_t *tmp = reinterpret_cast<uint64_t *>(base + ml.q);
     float *out_S = reinterpret_cast<float *>(base + ml.out_s);
     uint32_t *out_n = base + ml.out_n;
 
@@ -456,45 +429,40 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     __syncwarp();
 
     bool done = false;
-    if (E > 0) {
+    if (CAP > 0) {
         int bs = 0;
         const int ncand =
             bucket_threshold([&](int c) { return sval[c]; }, C, K, smax, hist, &bs);
-        if (ncand >= K && ncand <= 32 * E) {
-            int taken = 0;
-            for (int c0 = 0; c0 < C; c0 += 32) {
-                const int c = c0 + (int)lane;
-                const bool in_c = c < C && bucket_of(smax, sval[c]) <= bs;
-                const unsigned bal = __ballot_sync(0xffffffffu, in_c);
-                if (in_c) {
-                    const int pos = taken + __popc(bal & lanemask_lt());
+        if (ncand >= K && ncand <= CAP) {
+            bucket_starts(hist, cur);
+            for (int c = lane; c < C; c += 32) {
+                const float S = sval[c];
+                const int b = bucket_of(smax, S);
+                if (b <= bs) {
+                    const uint32_t pos = atomicAdd(&cur[b], 1u);
                     const uint32_t ab = table[c];
-                    const int a = (int)(ab >> 16), b = (int)(ab & 0xffffu);
-                    const uint32_t nn = ri[a] * (uint32_t)N_c + ci[b];
-                    stage[2 * pos] = ((uint64_t)f2key(sval[c]) << 32) | f2key(rv[a]);
-                    stage[2 * pos + 1] = ((uint64_t)f2key(cv[b]) << 32) | (uint64_t)(0xffffffffu - nn);
+                    const int a = (int)(ab >> 16), bb = (int)(ab & 0xffffu);
+                    const uint32_t nn = ri[a] * (uint32_t)N_c + ci[bb];
+                    tmp[2 * pos] = ((uint64_t)f2key(S) << 32) | f2key(rv[a]);
+                    tmp[2 * pos + 1] = ((uint64_t)f2key(cv[bb]) << 32) | (uint64_t)(0xffffffffu - nn);
                 }
-                taken += __popc(bal);
-            }
-            for (int i = taken + (int)lane; i < 32 * E; i += 32) {
-                stage[2 * i] = 0ull;
-                stage[2 * i + 1] = 0ull;
             }
             __syncwarp();
-            uint64_t hi[E > 0 ? E : 1], lo[E > 0 ? E : 1];
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                hi[i] = stage[2 * (lane + 32 * i)];
-                lo[i] = stage[2 * (lane + 32 * i) + 1];
-            }
-            bitonic_desc<(E > 0 ? E : 1), false>(hi, lo);
-            __syncwarp();
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const int r = (int)lane + 32 * i;
-                if (r < K) {
-                    out_S[r] = key2f((uint32_t)(hi[i] >> 32));
-                    out_n[r] = 0xffffffffu - (uint32_t)lo[i];
+            // inside a bucket, order by the full key: rank among its peers
+            for (int pos = lane; pos < ncand; pos += 32) {
+                const uint64_t kh = tmp[2 * pos], kl = tmp[2 * pos + 1];
+                const int b = bucket_of(smax, key2f((uint32_t)(kh >> 32)));
+                const int s0 = (int)hist[b];
+                const int s1 = b < bs ? (int)hist[b + 1] : ncand;
+                int r = 0;
+                for (int q = s0; q < s1; ++q) {
+                    const uint64_t qh = tmp[2 * q], ql = tmp[2 * q + 1];
+                    r += (qh > kh || (qh == kh && ql > kl)) ? 1 : 0;
+                }
+                const int fp = s0 + r;
+                if (fp < K) {
+                    out_S[fp] = key2f((uint32_t)(kh >> 32));
+                    out_n[fp] = 0xffffffffu - (uint32_t)kl;
                 }
             }
             done = true;
@@ -550,11 +518,9 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     }
 }
 
-int sort_capacity(int k) {
-    // warp bitonic capacity 32*E with room for the boundary bucket; 0 = none
-    int e = 1;
-    while (32 * e < k + 16) e <<= 1;
-    return e <= 8 ? e : 0;
+// candidates the fast path takes (the k best plus the boundary bucket); 0 = none
+int fast_capacity(int k) {
+    return k <= 1024 ? ((k + 64 + 31) / 32) * 32 : 0;
 }
 
 }  // namespace
@@ -570,7 +536,7 @@ int merge_candidates(int K, int Kr, int Kc) {
     return C;
 }
 
-template <int E>
+template <int CAP>
 static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logsoftmax,
                                  const float *part_r, const float *part_c,
                                  float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
@@ -578,8 +544,8 @@ static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logs
                                  cudaStream_t st) {
     const int nmax = N_r > N_c ? N_r : N_c;
     const int kmax = K < nmax ? K : nmax;
-    const size_t area = 2 * (size_t)kmax > 64 * (size_t)E ? 2 * (size_t)kmax : 64 * (size_t)E;
-    size_t words = (((size_t)nmax + kNB + 1) & ~(size_t)1) + area;
+    const size_t area = 2 * (size_t)kmax > 2 * (size_t)CAP ? 2 * (size_t)kmax : 2 * (size_t)CAP;
+    size_t words = (((size_t)nmax + 2 * kNB + 1) & ~(size_t)1) + area;
     words = (words + 3) & ~(size_t)3;
     const size_t per_warp = words * 4;
     int wpb = (int)((64 * 1024) / per_warp);
@@ -587,19 +553,19 @@ static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logs
     if (wpb < 1) wpb = 1;
     const size_t smem = per_warp * wpb;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(axis_topk_kernel<E>,
+        cudaError_t e = cudaFuncSetAttribute(axis_topk_kernel<CAP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
     }
     const int64_t probs = 2 * (int64_t)L;
     const unsigned grid = (unsigned)((probs + wpb - 1) / wpb);
-    axis_topk_kernel<E><<<grid, 32 * wpb, smem, st>>>(in_r, in_c, logsoftmax ? 1 : 0,
-                                                      reinterpret_cast<const float2 *>(part_r),
-                                                      reinterpret_cast<const float2 *>(part_c),
-                                                      p_r_out,
-                                                      p_c_out, L, N_r, N_c, K, row_val, row_idx,
-                                                      col_val, col_idx, nmax, kmax, words);
+    axis_topk_kernel<CAP><<<grid, 32 * wpb, smem, st>>>(in_r, in_c, logsoftmax ? 1 : 0,
+                                                        reinterpret_cast<const float2 *>(part_r),
+                                                        reinterpret_cast<const float2 *>(part_c),
+                                                        p_r_out, p_c_out, L, N_r, N_c, K, row_val,
+                                                        row_idx, col_val, col_idx, nmax, kmax,
+                                                        words);
     return cudaGetLastError();
 }
 
@@ -611,15 +577,18 @@ cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftm
     (void)status;
     const int nmax = N_r > N_c ? N_r : N_c;
     const int kmax = K < nmax ? K : nmax;
-    switch (sort_capacity(kmax)) {
-#define OMNI_AX(e) case e: return launch_axis_e<e>(in_r, in_c, logsoftmax, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
-        OMNI_AX(1) OMNI_AX(2) OMNI_AX(4) OMNI_AX(8)
-        default: OMNI_AX(0)
+    const int cap = fast_capacity(kmax);
+#define OMNI_AX(c) return launch_axis_e<c>(in_r, in_c, logsoftmax, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
+    if (cap == 0) { OMNI_AX(0) }
+    if (cap <= 96) { OMNI_AX(96) }
+    if (cap <= 192) { OMNI_AX(192) }
+    if (cap <= 320) { OMNI_AX(320) }
+    if (cap <= 576) { OMNI_AX(576) }
+    OMNI_AX(1088)
 #undef OMNI_AX
-    }
 }
 
-template <int E>
+template <int CAP>
 static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, const float *col_val,
                                   const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
                                   int32_t *idx, float *score, float *gate, cudaStream_t st) {
@@ -631,29 +600,31 @@ static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, cons
     if (wpb < 1) wpb = 1;
     const size_t smem = head * 4 + per_warp * wpb;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel<E>,
+        cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel<CAP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
     }
     const unsigned grid = (unsigned)((L + wpb - 1) / wpb);
-    merge_topk_kernel<E><<<grid, 32 * wpb, smem, st>>>(row_val, row_idx, col_val, col_idx, L, N_c,
-                                                       K, Kr, Kc, C, idx, score, gate);
+    merge_topk_kernel<CAP><<<grid, 32 * wpb, smem, st>>>(row_val, row_idx, col_val, col_idx, L,
+                                                         N_c, K, Kr, Kc, C, idx, score, gate);
     return cudaGetLastError();
 }
 
 cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
                               const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
                               int32_t *idx, float *score, float *gate, cudaStream_t st) {
-    // the bitonic staging lives in the Cand area (4 words per candidate)
-    int e = sort_capacity(K);
-    if (e > 0 && 32 * e > C) e = 0;
-    switch (e) {
-#define OMNI_MG(e) case e: return launch_merge_e<e>(row_val, row_idx, col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, st);
-        OMNI_MG(1) OMNI_MG(2) OMNI_MG(4) OMNI_MG(8)
-        default: OMNI_MG(0)
+    // the candidate keys (4 words each) live in the Cand area (4 words per candidate)
+    int cap = fast_capacity(K);
+    if (cap > C) cap = C >= K ? (C / 32) * 32 : 0;
+#define OMNI_MG(c) return launch_merge_e<c>(row_val, row_idx, col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, st);
+    if (cap < K) { OMNI_MG(0) }
+    if (cap <= 96) { OMNI_MG(96) }
+    if (cap <= 192) { OMNI_MG(192) }
+    if (cap <= 320) { OMNI_MG(320) }
+    if (cap <= 576) { OMNI_MG(576) }
+    OMNI_MG(1088)
 #undef OMNI_MG
-    }
 }
 
 }  // namespace omni
