@@ -10,10 +10,11 @@
 //
 // Pipeline (no host synchronisation, no spin-waits):
 //   1. prepare (warp per token): sort the token's K tasks by expert id, write
-//      them in (t, e) order, count tasks per group, mark experts in a bitmap,
-//      and count the first radix pass's digits per 2048-task tile (atomics).
-//   2. scans (one launch, two CTAs): group offsets, active-group list and
-//      distinct-expert count; the first pass's digit-major histogram.
+//      them in (t, e) order, count tasks per group, count distinct experts
+//      (the first task to set an expert's bit in a bitmap counts it), and
+//      count the first radix pass's digits per 2048-task tile (atomics).
+//   2. scans (one launch, two CTAs): group offsets and active-group list;
+//      the first pass's digit-major histogram.
 //   3. LSD radix sort of the tasks on q alone, digits of <= 8 bits, stable.
 //      The input is in (t, e) order, so a stable sort by q yields (q, t, e).
 //      Each pass: stable scatter (warps rank equal digits with
@@ -41,8 +42,9 @@ __global__ void sched_prepare_kernel(const int32_t *__restrict__ idx,
                                      const float *__restrict__ gate, int L, int K, int N, int B,
                                      int32_t *__restrict__ a_tok, int32_t *__restrict__ a_exp,
                                      float *__restrict__ a_gate, int32_t *__restrict__ counts,
-                                     uint32_t *__restrict__ bitmap, int32_t *__restrict__ hist0,
-                                     int64_t ntiles, uint32_t dmask0, int *status) {
+                                     uint32_t *__restrict__ bitmap, int32_t *__restrict__ num_distinct,
+                                     int32_t *__restrict__ hist0, int64_t ntiles, uint32_t dmask0,
+                                     int *status) {
     extern __shared__ int32_t sh_e[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
@@ -59,22 +61,30 @@ __global__ void sched_prepare_kernel(const int32_t *__restrict__ idx,
         e_s[k] = e;
     }
     __syncwarp();
-    for (int u = lane; u < K; u += 32) {
-        const int32_t eu = e_s[u];
-        int r = 0;
-        for (int v = 0; v < K; ++v) {
-            const int32_t ev = e_s[v];
-            r += (ev < eu) | ((ev == eu) & (v < u));
+    for (int u0 = 0; u0 < K; u0 += 32) {
+        const int u = u0 + (int)lane;
+        bool fresh = false;
+        if (u < K) {
+            const int32_t eu = e_s[u];
+            int r = 0;
+            for (int v = 0; v < K; ++v) {
+                const int32_t ev = e_s[v];
+                r += (ev < eu) | ((ev == eu) & (v < u));
+            }
+            const int32_t raw = idx[row + u];
+            const float g = (raw < 0 || raw >= N) ? 0.f : gate[row + u];
+            const size_t pos = row + r;
+            a_tok[pos] = t;
+            a_exp[pos] = eu;
+            a_gate[pos] = g;
+            atomicAdd(&counts[eu / B], 1);
+            const uint32_t bit = 1u << (eu & 31);
+            fresh = (atomicOr(&bitmap[eu >> 5], bit) & bit) == 0u;   // first task of expert eu
+            if (hist0)
+                atomicAdd(&hist0[(int64_t)digit_of(eu, B, 0, dmask0) * ntiles + pos / kSortTile], 1);
         }
-        const int32_t raw = idx[row + u];
-        const float g = (raw < 0 || raw >= N) ? 0.f : gate[row + u];
-        const size_t pos = row + r;
-        a_tok[pos] = t;
-        a_exp[pos] = eu;
-        a_gate[pos] = g;
-        atomicAdd(&counts[eu / B], 1);
-        atomicOr(&bitmap[eu >> 5], 1u << (eu & 31));
-        if (hist0) atomicAdd(&hist0[(int64_t)digit_of(eu, B, 0, dmask0) * ntiles + pos / kSortTile], 1);
+        const int nf = __popc(__ballot_sync(0xffffffffu, fresh));
+        if (lane == 0 && nf) atomicAdd(num_distinct, nf);
     }
 }
 
@@ -100,16 +110,28 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *sh32, int *total
 constexpr int kScanTile = 4096;            // elements per tile: 1024 threads x 4
 
 // In-place exclusive scan of a[0..n) by one CTA of 1024 threads.  Tiles of
-// 4096 are loaded coalesced into shared memory; each thread then owns 4
-// consecutive elements.  If `tail` is non-null the total is written there.
+// 4096 are loaded coalesced (the next tile's loads are issued before the
+// current tile is scanned) and staged through shared memory so each thread
+// owns 4 consecutive elements.  If `tail` is non-null the total is written
+// there.
 __device__ void cta_exclusive_scan(int32_t *a, int64_t n, int32_t *tail, int *tile, int *sh32) {
     const int tid = threadIdx.x;
     int carry = 0;
+    int nx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int64_t i = (int64_t)k * 1024 + tid;
+        nx[k] = i < n ? a[i] : 0;
+    }
     for (int64_t base = 0; base < n; base += kScanTile) {
         __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tile[k * 1024 + tid] = nx[k];
+        const int64_t nb = base + kScanTile;
+#pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int64_t i = base + k * 1024 + tid;
-            tile[k * 1024 + tid] = i < n ? a[i] : 0;
+            const int64_t i = nb + k * 1024 + tid;
+            nx[k] = i < n ? a[i] : 0;
         }
         __syncthreads();
         int v[4], sum = 0;
@@ -138,9 +160,8 @@ __device__ void cta_exclusive_scan(int32_t *a, int64_t n, int32_t *tail, int *ti
 // experts.  CTA 1 (if a radix pass follows): exclusive scan of the first
 // pass's digit-major histogram.
 __global__ void __launch_bounds__(1024) sched_scan_kernel(
-    const int32_t *__restrict__ counts, int64_t G, const uint32_t *__restrict__ bitmap,
-    int64_t nwords, int32_t *__restrict__ offsets, int32_t *__restrict__ active,
-    int32_t *__restrict__ num_active, int32_t *__restrict__ num_distinct,
+    const int32_t *__restrict__ counts, int64_t G, int32_t *__restrict__ offsets,
+    int32_t *__restrict__ active, int32_t *__restrict__ num_active,
     int32_t *__restrict__ hist0, int64_t nhist) {
     __shared__ int tile[kScanTile];
     __shared__ int tile2[kScanTile];
@@ -150,13 +171,22 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(
         cta_exclusive_scan(hist0, nhist, nullptr, tile, sh32);
         return;
     }
-    int carry = 0, acarry = 0, pop = 0;
-    for (int64_t w = tid; w < nwords; w += 1024) pop += __popc(bitmap[w]);
+    int carry = 0, acarry = 0;
+    int nx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int64_t i = (int64_t)k * 1024 + tid;
+        nx[k] = i < G ? counts[i] : 0;
+    }
     for (int64_t base = 0; base < G; base += kScanTile) {
         __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tile[k * 1024 + tid] = nx[k];
+        const int64_t nb = base + kScanTile;
+#pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int64_t i = base + k * 1024 + tid;
-            tile[k * 1024 + tid] = i < G ? counts[i] : 0;
+            const int64_t i = nb + k * 1024 + tid;
+            nx[k] = i < G ? counts[i] : 0;
         }
         __syncthreads();
         int v[4], sum = 0, act = 0;
@@ -182,12 +212,9 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(
             if (i < G) offsets[i] = tile2[k * 1024 + tid];
         }
     }
-    int ptotal;
-    block_exclusive_scan(pop, sh32, &ptotal);
     if (tid == 0) {
         offsets[G] = carry;
         *num_active = acarry;
-        *num_distinct = ptotal;
     }
 }
 
@@ -301,6 +328,7 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
 
     if ((e = cudaMemsetAsync(group_counts, 0, sizeof(int32_t) * G, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(bitmap, 0, sizeof(uint32_t) * nwords, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(num_distinct, 0, sizeof(int32_t), st)) != cudaSuccess) return e;
     if (passes > 0 &&
         (e = cudaMemsetAsync(hist, 0, sizeof(int32_t) * hstride * passes, st)) != cudaSuccess)
         return e;
@@ -309,12 +337,12 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
         const size_t smem = sizeof(int32_t) * (size_t)sz.K * wpb;
         sched_prepare_kernel<<<(unsigned)((sz.L + wpb - 1) / wpb), 32 * wpb, smem, st>>>(
             idx, gate, sz.L, sz.K, (int)sz.N, sz.B, a_tok, a_exp, a_gate, group_counts, bitmap,
-            passes ? hist : nullptr, ntiles, passes ? pass_mask(0) : 0u, status);
+            num_distinct, passes ? hist : nullptr, ntiles, passes ? pass_mask(0) : 0u, status);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     sched_scan_kernel<<<passes ? 2 : 1, 1024, 0, st>>>(
-        group_counts, G, bitmap, nwords, group_offsets, active_groups, num_active, num_distinct,
-        hist, passes ? (int64_t)(pass_mask(0) + 1) * ntiles : 0);
+        group_counts, G, group_offsets, active_groups, num_active, hist,
+        passes ? (int64_t)(pass_mask(0) + 1) * ntiles : 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     if (passes == 0) {

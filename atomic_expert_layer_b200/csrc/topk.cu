@@ -98,9 +98,38 @@ __device__ __forceinline__ int bucket_of(float vmax, float v) {
     return dv < (float)kNB ? (int)dv : kNB;           // kNB = beyond the range
 }
 
-// Zero the histogram, count vals[0..n) (optionally through `get`) into it and
-// find the bucket b* holding the k-th largest value.  Returns the number of
-// values in buckets <= b*, or -1 if fewer than k values are in range.
+// Find the bucket b* holding the k-th largest value from a filled histogram.
+// Returns the number of values in buckets <= b*, or -1 if fewer than k values
+// are in range.
+__device__ int bucket_find(const uint32_t *hist, int k, int *bstar) {
+    const unsigned lane = lane_id();
+    constexpr int per = kNB / 32;            // lane l owns buckets [l * per, (l + 1) * per)
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < per; ++j) tot += (int)hist[lane * per + j];
+    const int incl = warp_iscan(tot);
+    const int excl = incl - tot;
+    const bool mine = excl < k && k <= incl;
+    const unsigned bal = __ballot_sync(0xffffffffu, mine);
+    if (bal == 0u) return -1;
+    int bs = 0, through = 0;
+    if (mine) {
+        int run = excl;
+#pragma unroll
+        for (int j = 0; j < per; ++j) {
+            run += (int)hist[lane * per + j];
+            if (run >= k && through == 0) {
+                bs = lane * per + j;
+                through = run;
+            }
+        }
+    }
+    const int src = __ffs(bal) - 1;
+    *bstar = __shfl_sync(0xffffffffu, bs, src);
+    return __shfl_sync(0xffffffffu, through, src);
+}
+
+// Zero the histogram, count get(0..n) into it and find b* (see bucket_find).
 template <typename Get>
 __device__ int bucket_threshold(Get get, int n, int k, float vmax, uint32_t *hist, int *bstar) {
     const unsigned lane = lane_id();
@@ -111,29 +140,7 @@ __device__ int bucket_threshold(Get get, int n, int k, float vmax, uint32_t *his
         if (b < kNB) atomicAdd(&hist[b], 1u);
     }
     __syncwarp();
-    // lane l owns buckets [l * kNB/32, (l + 1) * kNB/32)
-    int tot = 0;
-    for (int j = 0; j < kNB / 32; ++j) tot += (int)hist[lane * (kNB / 32) + j];
-    const int incl = warp_iscan(tot);
-    const int excl = incl - tot;
-    const bool mine = excl < k && k <= incl;
-    const unsigned bal = __ballot_sync(0xffffffffu, mine);
-    if (bal == 0u) return -1;
-    int bs = 0, through = 0;
-    if (mine) {
-        int run = excl;
-        for (int j = 0; j < kNB / 32; ++j) {
-            run += (int)hist[lane * (kNB / 32) + j];
-            if (run >= k) {
-                bs = lane * (kNB / 32) + j;
-                through = run;
-                break;
-            }
-        }
-    }
-    const int src = __ffs(bal) - 1;
-    *bstar = __shfl_sync(0xffffffffu, bs, src);
-    return __shfl_sync(0xffffffffu, through, src);
+    return bucket_find(hist, k, bstar);
 }
 
 // --------------------------------------------------- bucket counting sort
@@ -196,6 +203,7 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     uint64_t *tmp = reinterpret_cast<uint64_t *>(base + area_off);
 
     float vmax = -INFINITY;
+    bool counted = false;                  // buckets already filled
     const float2 *part = axis ? part_c : part_r;
     if (logsoftmax && part) {
         // per 128-column tile: (max, sum exp(s - max)) from the router GEMM
@@ -211,12 +219,37 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
         float sum = (m > -INFINITY) ? sm_ * __expf(m - mx) : 0.f;
         sum = warp_sum(sum);
         const float lse = mx + __logf(sum);
-        for (int i = lane; i < n; i += 32) {
-            const float p = in[i] - lse;
+        vmax = mx - lse;                   // the p of the largest logit, same rounding
+        if (CAP > 0) {
+            for (int b = lane; b < kNB; b += 32) hist[b] = 0u;
+            __syncwarp();
+        }
+        // one pass: p = s - lse, kept in shared memory, counted into the buckets
+        auto one = [&](int i, float sv) {
+            const float p = sv - lse;
             if (pout) pout[(size_t)t * n + i] = p;
             vals[i] = p;
+            if (CAP > 0) {
+                const int b = bucket_of(vmax, p);
+                if (b < kNB) atomicAdd(&hist[b], 1u);
+            }
+        };
+        if ((n & 3) == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0) {
+            const float4 *in4 = reinterpret_cast<const float4 *>(in);
+            const int n4 = n >> 2;
+#pragma unroll 4
+            for (int i4 = lane; i4 < n4; i4 += 32) {
+                const float4 v = in4[i4];
+                one(4 * i4, v.x);
+                one(4 * i4 + 1, v.y);
+                one(4 * i4 + 2, v.z);
+                one(4 * i4 + 3, v.w);
+            }
+        } else {
+#pragma unroll 4
+            for (int i = lane; i < n; i += 32) one(i, in[i]);
         }
-        vmax = mx - lse;                   // the p of the largest logit, same rounding
+        counted = true;
     } else if (logsoftmax) {
         float mx = -INFINITY;
         for (int i = lane; i < n; i += 32) {
@@ -248,7 +281,8 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     if (CAP > 0) {
         int bs = 0;
         const int ncand =
-            bucket_threshold([&](int i) { return vals[i]; }, n, kx, vmax, hist, &bs);
+            counted ? bucket_find(hist, kx, &bs)
+                    : bucket_threshold([&](int i) { return vals[i]; }, n, kx, vmax, hist, &bs);
         if (ncand >= kx && ncand <= CAP) {
             // candidates go to their bucket's range; buckets are in value order
             bucket_starts(hist, cur);
@@ -421,18 +455,26 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
         ci[b] = (uint32_t)col_idx[(size_t)t * Kc + b];
     }
     __syncwarp();
+    const float smax = __fadd_rn(rv[0], cv[0]);           // cell (0, 0) is the largest
+    if (CAP > 0) {
+        for (int b = lane; b < kNB; b += 32) hist[b] = 0u;
+        __syncwarp();
+    }
     for (int c = lane; c < C; c += 32) {
         const uint32_t ab = table[c];
-        sval[c] = __fadd_rn(rv[ab >> 16], cv[ab & 0xffffu]);
+        const float S = __fadd_rn(rv[ab >> 16], cv[ab & 0xffffu]);
+        sval[c] = S;
+        if (CAP > 0) {
+            const int b = bucket_of(smax, S);
+            if (b < kNB) atomicAdd(&hist[b], 1u);
+        }
     }
-    const float smax = __fadd_rn(rv[0], cv[0]);           // cell (0, 0) is the largest
     __syncwarp();
 
     bool done = false;
     if (CAP > 0) {
         int bs = 0;
-        const int ncand =
-            bucket_threshold([&](int c) { return sval[c]; }, C, K, smax, hist, &bs);
+        const int ncand = bucket_find(hist, K, &bs);
         if (ncand >= K && ncand <= CAP) {
             bucket_starts(hist, cur);
             for (int c = lane; c < C; c += 32) {
