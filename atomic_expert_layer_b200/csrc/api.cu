@@ -56,8 +56,8 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
     if (regions & kRegRouter) {
         w.s_r = take(4 * L * sz.N_r);
         w.s_c = take(4 * L * sz.N_c);
-        w.part_r = take(8 * L * (size_t)((sz.N_r + kGemmTileN - 1) / kGemmTileN));
-        w.part_c = take(8 * L * (size_t)((sz.N_c + kGemmTileN - 1) / kGemmTileN));
+        w.part_r = take(8 * L * 2 * (size_t)((sz.N_r + 2 * kGemmPartCols - 1) / (2 * kGemmPartCols)));
+        w.part_c = take(8 * L * 2 * (size_t)((sz.N_c + 2 * kGemmPartCols - 1) / (2 * kGemmPartCols)));
         w.row_val = take(4 * L * sz.Kr);
         w.row_idx = take(4 * L * sz.Kr);
         w.col_val = take(4 * L * sz.Kc);

@@ -10,11 +10,12 @@
 // first, then those of W_c), K step 64 (one 128-byte swizzle atom of bf16).
 // Warp roles: warp 0 issues TMA tile loads (no multicast) into a 6-stage
 // shared-memory ring; warp 1 issues tcgen05.mma kind::f16 (bf16 in, fp32
-// accumulate) into one of two 128-column TMEM accumulators; warps 2-5 drain
-// the other accumulator with tcgen05.ld (one TMEM lane quarter each), write
-// the fp32 logits and, per (token, tile), the maximum and the sum of
-// exp(s - max) over the tile's columns -- the LogSoftmax partials -- so the
-// epilogue of one tile overlaps the main loop of the next.  Ragged edges (L,
+// accumulate) into one of two 128-column TMEM accumulators; warps 2-9 drain
+// the other accumulator with tcgen05.ld (two warps per TMEM lane quarter,
+// one per column half), write the fp32 logits and, per (token, tile, half),
+// the maximum and the sum of exp(s - max) over those columns -- the
+// LogSoftmax partials -- so the epilogue of one tile overlaps the main loop
+// of the next.  Ragged edges (L,
 // N_r, N_c, d not multiples of the tile) read as zeros through TMA
 // out-of-bounds fill and are masked on store.
 #include <cuda.h>
@@ -29,7 +30,8 @@ constexpr int BM = 128, BN = 128, BK = 64, STAGES = 6;
 constexpr int kTileBytesA = BM * BK * 2;     // 16 KB
 constexpr int kTileBytesB = BN * BK * 2;     // 16 KB
 constexpr uint32_t kTmemCols = 2 * BN;       // two fp32 accumulators
-constexpr int kThreads = 192;                // producer, MMA, 4 epilogue warps
+constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter, half the columns each
+constexpr int kThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue warps
 
 struct __align__(1024) GemmSmem {
     uint8_t a[STAGES][kTileBytesA];
@@ -133,7 +135,7 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.tfull[b], 1);
-            mbar_init(&sm.tempty[b], 4);
+            mbar_init(&sm.tempty[b], kEpiWarps);
         }
         sm.abort = 0;
         fence_barrier_init();
@@ -214,8 +216,11 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
         }
         __syncwarp();
     } else {
-        // ---- epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (accumulator rows)
+        // ---- epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (accumulator
+        // rows) and column half (w - 2) / 4 of the tile
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;
+        constexpr int kChunks = BN / 32 / 2;         // 32-column chunks per warp
         int lt = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
             const int buf = lt & 1;
@@ -225,25 +230,32 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
             const int nt = tile % nnt;
             const bool col_axis = nt >= ntile_r;
             const int tn = col_axis ? nt - ntile_r : nt;
-            const int n0 = tn * BN;
+            const int n0 = tn * BN + half * (BN / 2);
             const int n_axis = col_axis ? N_c : N_r;
             const int row = m0 + quarter * 32 + (int)lane;
             float *out = (col_axis ? s_c : s_r) + (size_t)row * n_axis;
             const bool vec = (n_axis & 3) == 0;
-            float cm[BN / 32], cs[BN / 32];
+            float cm[kChunks], cs[kChunks];
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = 0; c < kChunks; ++c) {
                 uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
+                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) +
+                              (uint32_t)(buf * BN + half * (BN / 2) + c * 32), r);
                 const int col = n0 + c * 32;
-                float mx = -INFINITY;
+                float mx = -INFINITY, sm_ = 0.f;
+                if (col + 32 <= n_axis) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (col + j < n_axis) mx = fmaxf(mx, __uint_as_float(r[j]));
-                float sm_ = 0.f;
+                    for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(r[j]));
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (col + j < n_axis) sm_ += __expf(__uint_as_float(r[j]) - mx);
+                    for (int j = 0; j < 32; ++j) sm_ += __expf(__uint_as_float(r[j]) - mx);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (col + j < n_axis) mx = fmaxf(mx, __uint_as_float(r[j]));
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (col + j < n_axis) sm_ += __expf(__uint_as_float(r[j]) - mx);
+                }
                 cm[c] = mx;
                 cs[c] = sm_;
                 if (row < L) {
@@ -267,14 +279,16 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
             if (row < L) {
                 float M = cm[0];
 #pragma unroll
-                for (int c = 1; c < BN / 32; ++c) M = fmaxf(M, cm[c]);
+                for (int c = 1; c < kChunks; ++c) M = fmaxf(M, cm[c]);
                 float S = 0.f;
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c)
+                for (int c = 0; c < kChunks; ++c)
                     if (cm[c] > -INFINITY) S += cs[c] * __expf(cm[c] - M);
+                // one (max, sum) pair per (row, tile, column half); a half with no
+                // valid column gives (-inf, 0)
                 float2 *part = col_axis ? part_c : part_r;
                 const int nta = col_axis ? ntile_c : ntile_r;
-                part[(size_t)row * nta + tn] = make_float2(M, S);
+                part[((size_t)row * nta + tn) * 2 + half] = make_float2(M, S);
             }
         }
     }

@@ -206,14 +206,16 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     bool counted = false;                  // buckets already filled
     const float2 *part = axis ? part_c : part_r;
     if (logsoftmax && part) {
-        // per 128-column tile: (max, sum exp(s - max)) from the router GEMM
-        const int nt = (n + kGemmTileN - 1) / kGemmTileN;
+        // per 64 columns: (max, sum exp(s - max)) from the router GEMM
+        const int nt = 2 * ((n + 2 * kGemmPartCols - 1) / (2 * kGemmPartCols));
         float m = -INFINITY, sm_ = 0.f;
         for (int u = lane; u < nt; u += 32) {
             const float2 pt = part[(size_t)t * nt + u];
-            const float mn = fmaxf(m, pt.x);
-            sm_ = sm_ * __expf(m - mn) + pt.y * __expf(pt.x - mn);
-            m = mn;
+            if (pt.x > -INFINITY) {
+                const float mn = fmaxf(m, pt.x);
+                sm_ = (m > -INFINITY ? sm_ * __expf(m - mn) : 0.f) + pt.y * __expf(pt.x - mn);
+                m = mn;
+            }
         }
         const float mx = warp_max(m);
         float sum = (m > -INFINITY) ? sm_ * __expf(m - mx) : 0.f;
@@ -225,29 +227,46 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
             __syncwarp();
         }
         // one pass: p = s - lse, kept in shared memory, counted into the buckets
-        auto one = [&](int i, float sv) {
-            const float p = sv - lse;
-            if (pout) pout[(size_t)t * n + i] = p;
-            vals[i] = p;
+        auto count = [&](float p) {
             if (CAP > 0) {
                 const int b = bucket_of(vmax, p);
                 if (b < kNB) atomicAdd(&hist[b], 1u);
             }
         };
         if ((n & 3) == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0) {
+            // 16-byte loads and 16-byte shared stores (no bank conflicts)
             const float4 *in4 = reinterpret_cast<const float4 *>(in);
+            float4 *v4 = reinterpret_cast<float4 *>(vals);
+            float *prow = pout ? pout + (size_t)t * n : nullptr;
+            const bool o_vec = prow && (reinterpret_cast<uintptr_t>(prow) & 15u) == 0;
+            float4 *o4 = reinterpret_cast<float4 *>(prow);
             const int n4 = n >> 2;
 #pragma unroll 4
             for (int i4 = lane; i4 < n4; i4 += 32) {
                 const float4 v = in4[i4];
-                one(4 * i4, v.x);
-                one(4 * i4 + 1, v.y);
-                one(4 * i4 + 2, v.z);
-                one(4 * i4 + 3, v.w);
+                const float4 p = make_float4(v.x - lse, v.y - lse, v.z - lse, v.w - lse);
+                v4[i4] = p;
+                if (o_vec) {
+                    o4[i4] = p;
+                } else if (prow) {
+                    prow[4 * i4] = p.x;
+                    prow[4 * i4 + 1] = p.y;
+                    prow[4 * i4 + 2] = p.z;
+                    prow[4 * i4 + 3] = p.w;
+                }
+                count(p.x);
+                count(p.y);
+                count(p.z);
+                count(p.w);
             }
         } else {
 #pragma unroll 4
-            for (int i = lane; i < n; i += 32) one(i, in[i]);
+            for (int i = lane; i < n; i += 32) {
+                const float p = in[i] - lse;
+                if (pout) pout[(size_t)t * n + i] = p;
+                vals[i] = p;
+                count(p);
+            }
         }
         counted = true;
     } else if (logsoftmax) {
