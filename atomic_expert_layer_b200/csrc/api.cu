@@ -58,6 +58,7 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.s_c = take(4 * L * sz.N_c);
         w.part_r = take(8 * L * 2 * (size_t)((sz.N_r + 2 * kGemmPartCols - 1) / (2 * kGemmPartCols)));
         w.part_c = take(8 * L * 2 * (size_t)((sz.N_c + 2 * kGemmPartCols - 1) / (2 * kGemmPartCols)));
+        w.flags = take(4 * 2 * L);
         w.row_val = take(4 * L * sz.Kr);
         w.row_idx = take(4 * L * sz.Kr);
         w.col_val = take(4 * L * sz.Kc);
@@ -137,10 +138,11 @@ int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c
     int *status = ws_at<int>(ws, lay.hdr);
     float *row_val = ws_at<float>(ws, lay.row_val), *col_val = ws_at<float>(ws, lay.col_val);
     int *row_idx = ws_at<int>(ws, lay.row_idx), *col_idx = ws_at<int>(ws, lay.col_idx);
+    int *row_flags = ws_at<int>(ws, lay.flags);
     cudaError_t e;
     if (flags & OMNI_ROUTER_LOGPROBS_IN) {
         e = launch_axis_topk(p_r, p_c, false, nullptr, nullptr, nullptr, nullptr, sz.L, sz.N_r,
-                             sz.N_c, sz.K, row_val, row_idx, col_val, col_idx, status, st);
+                             sz.N_c, sz.K, row_val, row_idx, col_val, col_idx, row_flags, status, st);
     } else {
         float *s_r = ws_at<float>(ws, lay.s_r), *s_c = ws_at<float>(ws, lay.s_c);
         float *part_r = ws_at<float>(ws, lay.part_r), *part_c = ws_at<float>(ws, lay.part_c);
@@ -148,7 +150,7 @@ int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c
                                status, st);
         if (e != cudaSuccess) return OMNI_ERR_CUDA;
         e = launch_axis_topk(s_r, s_c, true, part_r, part_c, p_r, p_c, sz.L, sz.N_r, sz.N_c,
-                             sz.K, row_val, row_idx, col_val, col_idx, status, st);
+                             sz.K, row_val, row_idx, col_val, col_idx, row_flags, status, st);
     }
     if (e != cudaSuccess) return OMNI_ERR_CUDA;
     e = launch_merge_topk(row_val, row_idx, col_val, col_idx, sz.L, sz.N_c, sz.K, sz.Kr, sz.Kc,

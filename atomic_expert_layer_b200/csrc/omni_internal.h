@@ -20,7 +20,7 @@ struct Sizes {
 };
 
 struct WsLayout {
-    size_t hdr, s_r, s_c, part_r, part_c, row_val, row_idx, col_val, col_idx, idx, score, gate;
+    size_t hdr, s_r, s_c, part_r, part_c, flags, row_val, row_idx, col_val, col_idx, idx, score, gate;
     size_t a_tok, a_exp, a_gate, b_tok, b_exp, b_gate, t_tok, t_exp, t_gate;
     size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, tok_count, tok_slots;
     size_t total;
@@ -61,7 +61,7 @@ cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftm
                              const float *part_r, const float *part_c,
                              float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
                              float *row_val, int *row_idx, float *col_val, int *col_idx,
-                             int *status, cudaStream_t st);
+                             int *flags, int *status, cudaStream_t st);
 cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
                               const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
                               int32_t *idx, float *score, float *gate, cudaStream_t st);

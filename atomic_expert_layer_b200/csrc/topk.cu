@@ -143,6 +143,27 @@ __device__ int bucket_threshold(Get get, int n, int k, float vmax, uint32_t *his
     return bucket_find(hist, k, bstar);
 }
 
+// LogSoftmax normaliser of row t from the router GEMM's partials: per 64
+// columns (max, sum exp(s - max)).  Returns lse; *mx is the row maximum.
+__device__ __forceinline__ float lse_from_partials(const float2 *part, int t, int n, float *mx_out) {
+    const unsigned lane = lane_id();
+    const int nt = 2 * ((n + 2 * kGemmPartCols - 1) / (2 * kGemmPartCols));
+    float m = -INFINITY, sm_ = 0.f;
+    for (int u = lane; u < nt; u += 32) {
+        const float2 pt = part[(size_t)t * nt + u];
+        if (pt.x > -INFINITY) {
+            const float mn = fmaxf(m, pt.x);
+            sm_ = (m > -INFINITY ? sm_ * __expf(m - mn) : 0.f) + pt.y * __expf(pt.x - mn);
+            m = mn;
+        }
+    }
+    const float mx = warp_max(m);
+    float sum = (m > -INFINITY) ? sm_ * __expf(m - mx) : 0.f;
+    sum = warp_sum(sum);
+    *mx_out = mx;
+    return mx + __logf(sum);
+}
+
 // --------------------------------------------------- bucket counting sort
 // After bucket_threshold: turn the counts of buckets [0, kNB) into starting
 // positions (exclusive prefix, written back into hist) and copy them to cur.
@@ -177,13 +198,15 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
                                  float *__restrict__ p_c_out, int L, int N_r, int N_c, int K,
                                  float *__restrict__ row_val, int *__restrict__ row_idx,
                                  float *__restrict__ col_val, int *__restrict__ col_idx,
-                                 int nmax, int kmax, size_t warp_words) {
+                                 int nmax, int kmax, size_t warp_words,
+                                 const int *__restrict__ only) {
     extern __shared__ __align__(16) uint32_t smem_u[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     const int wpb = blockDim.x >> 5;
     const int64_t prob = (int64_t)blockIdx.x * wpb + warp;
     if (prob >= 2 * (int64_t)L) return;
+    if (only && only[prob] == 0) return;          // handled by the register kernel
     const int t = (int)(prob >> 1);
     const int axis = (int)(prob & 1);
     const int n = axis ? N_c : N_r;
@@ -206,21 +229,8 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
     bool counted = false;                  // buckets already filled
     const float2 *part = axis ? part_c : part_r;
     if (logsoftmax && part) {
-        // per 64 columns: (max, sum exp(s - max)) from the router GEMM
-        const int nt = 2 * ((n + 2 * kGemmPartCols - 1) / (2 * kGemmPartCols));
-        float m = -INFINITY, sm_ = 0.f;
-        for (int u = lane; u < nt; u += 32) {
-            const float2 pt = part[(size_t)t * nt + u];
-            if (pt.x > -INFINITY) {
-                const float mn = fmaxf(m, pt.x);
-                sm_ = (m > -INFINITY ? sm_ * __expf(m - mn) : 0.f) + pt.y * __expf(pt.x - mn);
-                m = mn;
-            }
-        }
-        const float mx = warp_max(m);
-        float sum = (m > -INFINITY) ? sm_ * __expf(m - mx) : 0.f;
-        sum = warp_sum(sum);
-        const float lse = mx + __logf(sum);
+        float mx;
+        const float lse = lse_from_partials(part, t, n, &mx);
         vmax = mx - lse;                   // the p of the largest logit, same rounding
         if (CAP > 0) {
             for (int b = lane; b < kNB; b += 32) hist[b] = 0u;
@@ -366,6 +376,152 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
         oval[r] = key2f(ku);
         oidx[r] = sel_idx[u];
     }
+}
+
+// ------------------------------------------------- axis top-K, registers
+// Fast path for rows with n % 4 == 0 and n <= 128 * NPL: lane l holds float4
+// number l + 32 j of the row (j < NPL) in registers.  mode 0: the input is
+// p; mode 1: p = s - lse with lse from the GEMM partials; mode 2: p = s - lse
+// computed here.  A row this kernel cannot finish (too few values within 8
+// units of the maximum, or more than CAP candidates) sets flags[row] = 1 and
+// is redone by axis_topk_kernel; every other row gets flags[row] = 0.
+// Shared memory per warp (words): hist[kNB] | cur[kNB] | tmp[CAP] (u64).
+template <int NPL, int CAP>
+__global__ void __launch_bounds__(128)
+axis_topk_reg_kernel(const float *__restrict__ in_r, const float *__restrict__ in_c, int mode,
+                     const float2 *__restrict__ part_r, const float2 *__restrict__ part_c,
+                     float *__restrict__ p_r_out, float *__restrict__ p_c_out, int L, int N_r,
+                     int N_c, int K, float *__restrict__ row_val, int *__restrict__ row_idx,
+                     float *__restrict__ col_val, int *__restrict__ col_idx,
+                     int *__restrict__ flags) {
+    extern __shared__ __align__(16) uint32_t smem_u[];
+    constexpr int kWords = 2 * kNB + 2 * CAP;
+    const int warp = threadIdx.x >> 5;
+    const unsigned lane = lane_id();
+    const int64_t prob = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (prob >= 2 * (int64_t)L) return;
+    const int t = (int)(prob >> 1);
+    const int axis = (int)(prob & 1);
+    const int n = axis ? N_c : N_r;
+    const int n4 = n >> 2;
+    const int kx = K < n ? K : n;
+    const float4 *in4 = reinterpret_cast<const float4 *>((axis ? in_c : in_r) + (size_t)t * n);
+    float *pout = axis ? p_c_out : p_r_out;
+    uint32_t *hist = smem_u + (size_t)warp * kWords;
+    uint32_t *cur = hist + kNB;
+    uint64_t *tmp = reinterpret_cast<uint64_t *>(cur + kNB);
+
+    float4 v[NPL];
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+        const int i4 = (int)lane + 32 * j;
+        v[j] = i4 < n4 ? in4[i4] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+    float lse = 0.f, vmax;
+    if (mode == 1) {
+        float mx;
+        lse = lse_from_partials(axis ? part_c : part_r, t, n, &mx);
+        vmax = mx - lse;
+    } else {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NPL; ++j)
+            mx = fmaxf(fmaxf(mx, fmaxf(v[j].x, v[j].y)), fmaxf(v[j].z, v[j].w));
+        mx = warp_max(mx);
+        if (mode == 2) {
+            float sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < NPL; ++j)
+                if ((int)lane + 32 * j < n4)
+                    sum += __expf(v[j].x - mx) + __expf(v[j].y - mx) + __expf(v[j].z - mx) +
+                           __expf(v[j].w - mx);
+            sum = warp_sum(sum);
+            lse = mx + __logf(sum);
+            vmax = mx - lse;
+        } else {
+            vmax = mx;
+        }
+    }
+    if (mode != 0) {
+#pragma unroll
+        for (int j = 0; j < NPL; ++j) {
+            v[j].x -= lse;
+            v[j].y -= lse;
+            v[j].z -= lse;
+            v[j].w -= lse;
+        }
+        if (pout) {
+            float *prow = pout + (size_t)t * n;
+            const bool vec = (reinterpret_cast<uintptr_t>(prow) & 15u) == 0;
+#pragma unroll
+            for (int j = 0; j < NPL; ++j) {
+                const int i4 = (int)lane + 32 * j;
+                if (i4 < n4) {
+                    if (vec) {
+                        reinterpret_cast<float4 *>(prow)[i4] = v[j];
+                    } else {
+                        prow[4 * i4] = v[j].x;
+                        prow[4 * i4 + 1] = v[j].y;
+                        prow[4 * i4 + 2] = v[j].z;
+                        prow[4 * i4 + 3] = v[j].w;
+                    }
+                }
+            }
+        }
+    }
+    for (int b = lane; b < kNB; b += 32) hist[b] = 0u;
+    __syncwarp();
+    auto count = [&](float p) {
+        const int b = bucket_of(vmax, p);
+        if (b < kNB) atomicAdd(&hist[b], 1u);
+    };
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+        count(v[j].x);
+        count(v[j].y);
+        count(v[j].z);
+        count(v[j].w);
+    }
+    __syncwarp();
+    int bs = 0;
+    const int ncand = bucket_find(hist, kx, &bs);
+    if (ncand < kx || ncand > CAP) {
+        if (lane == 0) flags[prob] = 1;
+        return;
+    }
+    bucket_starts(hist, cur);
+    auto place = [&](float p, int i) {
+        const int b = bucket_of(vmax, p);
+        if (b <= bs) {
+            const uint32_t pos = atomicAdd(&cur[b], 1u);
+            tmp[pos] = ((uint64_t)f2key(p) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
+        }
+    };
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+        const int i = 4 * ((int)lane + 32 * j);
+        place(v[j].x, i);
+        place(v[j].y, i + 1);
+        place(v[j].z, i + 2);
+        place(v[j].w, i + 3);
+    }
+    __syncwarp();
+    float *oval = (axis ? col_val : row_val) + (size_t)t * kx;
+    int *oidx = (axis ? col_idx : row_idx) + (size_t)t * kx;
+    for (int pos = lane; pos < ncand; pos += 32) {
+        const uint64_t k = tmp[pos];
+        const int b = bucket_of(vmax, key2f((uint32_t)(k >> 32)));
+        const int s0 = (int)hist[b];
+        const int s1 = b < bs ? (int)hist[b + 1] : ncand;
+        int r = 0;
+        for (int q = s0; q < s1; ++q) r += tmp[q] > k ? 1 : 0;
+        const int fp = s0 + r;
+        if (fp < kx) {
+            oval[fp] = key2f((uint32_t)(k >> 32));
+            oidx[fp] = (int)(0xffffffffu - (uint32_t)k);
+        }
+    }
+    if (lane == 0) flags[prob] = 0;
 }
 
 // ----------------------------------------------------------- merge top-K
@@ -602,7 +758,7 @@ static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logs
                                  const float *part_r, const float *part_c,
                                  float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
                                  float *row_val, int *row_idx, float *col_val, int *col_idx,
-                                 cudaStream_t st) {
+                                 const int *only, cudaStream_t st) {
     const int nmax = N_r > N_c ? N_r : N_c;
     const int kmax = K < nmax ? K : nmax;
     const size_t area = 2 * (size_t)kmax > 2 * (size_t)CAP ? 2 * (size_t)kmax : 2 * (size_t)CAP;
@@ -626,20 +782,67 @@ static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logs
                                                         reinterpret_cast<const float2 *>(part_c),
                                                         p_r_out, p_c_out, L, N_r, N_c, K, row_val,
                                                         row_idx, col_val, col_idx, nmax, kmax,
-                                                        words);
+                                                        words, only);
     return cudaGetLastError();
+}
+
+template <int NPL, int CAP>
+static cudaError_t launch_axis_reg(const float *in_r, const float *in_c, int mode,
+                                   const float *part_r, const float *part_c, float *p_r_out,
+                                   float *p_c_out, int L, int N_r, int N_c, int K, float *row_val,
+                                   int *row_idx, float *col_val, int *col_idx, int *flags,
+                                   cudaStream_t st) {
+    constexpr int wpb = 4;
+    const size_t smem = (size_t)wpb * (2 * kNB + 2 * CAP) * 4;
+    const int64_t probs = 2 * (int64_t)L;
+    const unsigned grid = (unsigned)((probs + wpb - 1) / wpb);
+    axis_topk_reg_kernel<NPL, CAP><<<grid, 32 * wpb, smem, st>>>(
+        in_r, in_c, mode, reinterpret_cast<const float2 *>(part_r),
+        reinterpret_cast<const float2 *>(part_c), p_r_out, p_c_out, L, N_r, N_c, K, row_val,
+        row_idx, col_val, col_idx, flags);
+    return cudaGetLastError();
+}
+
+template <int CAP>
+static cudaError_t launch_axis_reg_npl(int npl, const float *in_r, const float *in_c, int mode,
+                                       const float *part_r, const float *part_c, float *p_r_out,
+                                       float *p_c_out, int L, int N_r, int N_c, int K,
+                                       float *row_val, int *row_idx, float *col_val,
+                                       int *col_idx, int *flags, cudaStream_t st) {
+#define OMNI_RG(np) return launch_axis_reg<np, CAP>(in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, flags, st);
+    if (npl <= 1) { OMNI_RG(1) }
+    if (npl <= 2) { OMNI_RG(2) }
+    if (npl <= 4) { OMNI_RG(4) }
+    if (npl <= 8) { OMNI_RG(8) }
+    if (npl <= 12) { OMNI_RG(12) }
+    OMNI_RG(16)
+#undef OMNI_RG
 }
 
 cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftmax,
                              const float *part_r, const float *part_c,
                              float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
                              float *row_val, int *row_idx, float *col_val, int *col_idx,
-                             int *status, cudaStream_t st) {
+                             int *flags, int *status, cudaStream_t st) {
     (void)status;
     const int nmax = N_r > N_c ? N_r : N_c;
     const int kmax = K < nmax ? K : nmax;
     const int cap = fast_capacity(kmax);
-#define OMNI_AX(c) return launch_axis_e<c>(in_r, in_c, logsoftmax, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
+    const bool aligned = ((reinterpret_cast<uintptr_t>(in_r) | reinterpret_cast<uintptr_t>(in_c)) & 15u) == 0;
+    const int npl = (nmax / 4 + 31) / 32;
+    const bool reg = flags && aligned && N_r % 4 == 0 && N_c % 4 == 0 && nmax <= 2048 && cap > 0 &&
+                     cap <= 320;
+    const int mode = !logsoftmax ? 0 : (part_r && part_c ? 1 : 2);
+    cudaError_t e;
+    const int *only = nullptr;
+    if (reg) {
+        if (cap <= 96) e = launch_axis_reg_npl<96>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, flags, st);
+        else if (cap <= 192) e = launch_axis_reg_npl<192>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, flags, st);
+        else e = launch_axis_reg_npl<320>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, flags, st);
+        if (e != cudaSuccess) return e;
+        only = flags;                      // the general kernel redoes the flagged rows
+    }
+#define OMNI_AX(c) return launch_axis_e<c>(in_r, in_c, logsoftmax, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, only, st);
     if (cap == 0) { OMNI_AX(0) }
     if (cap <= 96) { OMNI_AX(96) }
     if (cap <= 192) { OMNI_AX(192) }
