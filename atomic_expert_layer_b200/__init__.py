@@ -12,7 +12,8 @@ import torch
 
 from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_Y_ACCUMULATE, OmniError, load,  # noqa: F401
                    expert_workspace, omni_expert_workspace_size, omni_get_device_status,
-                   omni_grouped_expert_fwd, omni_routed_fwd, omni_router_topk,
+                   omni_grouped_expert_fwd, omni_grouped_expert_fwd_noalloc, omni_routed_fwd,
+                   omni_router_topk,
                    omni_router_workspace_size, omni_schedule, omni_schedule_workspace_size,
                    omni_selftest_wait_timeout,
                    omni_workspace_size, router_workspace, schedule_workspace, workspace)
@@ -20,7 +21,7 @@ from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_Y_ACCUMULATE, OmniError, load, 
 __all__ = [
     "load", "OmniError", "OMNI_ROUTER_LOGPROBS_IN", "OMNI_Y_ACCUMULATE",
     "omni_workspace_size", "omni_router_topk", "omni_schedule", "omni_grouped_expert_fwd",
-    "omni_routed_fwd", "omni_get_device_status", "workspace",
+    "omni_routed_fwd", "omni_get_device_status", "workspace", "omni_grouped_expert_fwd_noalloc",
     "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd",
 ]
 

@@ -40,6 +40,8 @@ SIGNATURES = {
                         _I),
     "omni_get_device_status": ([_P, _Z, _P, ctypes.POINTER(ctypes.c_int)], _I),
     "omni_selftest_wait_timeout": ([_P, _Z, _I, _P], _I),
+    "omni_grouped_expert_fwd_noalloc": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                                         _P, _U, _P], _I),
 }
 
 _lib = None
@@ -178,3 +180,14 @@ def omni_get_device_status(ws, stream=None) -> int:
 def omni_selftest_wait_timeout(ws, limit_ms: int, stream=None) -> None:
     rc = load().omni_selftest_wait_timeout(_ptr(ws), ws.numel(), limit_ms, _stream(stream))
     _check("omni_selftest_wait_timeout", rc)
+
+
+def omni_grouped_expert_fwd_noalloc(x, W, V, L, d, K, N, B, task_token, task_expert, task_gate,
+                                    group_offsets, active_groups, num_active, y, flags,
+                                    stream=None):
+    """The grouped expert call without a workspace (scratch inside the library)."""
+    rc = load().omni_grouped_expert_fwd_noalloc(
+        _ptr(x), _ptr(W), _ptr(V), L, d, K, N, B, _ptr(task_token), _ptr(task_expert),
+        _ptr(task_gate), _ptr(group_offsets), _ptr(active_groups), _ptr(num_active), _ptr(y),
+        flags, _stream(stream))
+    _check("omni_grouped_expert_fwd_noalloc", rc)

@@ -189,6 +189,34 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                     unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
 
 /*
+ * omni_grouped_expert_fwd without a workspace, for callers that cannot
+ * allocate device memory when they run the layer (a serving runtime whose
+ * memory is planned once at start-up, code where cudaMalloc is not allowed).
+ * The pages have no counterpart; it is a deployment convenience.
+ * Same arguments and result as omni_grouped_expert_fwd, minus ws / ws_bytes.
+ * Its scratch is a fixed array inside the library (about 2 MB on every GPU
+ * that loads it, held until the process exits), so:
+ *   - sizes are limited to L <= 16384 tokens and L * K <= 262144 tasks
+ *     (OMNI_ERR_UNSUPPORTED beyond), besides the limits of the workspace call;
+ *   - every call on a device shares the array: calls that overlap on the GPU
+ *     (different streams, or different host threads) race and must not be
+ *     issued; the array keeps the last call's contents, and the call clears
+ *     what has to start at zero itself;
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing a stream into a CUDA graph;
+ *   - device-detected problems are recorded in the array's own status word,
+ *     which omni_get_device_status cannot read.
+ * No device memory is allocated or freed.
+ */
+int omni_grouped_expert_fwd_noalloc(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
+                                    int L, int d, int K, int N, int B,
+                                    const int32_t *task_token, const int32_t *task_expert,
+                                    const float *task_gate, const int32_t *group_offsets,
+                                    const int32_t *active_groups, const int32_t *num_active,
+                                    float *y, unsigned flags, omni_stream_t stream);
+
+/*
  * Diagnostic, not part of the layer: launches one CTA that waits on a
  * shared-memory barrier nothing ever arrives at, through the same bounded
  * wait the pipelined kernels use, with its limit set to `limit_ms`
