@@ -170,12 +170,13 @@ class ClockSampler:
 
 
 def traffic_from_profile(kernel_src: str) -> float | None:
-    """DRAM bytes per launch of the grouped expert kernel from the committed
-    ncu summary, if it was taken on the current kernel source."""
+    """DRAM bytes (read + write) of one grouped expert stage call (both
+    kernels) from the committed ncu summary, if it was taken on the current
+    kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get("grouped_expert_kernel")
+    d = json.load(open(p)).get("grouped_expert_stage")
     if not d:
         return None
     sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
@@ -445,7 +446,7 @@ def time_oracle(cfg, n_tokens: int, seed: int = 0, repeats: int = 1) -> dict:
             "cores": oracle.max_threads()}
 
 
-def cpu_baseline(cfg, budget_s: float = 15.0) -> dict:
+def cpu_baseline(cfg, budget_s: float = 25.0) -> dict:
     """The oracle on a bounded sample: the first n tokens (n sized to about
     budget_s of CPU work), or all L tokens repeated until about budget_s."""
     probe = min(cfg.L, 64)
