@@ -43,6 +43,10 @@ bool make_sizes(int L, int d, int N_r, int N_c, int K, int B, Sizes *sz) {
     sz->Kc = K < N_c ? K : N_c;
     sz->C = merge_candidates(K, sz->Kr, sz->Kc);
     sz->ntiles = (sz->M + kSortTile - 1) / kSortTile;
+    int nbits = 0;
+    while (nbits < 31 && ((int64_t)1 << nbits) < sz->G) ++nbits;
+    sz->qbits = nbits;
+    sz->passes = (nbits + 7) / 8;
     return true;
 }
 
@@ -53,6 +57,15 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
     auto take = [&](size_t bytes) { const size_t at = o; o = align256(o + bytes); return at; };
     const size_t L = (size_t)sz.L, M = (size_t)sz.M, G = (size_t)sz.G;
     w.hdr = take(sizeof(WsHeader));
+    // counters that must be zero when a call starts: right after the header
+    if (regions & kRegSched) {
+        w.z_cnt = take(4 * G);
+        w.z_ndist = take(4);
+        w.bitmap = take(4 * (size_t)((sz.N + 31) / 32));
+        w.hist = take(4 * 256 * (size_t)sz.ntiles * (size_t)sz.passes);   // one per radix pass
+    }
+    if (regions & kRegExpert) w.tok_count = take(4 * L);
+    w.zero_end = o;
     if (regions & kRegRouter) {
         w.s_r = take(4 * L * sz.N_r);
         w.s_c = take(4 * L * sz.N_c);
@@ -70,8 +83,6 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
     if (regions & kRegSched) {
         w.a_tok = take(4 * M); w.a_exp = take(4 * M); w.a_gate = take(4 * M);
         w.b_tok = take(4 * M); w.b_exp = take(4 * M); w.b_gate = take(4 * M);
-        w.bitmap = take(4 * (size_t)((sz.N + 31) / 32));
-        w.hist = take(4 * 4 * 256 * (size_t)sz.ntiles);      // one per radix pass (<= 4)
     }
     if (regions & kRegSchedOut) {
         w.t_tok = take(4 * M); w.t_exp = take(4 * M); w.t_gate = take(4 * M);
@@ -81,10 +92,7 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.n_act = take(4);
         w.n_dist = take(4);
     }
-    if (regions & kRegExpert) {
-        w.tok_count = take(4 * L);
-        w.tok_slots = take(8 * M);
-    }
+    if (regions & kRegExpert) w.tok_slots = take(8 * M);
     w.total = o;
     return w;
 }
@@ -127,8 +135,9 @@ int check_ws(const Sizes &sz, unsigned regions, void *ws, size_t ws_bytes, WsLay
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? OMNI_OK : OMNI_ERR_CUDA; }
 
-int reset_header(void *ws, cudaStream_t st) {
-    return cuda_rc(cudaMemsetAsync(ws, 0, sizeof(WsHeader), st));
+// Clears the status word and the counters the call's kernels accumulate into.
+int reset_workspace(void *ws, const WsLayout &lay, cudaStream_t st) {
+    return cuda_rc(cudaMemsetAsync(ws, 0, lay.zero_end, st));
 }
 
 int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c,
@@ -139,6 +148,7 @@ int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c
     float *row_val = ws_at<float>(ws, lay.row_val), *col_val = ws_at<float>(ws, lay.col_val);
     int *row_idx = ws_at<int>(ws, lay.row_idx), *col_idx = ws_at<int>(ws, lay.col_idx);
     int *row_flags = ws_at<int>(ws, lay.flags);
+    const float *dead_r = nullptr, *dead_c = nullptr;
     cudaError_t e;
     if (flags & OMNI_ROUTER_LOGPROBS_IN) {
         e = launch_axis_topk(p_r, p_c, false, nullptr, nullptr, nullptr, nullptr, sz.L, sz.N_r,
@@ -151,10 +161,12 @@ int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c
         if (e != cudaSuccess) return OMNI_ERR_CUDA;
         e = launch_axis_topk(s_r, s_c, true, part_r, part_c, p_r, p_c, sz.L, sz.N_r, sz.N_c,
                              sz.K, row_val, row_idx, col_val, col_idx, row_flags, status, st);
+        dead_r = s_r;                      // the logits are dead after the axis kernels
+        dead_c = s_c;
     }
     if (e != cudaSuccess) return OMNI_ERR_CUDA;
     e = launch_merge_topk(row_val, row_idx, col_val, col_idx, sz.L, sz.N_c, sz.K, sz.Kr, sz.Kc,
-                          sz.C, idx, score, gate, st);
+                          sz.C, idx, score, gate, dead_r, dead_c, sz.N_r, st);
     return cuda_rc(e);
 }
 
@@ -228,7 +240,7 @@ int omni_router_topk(const omni_bf16 *x, const omni_bf16 *W_r, const omni_bf16 *
     WsLayout lay;
     if ((rc = check_ws(sz, kRegRouter, ws, ws_bytes, &lay))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = reset_header(ws, st))) return rc;
+    if ((rc = reset_workspace(ws, lay, st))) return rc;
     return router_topk_impl(x, W_r, W_c, sz, p_r, p_c, idx, score, gate, flags, ws, lay, st);
 }
 
@@ -247,7 +259,7 @@ int omni_schedule(const int32_t *idx, const float *gate, int L, int K, int N, in
     WsLayout lay;
     if ((rc = check_ws(sz, kRegSched, ws, ws_bytes, &lay))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = reset_header(ws, st))) return rc;
+    if ((rc = reset_workspace(ws, lay, st))) return rc;
     return cuda_rc(launch_schedule(idx, gate, sz, task_token, task_expert, task_gate,
                                    group_offsets, group_counts, active_groups, num_active,
                                    num_distinct, ws, lay, st));
@@ -272,7 +284,7 @@ int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_b
     WsLayout lay;
     if ((rc = check_ws(sz, kRegExpert, ws, ws_bytes, &lay))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = reset_header(ws, st))) return rc;
+    if ((rc = reset_workspace(ws, lay, st))) return rc;
     return cuda_rc(launch_grouped_expert(x, W, V, sz, task_token, task_expert, task_gate, y,
                                          (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st));
 }
@@ -292,7 +304,7 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     WsLayout lay;
     if ((rc = check_ws(sz, kRegAll, ws, ws_bytes, &lay))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = reset_header(ws, st))) return rc;
+    if ((rc = reset_workspace(ws, lay, st))) return rc;
     int32_t *idx = ws_at<int32_t>(ws, lay.idx);
     float *score = ws_at<float>(ws, lay.score), *gate = ws_at<float>(ws, lay.gate);
     rc = router_topk_impl(x, W_r, W_c, sz, nullptr, nullptr, idx, score, gate,
@@ -323,8 +335,7 @@ int omni_selftest_wait_timeout(void *ws, size_t ws_bytes, int limit_ms, omni_str
         return OMNI_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return OMNI_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    int rc = reset_header(ws, st);
-    if (rc) return rc;
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return OMNI_ERR_CUDA;
     selftest_wait_kernel<<<1, 32, 0, st>>>(ws_at<int>(ws, 0), (uint64_t)limit_ms * 1000000ull);
     return cuda_rc(cudaGetLastError());
 }

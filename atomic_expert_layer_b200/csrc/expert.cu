@@ -86,6 +86,29 @@ struct CombineCfg {
 // warp's cp.async ring, kStages-1 tasks ahead; p = g * SiLU(x . w) is written
 // with the expert id into the token's slot.  Inside a group the tasks of one
 // expert are close together, so a repeated W row is normally served by L2.
+// Consecutive tasks of one token (a token meets ~1.4 experts per group) load
+// and unpack its x row once.  Each lane keeps its partial dot products of 8
+// tasks and the warp reduces the 8 together (a transposed butterfly), so the
+// reduction costs about one shuffle per task instead of five.
+constexpr int kGateBlock = 8;             // tasks reduced together
+
+// bf16 pair (one 32-bit word) -> the two fp32 values, exactly
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// (a0, a1) += (x0, x1) * (w0, w1) as one packed fp32x2 FMA (round to nearest)
+__device__ __forceinline__ void fma_f32x2(float &a0, float &a1, float x0, float x1, float w0,
+                                          float w1) {
+    asm("{\n\t.reg .b64 a, x, w;\n\t"
+        "mov.b64 a, {%0, %1};\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 w, {%4, %5};\n\t"
+        "fma.rn.f32x2 a, x, w, a;\n\t"
+        "mov.b64 {%0, %1}, a;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(x0), "f"(x1), "f"(w0), "f"(w1));
+}
+
 template <int VPL>
 __global__ void __launch_bounds__(32 * GateCfg<VPL>::kWarps)
 group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W, int L, int N,
@@ -96,12 +119,16 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
     constexpr int D = 256 * VPL;
     constexpr int S = Cfg::kStages;
     constexpr int RB = Cfg::kRowBytes;
+    constexpr int U = kGateBlock;
     static_assert(S - 1 <= kChunk, "prefetch stays within two metadata chunks");
+    static_assert(kChunk % U == 0 && U == 8, "blocks of 8 tasks tile a metadata chunk");
     extern __shared__ __align__(16) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     uint8_t *wring = smem + (size_t)warp * 2 * S * RB;
     uint8_t *xring = wring + S * RB;
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     const int64_t gw = (int64_t)blockIdx.x * Cfg::kWarps + warp;
     const int64_t a0 = gw * per_warp;
@@ -130,56 +157,119 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
     float cg, ng;
     load_meta(0, ct, ce, cg, cs);
     load_meta(kChunk, nt, ne, ng, ns);
-    // task i (ring slot i % S) whose metadata is entry rel of the current
-    // (rel < 32) or the next (32 <= rel < 64) chunk
+    // Rows of task i into ring slot i % S (rel: its entry in the current
+    // (rel < 32) or next (32 <= rel < 64) chunk).  The x row is copied only
+    // when the token differs from the previous task's; the consumer makes the
+    // same comparison.
+    int x_issued = -1;
     auto issue = [&](int i, int rel) {
         const bool same = rel < kChunk;
         const int src = rel % kChunk;
         const int t = __shfl_sync(0xffffffffu, same ? ct : nt, src);
         const int e = __shfl_sync(0xffffffffu, same ? ce : ne, src);
         row_async<VPL>(wring + (i % S) * RB, W + (size_t)e * D, lane);
-        row_async<VPL>(xring + (i % S) * RB, x + (size_t)t * D, lane);
+        if (t != x_issued) {
+            row_async<VPL>(xring + (i % S) * RB, x + (size_t)t * D, lane);
+            x_issued = t;
+        }
     };
 #pragma unroll 1
     for (int i = 0; i < S - 1; ++i) {
         if (i < n) issue(i, i);
         cp_async_commit();
     }
-    int base = 0;                   // first task of the current chunk
-    for (int i = 0; i < n; ++i) {
-        if (i - base == kChunk) {   // move to the next chunk of metadata
-            base += kChunk;
+    float xf[8 * VPL];              // the current token's x slice, unpacked
+    int x_have = -1;
+#pragma unroll 1
+    for (int base = 0; base < n; base += kChunk) {
+        if (base > 0) {             // move to the next chunk of metadata
             ct = nt; ce = ne; cg = ng; cs = ns;
             load_meta(base + kChunk, nt, ne, ng, ns);
         }
-        cp_async_wait<S - 2>();     // task i's rows have landed
-        __syncwarp();
-        const int ip = i + S - 1;
-        if (ip < n) issue(ip, ip - base);
-        cp_async_commit();
-        const uint4 *wr = reinterpret_cast<const uint4 *>(wring + (i % S) * RB);
-        const uint4 *xr = reinterpret_cast<const uint4 *>(xring + (i % S) * RB);
-        float h = 0.f;
+#pragma unroll 1
+        for (int b0 = 0; b0 < kChunk && base + b0 < n; b0 += U) {
+            float hp[U];
 #pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-            float xf[8], wf[8];
-            bf16x8_to_f32(xr[v * 32 + lane], xf);
-            bf16x8_to_f32(wr[v * 32 + lane], wf);
+            for (int j = 0; j < U; ++j) {
+                const int i = base + b0 + j;
+                hp[j] = 0.f;
+                if (i < n) {                               // the same in every lane
+                    cp_async_wait<S - 2>();                // task i's rows have landed
+                    __syncwarp();
+                    const int ip = i + S - 1;
+                    if (ip < n) issue(ip, ip - base);
+                    cp_async_commit();
+                    const int t = __shfl_sync(0xffffffffu, ct, b0 + j);
+                    if (t != x_have) {
+                        const uint4 *xr = reinterpret_cast<const uint4 *>(xring + (i % S) * RB);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) h = fmaf(xf[c], wf[c], h);
-        }
-        h = warp_sum(h);
-        const int src = i - base;
-        const int t = __shfl_sync(0xffffffffu, ct, src);
-        const int e = __shfl_sync(0xffffffffu, ce, src);
-        const float g = __shfl_sync(0xffffffffu, cg, src);
-        const int slot = __shfl_sync(0xffffffffu, cs, src);
-        if (lane == 0) {
-            const float p = g * (h / (1.f + __expf(-h)));
-            if (slot < K)
-                tok_slots[(size_t)t * K + slot] = make_int2(e, __float_as_int(p));
-            else
-                set_status(status, OMNI_DEV_BAD_SCHEDULE);
+                        for (int v = 0; v < VPL; ++v) {
+                            const uint4 u = xr[v * 32 + lane];
+                            const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                xf[8 * v + 2 * q] = bf_lo(wd[q]);
+                                xf[8 * v + 2 * q + 1] = bf_hi(wd[q]);
+                            }
+                        }
+                        x_have = t;
+                    }
+                    const uint4 *wr = reinterpret_cast<const uint4 *>(wring + (i % S) * RB);
+                    float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll
+                    for (int v = 0; v < VPL; ++v) {
+                        const uint4 u = wr[v * 32 + lane];
+                        fma_f32x2(c0, c1, xf[8 * v + 0], xf[8 * v + 1], bf_lo(u.x), bf_hi(u.x));
+                        fma_f32x2(c2, c3, xf[8 * v + 2], xf[8 * v + 3], bf_lo(u.y), bf_hi(u.y));
+                        fma_f32x2(c0, c1, xf[8 * v + 4], xf[8 * v + 5], bf_lo(u.z), bf_hi(u.z));
+                        fma_f32x2(c2, c3, xf[8 * v + 6], xf[8 * v + 7], bf_lo(u.w), bf_hi(u.w));
+                    }
+                    hp[j] = (c0 + c1) + (c2 + c3);
+                }
+            }
+            // Transposed butterfly: after the three exchanges lane l holds
+            // the sum over lanes l ^ {4, 8, 16} of task (l >> 2) & 7's
+            // partials; two more exchanges add lanes l ^ {1, 2}.
+            {
+                const bool up = (lane & 16u) != 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float send = up ? hp[k] : hp[k + 4];
+                    const float keep = up ? hp[k + 4] : hp[k];
+                    hp[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+            }
+            {
+                const bool up = (lane & 8u) != 0;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const float send = up ? hp[k] : hp[k + 2];
+                    const float keep = up ? hp[k + 2] : hp[k];
+                    hp[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+            }
+            float h;
+            {
+                const bool up = (lane & 4u) != 0;
+                const float send = up ? hp[0] : hp[1];
+                const float keep = up ? hp[1] : hp[0];
+                h = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+            }
+            h += __shfl_xor_sync(0xffffffffu, h, 2);
+            h += __shfl_xor_sync(0xffffffffu, h, 1);
+            const int jt = (int)((lane >> 2) & 7u);
+            const int src = b0 + jt;
+            const int t = __shfl_sync(0xffffffffu, ct, src);
+            const int e = __shfl_sync(0xffffffffu, ce, src);
+            const float g = __shfl_sync(0xffffffffu, cg, src);
+            const int slot = __shfl_sync(0xffffffffu, cs, src);
+            if ((lane & 3u) == 0 && base + src < n) {
+                const float p = g * (h / (1.f + __expf(-h)));
+                if (slot < K)
+                    tok_slots[(size_t)t * K + slot] = make_int2(e, __float_as_int(p));
+                else
+                    set_status(status, OMNI_DEV_BAD_SCHEDULE);
+            }
         }
     }
     cp_async_wait<0>();
@@ -200,6 +290,8 @@ token_combine_kernel(const uint16_t *__restrict__ V, int L, int N, int K,
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     uint8_t *ring = smem + (size_t)warp * S * RB;
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int nwarps = gridDim.x * Cfg::kWarps;
     for (int t = blockIdx.x * Cfg::kWarps + warp; t < L; t += nwarps) {
         int n = tok_count[t];
@@ -286,7 +378,6 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     const int sms = device_sm_count();
-    if ((e = cudaMemsetAsync(tok_count, 0, sizeof(int) * (size_t)sz.L, st)) != cudaSuccess) return e;
     {
         int per_sm = (227 * 1024) / G::kSmem;
         if (per_sm < 1) per_sm = 1;
@@ -296,10 +387,10 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
         if (per_warp < 32) per_warp = 32;
         const int64_t needed = (sz.M + per_warp - 1) / per_warp;      // warps with work
         const int grid = (int)((needed + G::kWarps - 1) / G::kWarps);
-        group_gate_kernel<VPL><<<grid, 32 * G::kWarps, G::kSmem, st>>>(
-            x, W, sz.L, (int)sz.N, sz.K, (int)sz.M, (int)per_warp, tt, te, tg, tok_count,
-            tok_slots, status);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch(group_gate_kernel<VPL>, dim3(grid), dim3(32 * G::kWarps), G::kSmem, st, x, W,
+                   sz.L, (int)sz.N, sz.K, (int)sz.M, (int)per_warp, tt, te, tg, tok_count,
+                   tok_slots, status);
+        if (e != cudaSuccess) return e;
     }
     {
         int per_sm = (227 * 1024) / C::kSmem;
@@ -308,10 +399,11 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
         int64_t grid = (int64_t)sms * per_sm;
         const int64_t need = (sz.L + C::kWarps - 1) / C::kWarps;
         if (grid > need) grid = need;
-        token_combine_kernel<VPL><<<(unsigned)grid, 32 * C::kWarps, C::kSmem, st>>>(
-            V, sz.L, (int)sz.N, sz.K, tok_count, tok_slots, y, accumulate ? 1 : 0, status);
+        e = launch(token_combine_kernel<VPL>, dim3((unsigned)grid), dim3(32 * C::kWarps), C::kSmem,
+                   st, V, sz.L, (int)sz.N, sz.K, (const int *)tok_count,
+                   (const int2 *)tok_slots, y, accumulate ? 1 : 0, status);
     }
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace

@@ -87,8 +87,10 @@ extern "C" int omni_grouped_expert_fwd_noalloc(
     lay.hdr = 0;
     lay.tok_count = kOffCount;
     lay.tok_slots = kOffSlots;
+    lay.zero_end = kOffCount + 4 * (size_t)L;
     lay.total = kNoAllocBytes;
-    if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), st) != cudaSuccess) return OMNI_ERR_CUDA;
+    // status word and this call's slot counters
+    if (cudaMemsetAsync(scratch, 0, lay.zero_end, st) != cudaSuccess) return OMNI_ERR_CUDA;
     const cudaError_t e = launch_grouped_expert(x, W, V, sz, task_token, task_expert, task_gate,
                                                 y, (flags & OMNI_Y_ACCUMULATE) != 0, scratch, lay,
                                                 st);

@@ -1,10 +1,13 @@
 // omni_common.cuh -- device helpers shared by the sm_100a kernels of libomni:
-// the workspace status word, bounded mbarrier waits, bulk (TMA) copies and
-// order-preserving float keys.  Nothing here is method arithmetic.
+// the workspace status word, bounded mbarrier waits, order-preserving float
+// keys, warp reductions and the launch helper (programmatic dependent
+// launch).  Nothing here is method arithmetic.
 #pragma once
 
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <utility>
 
 #include "omni.h"
 
@@ -15,9 +18,7 @@ namespace omni {
 // status (OMNI_DEV_*), the rest are counters used by individual kernels.
 struct WsHeader {
     int status;
-    int item_counter;     // grouped-expert kernel: next work item to claim
-    int total_items;      // grouped-expert kernel: number of work items
-    int pad[61];
+    int pad[63];
 };
 static_assert(sizeof(WsHeader) == 256, "header must stay 256 bytes");
 
@@ -112,32 +113,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *s
     return mbar_wait_limit(bar, parity, status, kWaitLimitNs);
 }
 
-// ------------------------------------------------------------- bulk copies
-// L2 policy for data that is read once (expert rows): evict first.
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-// Contiguous global -> shared copy through the bulk-copy (TMA) engine,
-// completing `bytes` of transaction count on `bar`.  Both addresses 16-byte
-// aligned, bytes a multiple of 16.  No multicast.
-__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes,
-                                         uint64_t *bar, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1], %2, [%3], %4;"
-        ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
-// ------------------------------------------------------------ reductions
-__device__ __forceinline__ void red_add_v4(float *gaddr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
-                 ::"l"(gaddr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-
+// ------------------------------------------------------------ warp helpers
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -162,6 +138,38 @@ __device__ __forceinline__ int warp_iscan(int v) {
         if (l >= (unsigned)o) v += n;
     }
     return v;
+}
+
+// ------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialisation (launch() below): its CTAs may be scheduled while the
+// previous kernel in the stream is still finishing.  Each kernel therefore
+// calls grid_dependency_wait() in every thread, before its first access to
+// global memory that earlier work in the stream writes or reads; since every
+// kernel waits, a kernel's completion implies that of all earlier ones.
+// grid_dependents_launch() lets the next kernel's CTAs start their prologue
+// as this kernel's CTAs leave the SMs (it carries no memory ordering).
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace omni

@@ -17,18 +17,23 @@ struct Sizes {
     int Kr, Kc;          // row / column candidates: min(K, N_r), min(K, N_c)
     int C;               // merge candidates: cells (a, b) with (a+1)(b+1) <= K
     int64_t ntiles;      // radix tiles
+    int qbits, passes;   // bits of the largest group id G - 1; radix passes of <= 8 bits
 };
 
 struct WsLayout {
     size_t hdr, s_r, s_c, part_r, part_c, flags, row_val, row_idx, col_val, col_idx, idx, score, gate;
     size_t a_tok, a_exp, a_gate, b_tok, b_exp, b_gate, t_tok, t_exp, t_gate;
     size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, tok_count, tok_slots;
+    size_t z_cnt, z_ndist;   // schedule counters (workspace copies)
+    size_t zero_end;         // [0, zero_end) must be zero when a call starts
     size_t total;
 };
 
-// Workspace regions.  Every call puts the 256-byte header at offset 0 and then
-// only the regions it uses, in this order; the whole routed forward uses all
-// of them, so omni_workspace_size (the full layout) covers every call.
+// Workspace regions.  Every call puts the 256-byte header at offset 0, then
+// the counters of its regions that must start at zero (so one memset of
+// [0, zero_end) clears them with the status word), then the rest of its
+// regions in this order; the whole routed forward uses all of them, so
+// omni_workspace_size (the full layout) covers every call.
 enum WsRegion : unsigned {
     kRegRouter = 1u,      // s_r, s_c, axis candidates, idx / score / gate
     kRegSched = 2u,       // sort buffers, expert bitmap, radix histograms
@@ -62,18 +67,21 @@ cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftm
                              float *p_r_out, float *p_c_out, int L, int N_r, int N_c, int K,
                              float *row_val, int *row_idx, float *col_val, int *col_idx,
                              int *flags, int *status, cudaStream_t st);
+// dead_r / dead_c: the router GEMM's logits in the workspace, dropped from
+// L2 once read (null: nothing is dropped, e.g. caller-owned log-probabilities)
 cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
                               const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
-                              int32_t *idx, float *score, float *gate, cudaStream_t st);
+                              int32_t *idx, float *score, float *gate, const float *dead_r,
+                              const float *dead_c, int N_r, cudaStream_t st);
 
-// ---- schedule
+// ---- schedule (expects [0, lay.zero_end) of ws zeroed)
 cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &sz,
                             int32_t *task_token, int32_t *task_expert, float *task_gate,
                             int32_t *group_offsets, int32_t *group_counts,
                             int32_t *active_groups, int32_t *num_active, int32_t *num_distinct,
                             void *ws, const WsLayout &lay, cudaStream_t st);
 
-// ---- grouped expert stage
+// ---- grouped expert stage (expects the per-token slot counters zeroed)
 cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const uint16_t *V,
                                   const Sizes &sz, const int32_t *task_token,
                                   const int32_t *task_expert, const float *task_gate,

@@ -149,6 +149,9 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // everything above touches only this CTA's shared memory and TMEM
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -352,10 +355,9 @@ cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *W_r, const uin
     const int ntiles = ((L + BM - 1) / BM) * (ntile_r + ntile_c);
     const int sms = device_sm_count();
     const int grid = ntiles < sms ? ntiles : sms;
-    router_gemm_kernel<<<grid, kThreads, smem, st>>>(
-        tm_x, tm_wr, tm_wc, s_r, s_c, reinterpret_cast<float2 *>(part_r),
-        reinterpret_cast<float2 *>(part_c), L, d, N_r, N_c, ntile_r, ntile_c, status);
-    return cudaGetLastError();
+    return launch(router_gemm_kernel, dim3(grid), dim3(kThreads), (size_t)smem, st, tm_x, tm_wr,
+                  tm_wc, s_r, s_c, reinterpret_cast<float2 *>(part_r),
+                  reinterpret_cast<float2 *>(part_c), L, d, N_r, N_c, ntile_r, ntile_c, status);
 }
 
 }  // namespace omni

@@ -46,6 +46,8 @@ __global__ void sched_prepare_kernel(const int32_t *__restrict__ idx,
                                      int32_t *__restrict__ hist0, int64_t ntiles, uint32_t dmask0,
                                      int *status) {
     extern __shared__ int32_t sh_e[];
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     const int t = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -114,8 +116,64 @@ constexpr int kScanTile = 4096;            // elements per tile: 1024 threads x 
 // current tile is scanned) and staged through shared memory so each thread
 // owns 4 consecutive elements.  If `tail` is non-null the total is written
 // there.
+constexpr int kFastPer = 16;                               // elements per thread
+constexpr int64_t kFastScan = 1024 * kFastPer;             // one-shot scan limit
+
+// One-shot scan of n <= kFastScan ints by 1024 threads.  Warp w owns the
+// contiguous chunk [512 w, 512 w + 512); lane l holds its elements
+// 32 k + l (k < 16), so every load and store is a coalesced 128-byte row.
+// Loads the chunk into v, scans the warp totals across the CTA and returns
+// the exclusive prefix of the warp's first element; *total is the sum of all
+// n.  With act_total, the count of positive elements is scanned the same way
+// (*act_run0 = exclusive count before the warp, *act_total = all).
+__device__ __forceinline__ int fast_load_scan(const int32_t *a, int64_t n, int *v, int *sh32,
+                                              int *total, int *act_run0, int *act_total) {
+    const int warp = threadIdx.x >> 5;
+    const unsigned lane = lane_id();
+    const int64_t base = (int64_t)warp * (32 * kFastPer);
+    int sum = 0, act = 0;
+#pragma unroll
+    for (int k = 0; k < kFastPer; ++k) {
+        const int64_t i = base + k * 32 + lane;
+        v[k] = i < n ? a[i] : 0;
+        sum += v[k];
+        act += v[k] > 0;
+    }
+    sum = warp_isum(sum);
+    int run0 = block_exclusive_scan(lane == 0 ? sum : 0, sh32, total);
+    run0 = __shfl_sync(0xffffffffu, run0, 0);
+    if (act_total) {
+        act = warp_isum(act);
+        int ar = block_exclusive_scan(lane == 0 ? act : 0, sh32, act_total);
+        *act_run0 = __shfl_sync(0xffffffffu, ar, 0);
+    }
+    return run0;
+}
+
+// Writes the exclusive scan of the chunk loaded by fast_load_scan.
+__device__ __forceinline__ void fast_store_scan(int32_t *a, int64_t n, const int *v, int run) {
+    const int warp = threadIdx.x >> 5;
+    const unsigned lane = lane_id();
+    const int64_t base = (int64_t)warp * (32 * kFastPer);
+#pragma unroll
+    for (int k = 0; k < kFastPer; ++k) {
+        const int incl = warp_iscan(v[k]);
+        const int64_t i = base + k * 32 + lane;
+        if (i < n) a[i] = run + incl - v[k];
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+}
+
 __device__ void cta_exclusive_scan(int32_t *a, int64_t n, int32_t *tail, int *tile, int *sh32) {
     const int tid = threadIdx.x;
+    if (n <= kFastScan) {
+        int v[kFastPer];
+        int total;
+        const int run0 = fast_load_scan(a, n, v, sh32, &total, nullptr, nullptr);
+        fast_store_scan(a, n, v, run0);
+        if (tail && tid == 0) *tail = total;
+        return;
+    }
     int carry = 0;
     int nx[4];
 #pragma unroll
@@ -156,19 +214,49 @@ __device__ void cta_exclusive_scan(int32_t *a, int64_t n, int32_t *tail, int *ti
 }
 
 // ----------------------------------------------------- 2. group scan
-// CTA 0: group offsets (exclusive scan of counts), active groups, distinct
-// experts.  CTA 1 (if a radix pass follows): exclusive scan of the first
-// pass's digit-major histogram.
+// CTA 0: group offsets (exclusive scan of the counts), the caller's copy of
+// the counts, active groups, the distinct-expert count.  CTA 1 (if a radix
+// pass follows): exclusive scan of the first pass's digit-major histogram.
 __global__ void __launch_bounds__(1024) sched_scan_kernel(
-    const int32_t *__restrict__ counts, int64_t G, int32_t *__restrict__ offsets,
-    int32_t *__restrict__ active, int32_t *__restrict__ num_active,
+    const int32_t *__restrict__ counts, int64_t G, int32_t *__restrict__ counts_out,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ active, int32_t *__restrict__ num_active,
+    const int32_t *__restrict__ ndist_acc, int32_t *__restrict__ num_distinct,
     int32_t *__restrict__ hist0, int64_t nhist) {
     __shared__ int tile[kScanTile];
     __shared__ int tile2[kScanTile];
     __shared__ int sh32[33];
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int tid = threadIdx.x;
     if (blockIdx.x == 1) {
         cta_exclusive_scan(hist0, nhist, nullptr, tile, sh32);
+        return;
+    }
+    if (tid == 0) *num_distinct = *ndist_acc;
+    if (G <= kFastScan) {
+        int v[kFastPer];
+        int total, atotal, arun;
+        int run = fast_load_scan(counts, G, v, sh32, &total, &arun, &atotal);
+        const int warp = tid >> 5;
+        const unsigned lane = lane_id();
+        const int64_t base = (int64_t)warp * (32 * kFastPer);
+#pragma unroll
+        for (int k = 0; k < kFastPer; ++k) {
+            const int incl = warp_iscan(v[k]);
+            const unsigned act = __ballot_sync(0xffffffffu, v[k] > 0);
+            const int64_t g = base + k * 32 + lane;
+            if (g < G) {
+                offsets[g] = run + incl - v[k];
+                counts_out[g] = v[k];
+                if (v[k] > 0) active[arun + __popc(act & lanemask_lt())] = (int32_t)g;
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
+            arun += __popc(act);
+        }
+        if (tid == 0) {
+            offsets[G] = total;
+            *num_active = atotal;
+        }
         return;
     }
     int carry = 0, acarry = 0;
@@ -209,7 +297,10 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(
         __syncthreads();
         for (int k = 0; k < 4; ++k) {
             const int64_t i = base + k * 1024 + tid;
-            if (i < G) offsets[i] = tile2[k * 1024 + tid];
+            if (i < G) {
+                offsets[i] = tile2[k * 1024 + tid];
+                counts_out[i] = tile[k * 1024 + tid] < 0 ? 0 : counts[i];
+            }
         }
     }
     if (tid == 0) {
@@ -224,6 +315,8 @@ __global__ void __launch_bounds__(1024) exclusive_scan_kernel(int32_t *__restric
                                                              int64_t n) {
     __shared__ int tile[kScanTile];
     __shared__ int sh32[33];
+    grid_dependency_wait();
+    grid_dependents_launch();
     cta_exclusive_scan(a, n, nullptr, tile, sh32);
 }
 
@@ -239,6 +332,8 @@ __global__ void __launch_bounds__(kScatterThreads) radix_scatter_kernel(
     int32_t *__restrict__ dst_exp, float *__restrict__ dst_gate,
     int32_t *__restrict__ hist_next, int next_shift, uint32_t next_dmask) {
     __shared__ int wcount[kScatterThreads / 32][256];
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int tid = threadIdx.x, warp = tid >> 5;
     const unsigned lane = lane_id();
     for (int i = tid; i < (kScatterThreads / 32) * 256; i += kScatterThreads)
@@ -302,23 +397,25 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
                             int32_t *group_offsets, int32_t *group_counts,
                             int32_t *active_groups, int32_t *num_active, int32_t *num_distinct,
                             void *ws, const WsLayout &lay, cudaStream_t st) {
+    // The caller has zeroed [0, lay.zero_end) of ws: the status word, the
+    // group counters, the distinct-expert counter, the bitmap and the radix
+    // histograms.
     const int64_t M = sz.M, G = sz.G;
     int *status = ws_at<int>(ws, lay.hdr);
     int32_t *a_tok = ws_at<int32_t>(ws, lay.a_tok), *a_exp = ws_at<int32_t>(ws, lay.a_exp);
     float *a_gate = ws_at<float>(ws, lay.a_gate);
     int32_t *b_tok = ws_at<int32_t>(ws, lay.b_tok), *b_exp = ws_at<int32_t>(ws, lay.b_exp);
     float *b_gate = ws_at<float>(ws, lay.b_gate);
+    int32_t *counts = ws_at<int32_t>(ws, lay.z_cnt);
+    int32_t *ndist = ws_at<int32_t>(ws, lay.z_ndist);
     uint32_t *bitmap = ws_at<uint32_t>(ws, lay.bitmap);
     int32_t *hist = ws_at<int32_t>(ws, lay.hist);
-    const int64_t nwords = (sz.N + 31) / 32;
     const int64_t ntiles = sz.ntiles;
     const int64_t hstride = 256 * ntiles;                // one histogram per pass
     cudaError_t e;
 
-    // radix passes over q = e / B
-    int nbits = 0;
-    while (nbits < 31 && ((int64_t)1 << nbits) < G) ++nbits;       // bits of G - 1
-    const int passes = (nbits + 7) / 8;
+    // radix passes over q = e / B, digits of at most 8 bits
+    const int nbits = sz.qbits, passes = sz.passes;
     const int width = passes ? (nbits + passes - 1) / passes : 0;
     auto pass_mask = [&](int p) -> uint32_t {
         const int shift = p * width;
@@ -326,24 +423,19 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
         return (1u << w) - 1u;
     };
 
-    if ((e = cudaMemsetAsync(group_counts, 0, sizeof(int32_t) * G, st)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(bitmap, 0, sizeof(uint32_t) * nwords, st)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(num_distinct, 0, sizeof(int32_t), st)) != cudaSuccess) return e;
-    if (passes > 0 &&
-        (e = cudaMemsetAsync(hist, 0, sizeof(int32_t) * hstride * passes, st)) != cudaSuccess)
-        return e;
     {
         const int wpb = 8;
         const size_t smem = sizeof(int32_t) * (size_t)sz.K * wpb;
-        sched_prepare_kernel<<<(unsigned)((sz.L + wpb - 1) / wpb), 32 * wpb, smem, st>>>(
-            idx, gate, sz.L, sz.K, (int)sz.N, sz.B, a_tok, a_exp, a_gate, group_counts, bitmap,
-            num_distinct, passes ? hist : nullptr, ntiles, passes ? pass_mask(0) : 0u, status);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch(sched_prepare_kernel, dim3((unsigned)((sz.L + wpb - 1) / wpb)), dim3(32 * wpb),
+                   smem, st, idx, gate, sz.L, sz.K, (int)sz.N, sz.B, a_tok, a_exp, a_gate, counts,
+                   bitmap, ndist, passes ? hist : nullptr, ntiles, passes ? pass_mask(0) : 0u,
+                   status);
+        if (e != cudaSuccess) return e;
     }
-    sched_scan_kernel<<<passes ? 2 : 1, 1024, 0, st>>>(
-        group_counts, G, group_offsets, active_groups, num_active, hist,
-        passes ? (int64_t)(pass_mask(0) + 1) * ntiles : 0);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch(sched_scan_kernel, dim3(passes ? 2 : 1), dim3(1024), 0, st, counts, G,
+               group_counts, group_offsets, active_groups, num_active, ndist, num_distinct, hist,
+               passes ? (int64_t)(pass_mask(0) + 1) * ntiles : (int64_t)0);
+    if (e != cudaSuccess) return e;
 
     if (passes == 0) {
         if ((e = cudaMemcpyAsync(task_token, a_tok, 4 * M, cudaMemcpyDeviceToDevice, st))) return e;
@@ -358,8 +450,9 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
         const bool last = p == passes - 1;
         int32_t *h = hist + hstride * p;
         if (p > 0) {
-            exclusive_scan_kernel<<<1, 1024, 0, st>>>(h, (int64_t)(dmask + 1) * ntiles);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            e = launch(exclusive_scan_kernel, dim3(1), dim3(1024), 0, st, h,
+                       (int64_t)(dmask + 1) * ntiles);
+            if (e != cudaSuccess) return e;
         }
         // ping-pong: the last pass writes the caller's arrays
         int32_t *d_tok, *d_exp;
@@ -371,11 +464,11 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
         } else {
             d_tok = a_tok; d_exp = a_exp; d_gate = a_gate;
         }
-        radix_scatter_kernel<<<(unsigned)ntiles, kScatterThreads, 0, st>>>(
-            s_tok, s_exp, s_gate, M, sz.B, shift, dmask, ntiles, h, d_tok, d_exp, d_gate,
-            last ? nullptr : hist + hstride * (p + 1), (p + 1) * width,
-            last ? 0u : pass_mask(p + 1));
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch(radix_scatter_kernel, dim3((unsigned)ntiles), dim3(kScatterThreads), 0, st,
+                   s_tok, s_exp, s_gate, M, sz.B, shift, dmask, ntiles, (const int32_t *)h, d_tok,
+                   d_exp, d_gate, last ? nullptr : hist + hstride * (p + 1), (p + 1) * width,
+                   last ? 0u : pass_mask(p + 1));
+        if (e != cudaSuccess) return e;
         s_tok = d_tok; s_exp = d_exp; s_gate = d_gate;
     }
     return cudaSuccess;

@@ -201,6 +201,8 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
                                  int nmax, int kmax, size_t warp_words,
                                  const int *__restrict__ only) {
     extern __shared__ __align__(16) uint32_t smem_u[];
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     const int wpb = blockDim.x >> 5;
@@ -396,6 +398,8 @@ axis_topk_reg_kernel(const float *__restrict__ in_r, const float *__restrict__ i
                      int *__restrict__ flags) {
     extern __shared__ __align__(16) uint32_t smem_u[];
     constexpr int kWords = 2 * kNB + 2 * CAP;
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     const int64_t prob = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
@@ -562,15 +566,33 @@ __host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C
     return m;
 }
 
+// Drops from L2, without a write-back, the 128-byte lines lying wholly
+// inside [p, p + n) (discard.global.L2 leaves their contents undefined).
+__device__ __forceinline__ void discard_l2_lines(const float *p, int n) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    const uintptr_t first = (lo + 127u) & ~(uintptr_t)127u;
+    const uintptr_t end = (lo + (uintptr_t)n * 4u) & ~(uintptr_t)127u;
+    for (uintptr_t a = first + 128u * lane_id(); a < end; a += 128u * 32u)
+        asm volatile("discard.global.L2 [%0], 128;" ::"l"(a) : "memory");
+}
+
 // Shared by the CTA: table[c] = (a << 16) | b for the c-th candidate, a-major.
+// dead_r / dead_c (may be null): the router GEMM's logits s_r [L, N_r] and
+// s_c [L, N_c] in the library's workspace.  Every reader of them has finished
+// when this kernel runs, so each warp drops its token's rows from L2: about
+// 43 MB of dirty lines at 4096 tokens of 2 x 1304 logits that would otherwise
+// be written back to HBM while the expert stage streams its rows.
 template <int CAP>
 __global__ void merge_topk_kernel(const float *__restrict__ row_val,
                                   const int *__restrict__ row_idx,
                                   const float *__restrict__ col_val,
                                   const int *__restrict__ col_idx, int L, int N_c, int K, int Kr,
                                   int Kc, int C, int32_t *__restrict__ idx,
-                                  float *__restrict__ score, float *__restrict__ gate) {
+                                  float *__restrict__ score, float *__restrict__ gate,
+                                  const float *dead_r, const float *dead_c, int N_r) {
     extern __shared__ __align__(16) uint32_t smem_u[];
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     const int wpb = blockDim.x >> 5;
@@ -608,6 +630,10 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
 
     const int t = blockIdx.x * wpb + warp;
     if (t >= L) return;
+    if (dead_r) {
+        discard_l2_lines(dead_r + (size_t)t * N_r, N_r);
+        discard_l2_lines(dead_c + (size_t)t * N_c, N_c);
+    }
     uint32_t *base = smem_u + head + (size_t)warp * ml.words;
     float *rv = reinterpret_cast<float *>(base + ml.rv);
     uint32_t *ri = base + ml.ri;
@@ -777,13 +803,10 @@ static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logs
     }
     const int64_t probs = 2 * (int64_t)L;
     const unsigned grid = (unsigned)((probs + wpb - 1) / wpb);
-    axis_topk_kernel<CAP><<<grid, 32 * wpb, smem, st>>>(in_r, in_c, logsoftmax ? 1 : 0,
-                                                        reinterpret_cast<const float2 *>(part_r),
-                                                        reinterpret_cast<const float2 *>(part_c),
-                                                        p_r_out, p_c_out, L, N_r, N_c, K, row_val,
-                                                        row_idx, col_val, col_idx, nmax, kmax,
-                                                        words, only);
-    return cudaGetLastError();
+    return launch(axis_topk_kernel<CAP>, dim3(grid), dim3(32 * wpb), smem, st, in_r, in_c,
+                  logsoftmax ? 1 : 0, reinterpret_cast<const float2 *>(part_r),
+                  reinterpret_cast<const float2 *>(part_c), p_r_out, p_c_out, L, N_r, N_c, K,
+                  row_val, row_idx, col_val, col_idx, nmax, kmax, words, only);
 }
 
 template <int NPL, int CAP>
@@ -796,11 +819,10 @@ static cudaError_t launch_axis_reg(const float *in_r, const float *in_c, int mod
     const size_t smem = (size_t)wpb * (2 * kNB + 2 * CAP) * 4;
     const int64_t probs = 2 * (int64_t)L;
     const unsigned grid = (unsigned)((probs + wpb - 1) / wpb);
-    axis_topk_reg_kernel<NPL, CAP><<<grid, 32 * wpb, smem, st>>>(
-        in_r, in_c, mode, reinterpret_cast<const float2 *>(part_r),
-        reinterpret_cast<const float2 *>(part_c), p_r_out, p_c_out, L, N_r, N_c, K, row_val,
-        row_idx, col_val, col_idx, flags);
-    return cudaGetLastError();
+    return launch(axis_topk_reg_kernel<NPL, CAP>, dim3(grid), dim3(32 * wpb), smem, st, in_r, in_c,
+                  mode, reinterpret_cast<const float2 *>(part_r),
+                  reinterpret_cast<const float2 *>(part_c), p_r_out, p_c_out, L, N_r, N_c, K,
+                  row_val, row_idx, col_val, col_idx, flags);
 }
 
 template <int CAP>
@@ -855,7 +877,8 @@ cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftm
 template <int CAP>
 static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, const float *col_val,
                                   const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
-                                  int32_t *idx, float *score, float *gate, cudaStream_t st) {
+                                  int32_t *idx, float *score, float *gate, const float *dead_r,
+                                  const float *dead_c, int N_r, cudaStream_t st) {
     const MergeLayout ml = merge_layout(K, Kr, Kc, C);
     const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
     const size_t per_warp = ml.words * 4;
@@ -870,18 +893,18 @@ static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, cons
         if (e != cudaSuccess) return e;
     }
     const unsigned grid = (unsigned)((L + wpb - 1) / wpb);
-    merge_topk_kernel<CAP><<<grid, 32 * wpb, smem, st>>>(row_val, row_idx, col_val, col_idx, L,
-                                                         N_c, K, Kr, Kc, C, idx, score, gate);
-    return cudaGetLastError();
+    return launch(merge_topk_kernel<CAP>, dim3(grid), dim3(32 * wpb), smem, st, row_val, row_idx,
+                  col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, dead_r, dead_c, N_r);
 }
 
 cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
                               const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
-                              int32_t *idx, float *score, float *gate, cudaStream_t st) {
+                              int32_t *idx, float *score, float *gate, const float *dead_r,
+                              const float *dead_c, int N_r, cudaStream_t st) {
     // the candidate keys (4 words each) live in the Cand area (4 words per candidate)
     int cap = fast_capacity(K);
     if (cap > C) cap = C >= K ? (C / 32) * 32 : 0;
-#define OMNI_MG(c) return launch_merge_e<c>(row_val, row_idx, col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, st);
+#define OMNI_MG(c) return launch_merge_e<c>(row_val, row_idx, col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, dead_r, dead_c, N_r, st);
     if (cap < K) { OMNI_MG(0) }
     if (cap <= 96) { OMNI_MG(96) }
     if (cap <= 192) { OMNI_MG(192) }
