@@ -41,6 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 E2E_BATCHES = 4
+GRAPH_MAX_L = 256          # batches this small are also timed as one CUDA graph replay
 
 
 # ------------------------------------------------------------------ helpers
@@ -227,6 +228,29 @@ def run_omni(args, cfg, world, rank, local):
     ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     ms_max = reduce_max(ms, world, dev)
 
+    # ---- small batches are launch-bound: the same step as one CUDA graph
+    graph = None
+    if L <= GRAPH_MAX_L:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            gev[i][0].record(stream)
+            g.replay()
+            gev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        gms = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in gev])), world, dev)
+        graph = {"value": job_throughput(world, L, gms), "unit": "tokens/s", "ms_per_step": gms}
+        del g
+
     # ---- staged loop: the same kernels through the three stage calls, for
     # per-stage times and the grouped-expert kernel's duration
     rt = omni.router_topk(t["x"], t["W_r"], t["W_c"], cfg.K)
@@ -369,6 +393,7 @@ def run_omni(args, cfg, world, rank, local):
                 "method": f"omni_routed_fwd on pinned host x/y, copies pipelined over 3 streams, "
                           f"{E2E_BATCHES} distinct token batches cycled, no L2 flush"},
         "gpu_launches": launches_per_step(cfg) * args.steps,
+        "graph": graph,
         "clocks": clocks,
     }
     del t, ws, flush
@@ -410,6 +435,55 @@ def profile_stage(args, cfg):
     if status != 0:
         raise RuntimeError(f"device status {status}")
     print(f"profile-stage {args.profile_stage} {cfg.name}: {args.warmup + args.steps} runs ok")
+
+
+def timeline(args, cfg):
+    """In-stream kernel timeline of omni_routed_fwd (CUPTI through
+    torch.profiler): start and end of every library launch of the last step,
+    relative to the step's first kernel.  With programmatic dependent launch a
+    kernel's CTAs start before its predecessor ends, so a kernel's cost is the
+    gap between consecutive end times ("end delta")."""
+    import atomic_expert_layer_b200 as omni
+    from torch.profiler import profile, ProfilerActivity
+    dev = torch.device("cuda", 0)
+    omni.load()
+    t = inputs.make_inputs(cfg, dev, seed=0)
+    L, d = cfg.L, cfg.d
+    ws = omni.workspace(L, d, cfg.N_r, cfg.N_c, cfg.K, cfg.B, dev)
+    y = torch.empty((L, d), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        omni.omni_routed_fwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r, cfg.N_c,
+                             cfg.K, cfg.B, y, None, None, 0, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(args.steps):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+    rows = sorted((e.time_range.start, e.time_range.end, e.name) for e in prof.events()
+                  if e.device_type == torch.autograd.DeviceType.CUDA)
+    steps, cur = [], None
+    for a, b, n in rows:
+        if "router_gemm" in n:
+            cur = []
+            steps.append(cur)
+        if cur is not None and "omni::" in n:
+            cur.append((a, b, n))
+    spans = [st[-1][1] - st[0][0] for st in steps]
+    last = steps[-1]
+    t0, prev_end = last[0][0], last[0][0]
+    print(f"{'kernel':44s} {'start us':>9s} {'end us':>9s} {'end delta':>10s}")
+    for a, b, n in last:
+        short = n.split("::")[-1].split("(")[0][:44]
+        print(f"{short:44s} {a - t0:9.2f} {b - t0:9.2f} {b - prev_end:10.2f}")
+        prev_end = max(prev_end, b)
+    print(f"first kernel start to last kernel end, per step (us): "
+          f"{', '.join(f'{x:.1f}' for x in spans)}")
 
 
 # ------------------------------------------------------- oracle (CPU) arm
@@ -505,6 +579,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-stage", choices=["router", "schedule", "expert", "all"],
                     help="run only this stage W + K times (for profiler captures; no JSON)")
+    ap.add_argument("--timeline", action="store_true",
+                    help="print the in-stream kernel timeline of the last of K steps (no JSON)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -518,6 +594,9 @@ def main():
     try:
         if args.profile_stage:
             profile_stage(args, cfg)
+            return
+        if args.timeline:
+            timeline(args, cfg)
             return
         if args.impl == "reference":
             out = run_reference(args, cfg, world, rank)
