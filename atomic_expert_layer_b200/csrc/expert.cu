@@ -364,6 +364,120 @@ token_combine_kernel(const uint16_t *__restrict__ V, int L, int N, int K,
     }
 }
 
+// ------------------------------------------------- 2b. token pass, split
+// Small batches: one CTA per token, its slots dealt round-robin to kSplit
+// warps (slot w, w + kSplit, ...), so a token's V rows are fetched kSplit at
+// a time instead of one warp walking all K.  Each warp's partial row goes to
+// shared memory (reusing the row rings once every copy has landed) and the
+// CTA adds the kSplit partials in a fixed order and writes y once.
+constexpr int kSplit = 8;
+
+template <int VPL>
+struct SplitCfg {
+    static constexpr int kStages = 3;
+    static constexpr int kRowBytes = 512 * VPL;
+    static constexpr int kRing = kSplit * kStages * kRowBytes;
+    static constexpr int kPart = kSplit * 256 * VPL * 4;        // fp32 partial rows
+    static constexpr int kSmem = kRing > kPart ? kRing : kPart;
+};
+
+template <int VPL>
+__global__ void __launch_bounds__(32 * kSplit)
+token_split_kernel(const uint16_t *__restrict__ V, int L, int N, int K,
+                   const int *__restrict__ tok_count, const int2 *__restrict__ tok_slots,
+                   float *__restrict__ y, int accumulate, int *status) {
+    using Cfg = SplitCfg<VPL>;
+    constexpr int D = 256 * VPL;
+    constexpr int S = Cfg::kStages;
+    constexpr int RB = Cfg::kRowBytes;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const unsigned lane = lane_id();
+    uint8_t *ring = smem + (size_t)warp * S * RB;
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int t = blockIdx.x;
+    if (t >= L) return;                                  // the same in every thread
+    int n = tok_count[t];
+    if (n > K) {
+        set_status(status, OMNI_DEV_BAD_SCHEDULE);
+        n = K;
+    }
+    const int2 *sl = tok_slots + (size_t)t * K;
+    const int nw = n > warp ? (n - warp + kSplit - 1) / kSplit : 0;   // this warp's slots
+    // (expert, p) of this warp's slots j, j < 32 per block: slot warp + kSplit * j
+    auto load_block = [&](int j0) {
+        const int j = j0 + (int)lane;
+        int2 v = j < nw ? sl[warp + kSplit * j] : make_int2(0, 0);
+        if (v.x < 0 || v.x >= N) v.x = 0;
+        return v;
+    };
+    int2 mine = load_block(0);
+    float acc[VPL * 8];
+#pragma unroll
+    for (int c = 0; c < VPL * 8; ++c) acc[c] = 0.f;
+#pragma unroll
+    for (int j = 0; j < S - 1; ++j) {
+        if (j < nw) {
+            const int e = __shfl_sync(0xffffffffu, mine.x, j);
+            row_async<VPL>(ring + (j % S) * RB, V + (size_t)e * D, lane);
+        }
+        cp_async_commit();
+    }
+    for (int j = 0; j < nw; ++j) {
+        cp_async_wait<S - 2>();
+        __syncwarp();
+        const float p = __int_as_float(__shfl_sync(0xffffffffu, mine.y, j & 31));
+        const int jn = j + S - 1;
+        if (jn < nw) {
+            int en;
+            if ((jn >> 5) == (j >> 5)) {
+                en = __shfl_sync(0xffffffffu, mine.x, jn & 31);
+            } else {
+                const int2 nx = sl[warp + kSplit * jn];
+                en = (nx.x < 0 || nx.x >= N) ? 0 : nx.x;
+            }
+            row_async<VPL>(ring + (jn % S) * RB, V + (size_t)en * D, lane);
+        }
+        cp_async_commit();
+        const uint4 *vr = reinterpret_cast<const uint4 *>(ring + (j % S) * RB);
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+            float vf[8];
+            bf16x8_to_f32(vr[v * 32 + lane], vf);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[8 * v + c] = fmaf(p, vf[c], acc[8 * v + c]);
+        }
+        if (((j + 1) & 31) == 0 && j + 1 < nw) mine = load_block(j + 1);
+    }
+    cp_async_wait<0>();
+    __syncthreads();                                     // every ring is idle: reuse as partials
+    float *part = reinterpret_cast<float *>(smem) + (size_t)warp * D;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        float4 *dst = reinterpret_cast<float4 *>(part + (size_t)(v * 32 + lane) * 8);
+        dst[0] = make_float4(acc[8 * v], acc[8 * v + 1], acc[8 * v + 2], acc[8 * v + 3]);
+        dst[1] = make_float4(acc[8 * v + 4], acc[8 * v + 5], acc[8 * v + 6], acc[8 * v + 7]);
+    }
+    __syncthreads();
+    const float *P = reinterpret_cast<const float *>(smem);
+    float *yr = y + (size_t)t * D;
+    for (int i = (int)threadIdx.x * 4; i < D; i += 32 * kSplit * 4) {
+        float4 r = reinterpret_cast<const float4 *>(P + i)[0];
+#pragma unroll
+        for (int w = 1; w < kSplit; ++w) {
+            const float4 q = reinterpret_cast<const float4 *>(P + (size_t)w * D + i)[0];
+            r.x += q.x; r.y += q.y; r.z += q.z; r.w += q.w;
+        }
+        float4 *dst = reinterpret_cast<float4 *>(yr + i);
+        if (accumulate) {
+            const float4 o = dst[0];
+            r.x += o.x; r.y += o.y; r.z += o.z; r.w += o.w;
+        }
+        dst[0] = r;
+    }
+}
+
 template <int VPL>
 cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, const Sizes &sz,
                        const int32_t *tt, const int32_t *te, const float *tg, float *y,
@@ -377,14 +491,17 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
     e = cudaFuncSetAttribute(token_combine_kernel<VPL>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(token_split_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SplitCfg<VPL>::kSmem);
+    if (e != cudaSuccess) return e;
     const int sms = device_sm_count();
     {
         int per_sm = (227 * 1024) / G::kSmem;
         if (per_sm < 1) per_sm = 1;
         if (per_sm > 16) per_sm = 16;
         const int64_t warps = (int64_t)sms * per_sm * G::kWarps;
-        int64_t per_warp = (sz.M + warps - 1) / warps;
-        if (per_warp < 32) per_warp = 32;
+        // small batches spread down to one task per warp (latency, not issue, bounds them)
+        const int64_t per_warp = (sz.M + warps - 1) / warps;
         const int64_t needed = (sz.M + per_warp - 1) / per_warp;      // warps with work
         const int grid = (int)((needed + G::kWarps - 1) / G::kWarps);
         e = launch(group_gate_kernel<VPL>, dim3(grid), dim3(32 * G::kWarps), G::kSmem, st, x, W,
@@ -392,7 +509,13 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
                    tok_slots, status);
         if (e != cudaSuccess) return e;
     }
-    {
+    if (sz.L <= 4 * sms) {
+        // few tokens: one CTA of kSplit warps per token
+        e = launch(token_split_kernel<VPL>, dim3((unsigned)sz.L), dim3(32 * kSplit),
+                   (size_t)SplitCfg<VPL>::kSmem, st, V, sz.L, (int)sz.N, sz.K,
+                   (const int *)tok_count, (const int2 *)tok_slots, y, accumulate ? 1 : 0,
+                   status);
+    } else {
         int per_sm = (227 * 1024) / C::kSmem;
         if (per_sm < 1) per_sm = 1;
         if (per_sm > 16) per_sm = 16;
