@@ -10,7 +10,8 @@ from __future__ import annotations
 
 import torch
 
-from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_Y_ACCUMULATE, OmniError, load,  # noqa: F401
+from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_Y_ACCUMULATE,  # noqa: F401
+                   OmniError, load,
                    expert_workspace, omni_expert_workspace_size, omni_get_device_status,
                    omni_grouped_expert_fwd, omni_grouped_expert_fwd_noalloc, omni_routed_fwd,
                    omni_router_topk,
@@ -19,7 +20,7 @@ from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_Y_ACCUMULATE, OmniError, load, 
                    omni_workspace_size, router_workspace, schedule_workspace, workspace)
 
 __all__ = [
-    "load", "OmniError", "OMNI_ROUTER_LOGPROBS_IN", "OMNI_Y_ACCUMULATE",
+    "load", "OmniError", "OMNI_ROUTER_LOGPROBS_IN", "OMNI_Y_ACCUMULATE", "OMNI_TOKEN_ORDER",
     "omni_workspace_size", "omni_router_topk", "omni_schedule", "omni_grouped_expert_fwd",
     "omni_routed_fwd", "omni_get_device_status", "workspace", "omni_grouped_expert_fwd_noalloc",
     "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd",
@@ -81,7 +82,7 @@ def grouped_expert_fwd(x, W, V, sched, K, B, y=None, accumulate=False, ws=None, 
 
 
 def routed_fwd(x, W, V, W_r, W_c, K, B, y=None, ws=None, want_routing=False, accumulate=False,
-               stream=None):
+               token_order=False, stream=None):
     L, d = x.shape
     N_r, N_c = W_r.shape[0], W_c.shape[0]
     y = torch.empty((L, d), dtype=torch.float32, device=x.device) if y is None else y
@@ -90,6 +91,6 @@ def routed_fwd(x, W, V, W_r, W_c, K, B, y=None, ws=None, want_routing=False, acc
     if want_routing:
         idx = torch.empty((L, K), dtype=torch.int32, device=x.device)
         gate = torch.empty((L, K), dtype=torch.float32, device=x.device)
-    omni_routed_fwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, B, y, idx, gate,
-                    OMNI_Y_ACCUMULATE if accumulate else 0, ws, stream)
+    flags = (OMNI_Y_ACCUMULATE if accumulate else 0) | (OMNI_TOKEN_ORDER if token_order else 0)
+    omni_routed_fwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, B, y, idx, gate, flags, ws, stream)
     return (y, idx, gate) if want_routing else y

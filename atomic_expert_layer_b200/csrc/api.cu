@@ -13,6 +13,7 @@ namespace omni {
 
 namespace {
 constexpr int kVersion = 1;
+constexpr int kTokenOrderMaxL = 16;   // decode batches skip the schedule (see omni.h)
 
 inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -310,17 +311,24 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     rc = router_topk_impl(x, W_r, W_c, sz, nullptr, nullptr, idx, score, gate,
                           flags & ~OMNI_ROUTER_LOGPROBS_IN, ws, lay, st);
     if (rc) return rc;
-    int32_t *tt = ws_at<int32_t>(ws, lay.t_tok), *te = ws_at<int32_t>(ws, lay.t_exp);
-    float *tg = ws_at<float>(ws, lay.t_gate);
-    int32_t *goff = ws_at<int32_t>(ws, lay.g_off), *gcnt = ws_at<int32_t>(ws, lay.g_cnt);
-    int32_t *gact = ws_at<int32_t>(ws, lay.g_act), *nact = ws_at<int32_t>(ws, lay.n_act);
-    int32_t *ndist = ws_at<int32_t>(ws, lay.n_dist);
-    if ((rc = cuda_rc(launch_schedule(idx, gate, sz, tt, te, tg, goff, gcnt, gact, nact, ndist,
-                                      ws, lay, st))))
-        return rc;
-    if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, tt, te, tg, y,
-                                            (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st))))
-        return rc;
+    if ((flags & OMNI_TOKEN_ORDER) || L <= kTokenOrderMaxL) {
+        // tasks in token order, read straight from the routing (no schedule)
+        if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, nullptr, idx, gate, y,
+                                                (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st))))
+            return rc;
+    } else {
+        int32_t *tt = ws_at<int32_t>(ws, lay.t_tok), *te = ws_at<int32_t>(ws, lay.t_exp);
+        float *tg = ws_at<float>(ws, lay.t_gate);
+        int32_t *goff = ws_at<int32_t>(ws, lay.g_off), *gcnt = ws_at<int32_t>(ws, lay.g_cnt);
+        int32_t *gact = ws_at<int32_t>(ws, lay.g_act), *nact = ws_at<int32_t>(ws, lay.n_act);
+        int32_t *ndist = ws_at<int32_t>(ws, lay.n_dist);
+        if ((rc = cuda_rc(launch_schedule(idx, gate, sz, tt, te, tg, goff, gcnt, gact, nact,
+                                          ndist, ws, lay, st))))
+            return rc;
+        if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, tt, te, tg, y,
+                                                (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st))))
+            return rc;
+    }
     if (idx_out &&
         (rc = cuda_rc(cudaMemcpyAsync(idx_out, idx, 4 * (size_t)sz.M, cudaMemcpyDeviceToDevice, st))))
         return rc;

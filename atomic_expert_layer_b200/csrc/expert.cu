@@ -142,7 +142,8 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
         const int i = c0 + (int)lane;
         t = 0; e = 0; g = 0.f; slot = K;
         if (i < n) {
-            t = task_token[a0 + i];
+            // token order (no schedule): task m is (m / K, idx[m], gate[m])
+            t = task_token ? task_token[a0 + i] : (int)((a0 + i) / K);
             e = task_expert[a0 + i];
             g = task_gate[a0 + i];
             if (e < 0 || e >= N || t < 0 || t >= L) {

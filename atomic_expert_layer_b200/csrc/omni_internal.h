@@ -81,7 +81,9 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
                             int32_t *active_groups, int32_t *num_active, int32_t *num_distinct,
                             void *ws, const WsLayout &lay, cudaStream_t st);
 
-// ---- grouped expert stage (expects the per-token slot counters zeroed)
+// ---- grouped expert stage (expects the per-token slot counters zeroed).
+// task_token == nullptr: the tasks are in token order, task m belongs to
+// token m / K (task_expert / task_gate are then the router's idx / gate).
 cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const uint16_t *V,
                                   const Sizes &sz, const int32_t *task_token,
                                   const int32_t *task_expert, const float *task_gate,

@@ -105,6 +105,8 @@ def launches_per_step(cfg) -> int:
     router = 1 + (2 if reg else 1) + 1            # GEMM, axis top-K (+ flagged redo), merge
     p = radix_passes(cfg.G)
     sched = 2 + (p + max(p - 1, 0))               # prepare, scan, scatters, histogram scans
+    if cfg.L <= 16:
+        sched = 0                                 # decode batches run in token order
     return router + sched + 2                     # group pass, token pass
 
 
@@ -227,6 +229,29 @@ def run_omni(args, cfg, world, rank, local):
     clocks = clk.summary()
     ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     ms_max = reduce_max(ms, world, dev)
+
+    # ---- ablation: the same layer with the expert stage in token order and
+    # no expert-centric schedule (OMNI_TOKEN_ORDER; the path L <= 16 always takes)
+    def step_token_order():
+        omni.omni_routed_fwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r, cfg.N_c,
+                             cfg.K, cfg.B, y, None, None, omni.OMNI_TOKEN_ORDER, ws)
+
+    for _ in range(3):
+        step_token_order()
+    aev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        aev[i][0].record(stream)
+        step_token_order()
+        aev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    tok_ms = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in aev])), world, dev)
+    ablation = {"token_order_ms_per_step": tok_ms, "expert_centric_ms_per_step": ms_max,
+                "token_order_over_expert_centric": tok_ms / ms_max}
 
     # ---- small batches are launch-bound: the same step as one CUDA graph
     graph = None
@@ -394,6 +419,7 @@ def run_omni(args, cfg, world, rank, local):
                           f"{E2E_BATCHES} distinct token batches cycled, no L2 flush"},
         "gpu_launches": launches_per_step(cfg) * args.steps,
         "graph": graph,
+        "ablation": ablation,
         "clocks": clocks,
     }
     del t, ws, flush

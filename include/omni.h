@@ -66,6 +66,7 @@ typedef enum {
 /* flags */
 #define OMNI_ROUTER_LOGPROBS_IN 1u  /* omni_router_topk: p_r, p_c are inputs (skip s = xW^T and LogSoftmax) */
 #define OMNI_Y_ACCUMULATE       2u  /* y += routed(x) instead of y = routed(x)                           */
+#define OMNI_TOKEN_ORDER        4u  /* omni_routed_fwd: expert stage in token order, no schedule (below)  */
 
 /* Device status codes written into the workspace status word. */
 #define OMNI_DEV_OK              0
@@ -160,9 +161,10 @@ int omni_schedule(const int32_t *idx, const float *gate, int L, int K, int N, in
  *   x [L, d] bf16, W [N, d] bf16, V [N, d] bf16
  *   schedule arrays as produced by omni_schedule for the same L, K, N, B
  *   y [L, d] fp32  output (overwritten, or accumulated with OMNI_Y_ACCUMULATE)
- * Summation order inside y is not fixed (fp32 atomic adds), so y may differ
- * in the last bits between runs.  Limits: d % 256 == 0, d <= OMNI_MAX_D,
- * B <= OMNI_MAX_B.
+ * Each y row is written once, but the order in which a token's tasks are
+ * summed follows the order their slots were claimed (atomic counters), so y
+ * may differ in the last bits between runs.  Limits: d % 256 == 0,
+ * d <= OMNI_MAX_D, B <= OMNI_MAX_B.
  */
 int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                             int L, int d, int K, int N, int B,
@@ -180,6 +182,14 @@ int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_b
  *   x [L, d], W [N, d], V [N, d], W_r [N_r, d], W_c [N_c, d]  bf16
  *   y [L, d] fp32 output;  idx_out [L, K] int32, gate_out [L, K] fp32 are
  *   optional copies of the routing (NULL to skip).
+ * Token order: with flag OMNI_TOKEN_ORDER, and always for L <= 16 tokens,
+ * the expert stage takes the tasks in token order straight from the router
+ * (task t*K + k = (t, idx[t,k], gate[t,k])) and the schedule is skipped.
+ * y is the same sum (up to summation order); only the order in which expert
+ * rows are fetched changes.  For a few tokens the grouping has nothing to
+ * reuse and the schedule's launches are pure latency; for large batches the
+ * flag is the token-centric execution the expert-centric schedule replaces
+ * (an ablation).
  * Limits: those of the three calls above.
  */
 int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
