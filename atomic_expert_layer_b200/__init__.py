@@ -10,7 +10,8 @@ from __future__ import annotations
 
 import torch
 
-from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_Y_ACCUMULATE,  # noqa: F401
+from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_TOPK_BLOCKWISE,  # noqa: F401
+                   OMNI_Y_ACCUMULATE,
                    OmniError, load,
                    expert_workspace, omni_expert_workspace_size, omni_get_device_status,
                    omni_grouped_expert_fwd, omni_grouped_expert_fwd_noalloc, omni_routed_fwd,
@@ -20,16 +21,19 @@ from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_Y_ACCUMULATE,
                    omni_workspace_size, router_workspace, schedule_workspace, workspace)
 
 __all__ = [
-    "load", "OmniError", "OMNI_ROUTER_LOGPROBS_IN", "OMNI_Y_ACCUMULATE", "OMNI_TOKEN_ORDER",
+    "load", "OmniError", "OMNI_ROUTER_LOGPROBS_IN", "OMNI_Y_ACCUMULATE", "OMNI_TOKEN_ORDER", "OMNI_TOPK_BLOCKWISE",
     "omni_workspace_size", "omni_router_topk", "omni_schedule", "omni_grouped_expert_fwd",
     "omni_routed_fwd", "omni_get_device_status", "workspace", "omni_grouped_expert_fwd_noalloc",
     "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd",
 ]
 
 
-def router_topk(x, W_r, W_c, K, ws=None, p_r=None, p_c=None, logprobs_in=False, stream=None):
+def router_topk(x, W_r, W_c, K, ws=None, p_r=None, p_c=None, logprobs_in=False,
+                blockwise=False, stream=None):
     """Top-K experts per token.  With logprobs_in, p_r / p_c are inputs and
-    x may be None (then pass W_r / W_c as None too)."""
+    x may be None (then pass W_r / W_c as None too).  blockwise (with
+    logprobs_in) selects with the blockwise grid scan instead of the
+    row / column pruning; the result is the same."""
     if logprobs_in:
         L, N_r = p_r.shape
         N_c = p_c.shape[1]
@@ -45,8 +49,8 @@ def router_topk(x, W_r, W_c, K, ws=None, p_r=None, p_c=None, logprobs_in=False, 
     score = torch.empty((L, K), dtype=torch.float32, device=dev)
     gate = torch.empty((L, K), dtype=torch.float32, device=dev)
     ws = router_workspace(L, N_r, N_c, K, dev) if ws is None else ws
-    omni_router_topk(x, W_r, W_c, L, d, N_r, N_c, K, p_r, p_c, idx, score, gate,
-                     OMNI_ROUTER_LOGPROBS_IN if logprobs_in else 0, ws, stream)
+    flags = (OMNI_ROUTER_LOGPROBS_IN if logprobs_in else 0) | (OMNI_TOPK_BLOCKWISE if blockwise else 0)
+    omni_router_topk(x, W_r, W_c, L, d, N_r, N_c, K, p_r, p_c, idx, score, gate, flags, ws, stream)
     return dict(p_r=p_r, p_c=p_c, idx=idx, score=score, gate=gate)
 
 

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libomni.so")
 OMNI_ROUTER_LOGPROBS_IN = 1
 OMNI_Y_ACCUMULATE = 2
 OMNI_TOKEN_ORDER = 4
+OMNI_TOPK_BLOCKWISE = 8
 
 STATUS = {0: "OMNI_OK", -1: "OMNI_ERR_INVALID_ARG", -2: "OMNI_ERR_UNSUPPORTED",
           -3: "OMNI_ERR_WORKSPACE", -4: "OMNI_ERR_CUDA", -5: "OMNI_ERR_DEVICE"}

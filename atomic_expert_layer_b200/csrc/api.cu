@@ -241,6 +241,14 @@ int omni_router_topk(const omni_bf16 *x, const omni_bf16 *W_r, const omni_bf16 *
     WsLayout lay;
     if ((rc = check_ws(sz, kRegRouter, ws, ws_bytes, &lay))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (flags & OMNI_TOPK_BLOCKWISE) {
+        // the pages' blockwise grid top-K, on caller log-probabilities; its
+        // candidates use the logits area (s_r, s_c), idle in this mode
+        if (!lp_in || blockwise_bands(N_r, N_c, K) < 1) return OMNI_ERR_UNSUPPORTED;
+        if ((rc = reset_workspace(ws, lay, st))) return rc;
+        return cuda_rc(launch_topk_blockwise(p_r, p_c, L, N_r, N_c, K, ws_at<void>(ws, lay.s_r),
+                                             idx, score, gate, st));
+    }
     if ((rc = reset_workspace(ws, lay, st))) return rc;
     return router_topk_impl(x, W_r, W_c, sz, p_r, p_c, idx, score, gate, flags, ws, lay, st);
 }
@@ -299,6 +307,7 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     if (rc) return rc;
     if (!x || !W || !V || !W_r || !W_c || !y) return OMNI_ERR_INVALID_ARG;
     if (d % 256 != 0 || d > OMNI_MAX_D) return OMNI_ERR_UNSUPPORTED;
+    if (flags & OMNI_TOPK_BLOCKWISE) return OMNI_ERR_UNSUPPORTED;   // router_topk only
     if (!aligned16(x) || !aligned16(W) || !aligned16(V) || !aligned16(W_r) || !aligned16(W_c) ||
         !aligned16(y))
         return OMNI_ERR_INVALID_ARG;

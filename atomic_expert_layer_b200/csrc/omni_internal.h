@@ -74,6 +74,13 @@ cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const fl
                               int32_t *idx, float *score, float *gate, const float *dead_r,
                               const float *dead_c, int N_r, cudaStream_t st);
 
+// ---- the pages' blockwise grid top-K (alternative to axis + merge); its
+// candidates need L * blockwise_bands(...) * K * 16 bytes at `cand`
+int blockwise_bands(int N_r, int N_c, int K);
+cudaError_t launch_topk_blockwise(const float *p_r, const float *p_c, int L, int N_r, int N_c,
+                                  int K, void *cand, int32_t *idx, float *score, float *gate,
+                                  cudaStream_t st);
+
 // ---- schedule (expects [0, lay.zero_end) of ws zeroed)
 cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &sz,
                             int32_t *task_token, int32_t *task_expert, float *task_gate,

@@ -320,6 +320,36 @@ def run_omni(args, cfg, world, rank, local):
     st_sched = float(np.mean([e[1].elapsed_time(e[2]) for e in sev]))
     st_expert = float(np.mean([e[2].elapsed_time(e[3]) for e in sev]))
 
+    # ---- the selection (row / column top-K + merge, on the same p) against the
+    # pages' blockwise grid scan; a few steps, the scan scores all N cells
+    topk_cmp = None
+    if 4 * cfg.K <= cfg.N_r + cfg.N_c:
+        ws_r2 = omni.router_workspace(L, cfg.N_r, cfg.N_c, cfg.K, dev)
+        o = {k: torch.empty_like(rt[k]) for k in ("idx", "score", "gate")}
+        res = {}
+        for name, fl in (("pruned", omni.OMNI_ROUTER_LOGPROBS_IN),
+                         ("blockwise", omni.OMNI_ROUTER_LOGPROBS_IN | omni.OMNI_TOPK_BLOCKWISE)):
+            def sel(fl=fl):
+                omni.omni_router_topk(None, None, None, L, 0, cfg.N_r, cfg.N_c, cfg.K,
+                                      rt["p_r"], rt["p_c"], o["idx"], o["score"], o["gate"],
+                                      fl, ws_r2)
+            sel()
+            reps = 5
+            cev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(reps)]
+            torch.cuda.synchronize()
+            for i in range(reps):
+                flush.zero_()
+                cev[i][0].record(stream)
+                sel()
+                cev[i][1].record(stream)
+            torch.cuda.synchronize()
+            res[name] = float(np.mean([a.elapsed_time(b) for a, b in cev]))
+        topk_cmp = {"pruned_ms": res["pruned"], "blockwise_ms": res["blockwise"],
+                    "blockwise_over_pruned": res["blockwise"] / res["pruned"]}
+        del ws_r2, o
+
+
     # ---- end to end: host buffers, copies inside the timed region.  Every
     # step copies its token batch in from pinned host memory and its y out to
     # pinned host memory.  Steps are pipelined over three streams (copy-in of
@@ -420,6 +450,7 @@ def run_omni(args, cfg, world, rank, local):
         "gpu_launches": launches_per_step(cfg) * args.steps,
         "graph": graph,
         "ablation": ablation,
+        "topk_compare": topk_cmp,
         "clocks": clocks,
     }
     del t, ws, flush

@@ -67,6 +67,7 @@ typedef enum {
 #define OMNI_ROUTER_LOGPROBS_IN 1u  /* omni_router_topk: p_r, p_c are inputs (skip s = xW^T and LogSoftmax) */
 #define OMNI_Y_ACCUMULATE       2u  /* y += routed(x) instead of y = routed(x)                           */
 #define OMNI_TOKEN_ORDER        4u  /* omni_routed_fwd: expert stage in token order, no schedule (below)  */
+#define OMNI_TOPK_BLOCKWISE     8u  /* omni_router_topk: the pages' blockwise grid top-K (below)           */
 
 /* Device status codes written into the workspace status word. */
 #define OMNI_DEV_OK              0
@@ -118,6 +119,12 @@ size_t omni_expert_workspace_size(int L, int d, int K, int N, int B);
  * Row and column candidates are the top min(K, N_r) rows and min(K, N_c)
  * columns.  Limits: K <= N_r * N_c, K <= OMNI_MAX_K, N_r, N_c <= OMNI_MAX_AXIS.
  * p must be finite (NaN / Inf give an unspecified but in-range selection).
+ * OMNI_TOPK_BLOCKWISE (with OMNI_ROUTER_LOGPROBS_IN only): the same result by
+ * the selection [R] step 2 describes -- the implicit grid cut into blocks of
+ * rows, each scored cell by cell by a thread block that keeps its local
+ * top-K, then a per-token merge -- instead of the row / column pruning.  It
+ * scores all N_r * N_c cells (an alternative kept for comparison).  Extra
+ * limit: K <= (N_r + N_c) / 4, else OMNI_ERR_UNSUPPORTED.
  */
 int omni_router_topk(const omni_bf16 *x, const omni_bf16 *W_r, const omni_bf16 *W_c,
                      int L, int d, int N_r, int N_c, int K,

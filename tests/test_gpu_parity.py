@@ -60,6 +60,38 @@ def test_router_topk_from_logprobs_bitexact(L, N_r, N_c, K, quantum, seed):
     np.testing.assert_allclose(host(out["gate"]), gate, rtol=4e-6, atol=1e-12)
 
 
+@pytest.mark.parametrize("L,N_r,N_c,K,quantum,seed", [
+    (300, 512, 512, 64, None, 21),        # small grid, 4 bands
+    (97, 1304, 1304, 64, None, 22),       # headline grid, 10 bands
+    (64, 1024, 1024, 128, None, 23),      # skewed-config grid, K = 128
+    (50, 8, 64, 16, None, 24),            # K > N_r, one band
+    (50, 1, 300, 40, None, 25),           # single row
+    (40, 300, 1, 40, None, 26),           # single column
+    (33, 12, 12, 1, None, 27),            # K = 1, more bands than needed rows
+    (17, 2000, 3000, 512, None, 28),      # K at the limit
+    (64, 256, 256, 32, 2.0 ** -3, 29),    # forced exact ties across bands
+    (100, 96, 160, 16, 0.25, 30),         # forced ties, coarse quantum
+])
+def test_router_topk_blockwise_bitexact(L, N_r, N_c, K, quantum, seed):
+    """The pages' blockwise grid top-K gives the oracle's selection exactly."""
+    p_r = inputs.random_logprobs(L, N_r, seed, quantum)
+    p_c = inputs.random_logprobs(L, N_c, seed + 1000, quantum)
+    idx, score, gate = oracle.topk_from_logprobs(p_r, p_c, K)
+    out = omni.router_topk(None, None, None, K, p_r=torch.from_numpy(p_r).to(DEV),
+                           p_c=torch.from_numpy(p_c).to(DEV), logprobs_in=True, blockwise=True)
+    np.testing.assert_array_equal(host(out["idx"]), idx)
+    np.testing.assert_array_equal(host(out["score"]), score)
+    np.testing.assert_allclose(host(out["gate"]), gate, rtol=4e-6, atol=1e-12)
+
+
+def test_router_topk_blockwise_limits():
+    """K above (N_r + N_c) / 4 is refused on the host, before any launch."""
+    p_r = torch.zeros((4, 8), device=DEV)
+    p_c = torch.zeros((4, 8), device=DEV)
+    with pytest.raises(omni.OmniError):
+        omni.router_topk(None, None, None, 8, p_r=p_r, p_c=p_c, logprobs_in=True, blockwise=True)
+
+
 def test_router_full_tiny_against_oracle():
     cfg = configs.TINY
     t = inputs.make_inputs(cfg, DEV, seed=0, with_experts=False)
