@@ -52,6 +52,8 @@ def _load():
         lib.oracle_schedule.argtypes = [P, P, I, I, I, I, P, P, P, P, P, P, P, P]
         lib.oracle_expert_fwd_token_centric.argtypes = [P, P, P, I, I, P, P, P, I, P, I]
         lib.oracle_expert_fwd_expert_centric.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, I, P]
+        lib.oracle_expert_bwd.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P]
+        lib.oracle_router_bwd.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P]
         lib.oracle_max_threads.argtypes = []
         for f in (lib.oracle_router_logprobs, lib.oracle_topk_from_logprobs, lib.oracle_schedule,
                   lib.oracle_expert_fwd_token_centric, lib.oracle_expert_fwd_expert_centric,
@@ -174,3 +176,46 @@ def routed_fwd(x, W, V, W_r, W_c, K: int, B: int, tokens=None, nthreads: int = 0
     idx, score, gate = topk_from_logprobs(p_r, p_c, K, nthreads)
     y = expert_fwd_token_centric(xs, W, V, idx, gate, None, nthreads)
     return dict(p_r=p_r, p_c=p_c, idx=idx, score=score, gate=gate, y=y)
+
+
+# ------------------------------------------------------------------ backward
+def expert_bwd(x, W, V, idx, gate, dy):
+    """Backward of the expert part with the routing fixed (fp64): returns
+    dx [L, d], dW and dV [rows of W, d], dgate [L, K].  W / V may be the
+    compacted rows the tokens use, idx then holding row numbers."""
+    x, W, V = _c(x, np.uint16), _c(W, np.uint16), _c(V, np.uint16)
+    idx, gate, dy = _c(idx, np.int32), _c(gate, np.float32), _c(dy, np.float32)
+    L, d = x.shape
+    K = idx.shape[1]
+    rows = W.shape[0]
+    out = dict(dx=np.empty((L, d)), dW=np.empty((rows, d)), dV=np.empty((rows, d)),
+               dgate=np.empty((L, K)))
+    _check(_load().oracle_expert_bwd(_p(x), _p(W), _p(V), L, d, K, rows, _p(idx), _p(gate),
+                                     _p(dy), _p(out["dx"]), _p(out["dW"]), _p(out["dV"]),
+                                     _p(out["dgate"])), "expert_bwd")
+    return out
+
+
+def router_bwd(x, W_r, W_c, p_r, p_c, idx, gate, dgate, dx=None):
+    """Backward of the router given dgate (fp64): returns dx (added to the
+    given dx if any), dW_r [N_r, d], dW_c [N_c, d]."""
+    x, W_r, W_c = _c(x, np.uint16), _c(W_r, np.uint16), _c(W_c, np.uint16)
+    p_r, p_c = _c(p_r, np.float32), _c(p_c, np.float32)
+    idx, gate, dgate = _c(idx, np.int32), _c(gate, np.float32), _c(dgate, np.float64)
+    L, d = x.shape
+    N_r, N_c = W_r.shape[0], W_c.shape[0]
+    K = idx.shape[1]
+    dx = np.zeros((L, d)) if dx is None else _c(dx, np.float64).copy()
+    dW_r, dW_c = np.empty((N_r, d)), np.empty((N_c, d))
+    _check(_load().oracle_router_bwd(_p(x), _p(W_r), _p(W_c), L, d, N_r, N_c, K, _p(p_r), _p(p_c),
+                                     _p(idx), _p(gate), _p(dgate), _p(dx), _p(dW_r), _p(dW_c)),
+           "router_bwd")
+    return dict(dx=dx, dW_r=dW_r, dW_c=dW_c)
+
+
+def routed_bwd(x, W, V, W_r, W_c, p_r, p_c, idx, gate, dy):
+    """Whole routed-branch backward with the forward's routing fixed (fp64)."""
+    e = expert_bwd(x, W, V, idx, gate, dy)
+    r = router_bwd(x, W_r, W_c, p_r, p_c, idx, gate, e["dgate"], dx=e["dx"])
+    return dict(dx=r["dx"], dW=e["dW"], dV=e["dV"], dW_r=r["dW_r"], dW_c=r["dW_c"],
+                dgate=e["dgate"])

@@ -353,3 +353,110 @@ int oracle_expert_fwd_expert_centric(const uint16_t *x, const uint16_t *W, const
     }
     return 0;
 }
+
+/* ---- Backward of the routed branch ----------------------------------------
+ * The pages give no backward; it is the derivative of the forward above with
+ * the top-K selection held fixed (a selection has no gradient).
+ *
+ * Expert part, for each task (t, k), e = idx[t,k], g = gate[t,k]:
+ *   h = x_t . w_e,  a = SiLU(h),  c = dy_t . v_e
+ *   dgate[t,k] = a c
+ *   dV[e] += g a dy_t
+ *   dh = g c SiLU'(h),  SiLU'(h) = s (1 + h (1 - s)),  s = 1 / (1 + exp(-h))
+ *   dW[e] += dh x_t,    dx_t += dh w_e
+ * W and V may be passed compacted to the rows the tokens use (idx then holds
+ * row numbers 0..rows-1); dW and dV are [rows, d].  dx, dW, dV, dgate are
+ * overwritten.  fp64, single-threaded (the scatter into dW, dV is ordered). */
+static double silu_grad(double z) {
+    const double s = 1.0 / (1.0 + exp(-z));
+    return s * (1.0 + z * (1.0 - s));
+}
+
+int oracle_expert_bwd(const uint16_t *x, const uint16_t *W, const uint16_t *V, int L, int d,
+                      int K, int rows, const int32_t *idx, const float *gate, const float *dy,
+                      double *dx, double *dW, double *dV, double *dgate) {
+    if (L < 0 || d <= 0 || K <= 0 || rows <= 0) return -1;
+    for (int64_t u = 0; u < (int64_t)L * d; ++u) dx[u] = 0.0;
+    for (int64_t u = 0; u < (int64_t)rows * d; ++u) { dW[u] = 0.0; dV[u] = 0.0; }
+    for (int t = 0; t < L; ++t) {
+        const uint16_t *xt = x + (size_t)t * d;
+        const float *dyt = dy + (size_t)t * d;
+        for (int k = 0; k < K; ++k) {
+            const int64_t e = idx[(size_t)t * K + k];
+            if (e < 0 || e >= rows) return -2;
+            const uint16_t *w = W + (size_t)e * d, *v = V + (size_t)e * d;
+            const double g = (double)gate[(size_t)t * K + k];
+            double h = 0.0, c = 0.0;
+            for (int j = 0; j < d; ++j) {
+                h += bf16_to_double(xt[j]) * bf16_to_double(w[j]);
+                c += (double)dyt[j] * bf16_to_double(v[j]);
+            }
+            const double a = silu(h);
+            dgate[(size_t)t * K + k] = a * c;
+            const double dh = g * c * silu_grad(h);
+            for (int j = 0; j < d; ++j) {
+                dV[(size_t)e * d + j] += g * a * (double)dyt[j];
+                dW[(size_t)e * d + j] += dh * bf16_to_double(xt[j]);
+                dx[(size_t)t * d + j] += dh * bf16_to_double(w[j]);
+            }
+        }
+    }
+    return 0;
+}
+
+/* Router part, given dgate:
+ *   gates are the softmax over the K selected S:  dS_k = g_k (dgate_k - sum_j g_j dgate_j)
+ *   S = p_r[i] + p_c[j], n = i N_c + j:           dp_r[i] += dS_k,  dp_c[j] += dS_k
+ *   p = s - logsumexp(s):                          ds = dp - exp(p) * sum(dp)
+ *   s_r = x W_r^T:                                 dx_t += sum_i ds_r[i] W_r[i],
+ *                                                  dW_r[i] += ds_r[i] x_t   (columns alike)
+ * dx is ADDED to (so the expert part can go first); dW_r, dW_c are
+ * overwritten.  p_r, p_c are the forward's fp32 log-probabilities.  Dense over
+ * the grid axes in fp64, single-threaded.                                  */
+int oracle_router_bwd(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c, int L, int d,
+                      int N_r, int N_c, int K, const float *p_r, const float *p_c,
+                      const int32_t *idx, const float *gate, const double *dgate, double *dx,
+                      double *dW_r, double *dW_c) {
+    if (L < 0 || d <= 0 || N_r <= 0 || N_c <= 0 || K <= 0) return -1;
+    for (int64_t u = 0; u < (int64_t)N_r * d; ++u) dW_r[u] = 0.0;
+    for (int64_t u = 0; u < (int64_t)N_c * d; ++u) dW_c[u] = 0.0;
+    double *dp_r = (double *)malloc(sizeof(double) * (size_t)N_r);
+    double *dp_c = (double *)malloc(sizeof(double) * (size_t)N_c);
+    if (!dp_r || !dp_c) { free(dp_r); free(dp_c); return -3; }
+    for (int t = 0; t < L; ++t) {
+        double sgd = 0.0;
+        for (int k = 0; k < K; ++k) sgd += (double)gate[(size_t)t * K + k] * dgate[(size_t)t * K + k];
+        for (int i = 0; i < N_r; ++i) dp_r[i] = 0.0;
+        for (int j = 0; j < N_c; ++j) dp_c[j] = 0.0;
+        for (int k = 0; k < K; ++k) {
+            const int64_t n = idx[(size_t)t * K + k];
+            if (n < 0 || n >= (int64_t)N_r * N_c) { free(dp_r); free(dp_c); return -2; }
+            const double dS = (double)gate[(size_t)t * K + k] * (dgate[(size_t)t * K + k] - sgd);
+            dp_r[n / N_c] += dS;
+            dp_c[n % N_c] += dS;
+        }
+        double sr = 0.0, sc = 0.0;
+        for (int i = 0; i < N_r; ++i) sr += dp_r[i];
+        for (int j = 0; j < N_c; ++j) sc += dp_c[j];
+        const uint16_t *xt = x + (size_t)t * d;
+        for (int i = 0; i < N_r; ++i) {
+            const double ds = dp_r[i] - exp((double)p_r[(size_t)t * N_r + i]) * sr;
+            if (ds == 0.0) continue;
+            for (int j = 0; j < d; ++j) {
+                dx[(size_t)t * d + j] += ds * bf16_to_double(W_r[(size_t)i * d + j]);
+                dW_r[(size_t)i * d + j] += ds * bf16_to_double(xt[j]);
+            }
+        }
+        for (int i = 0; i < N_c; ++i) {
+            const double ds = dp_c[i] - exp((double)p_c[(size_t)t * N_c + i]) * sc;
+            if (ds == 0.0) continue;
+            for (int j = 0; j < d; ++j) {
+                dx[(size_t)t * d + j] += ds * bf16_to_double(W_c[(size_t)i * d + j]);
+                dW_c[(size_t)i * d + j] += ds * bf16_to_double(xt[j]);
+            }
+        }
+    }
+    free(dp_r);
+    free(dp_c);
+    return 0;
+}

@@ -259,3 +259,89 @@ def test_routed_fwd_token_subset_matches_full():
     np.testing.assert_array_equal(part["idx"], full["idx"][toks])
     np.testing.assert_array_equal(part["y"], full["y"][toks])
     np.testing.assert_array_equal(full["idx"], idx)
+
+
+# ------------------------------------------------------------------ backward
+def _bf16_values(rng, shape, scale):
+    """Random values that are exact in bf16: (bit patterns, float64 values)."""
+    t = torch.tensor(rng.normal(0.0, scale, size=shape).astype(np.float32)).to(torch.bfloat16)
+    return inputs.to_u16(t), t.to(torch.float64).numpy()
+
+
+def _np_forward(x, W, V, W_r, W_c, idx, N_c):
+    """The routed branch in numpy fp64 with the expert selection idx fixed:
+    an implementation independent of the oracle's C code, used only to take
+    finite differences."""
+    def log_softmax(s):
+        m = s.max(axis=1, keepdims=True)
+        return s - (m + np.log(np.exp(s - m).sum(axis=1, keepdims=True)))
+    p_r, p_c = log_softmax(x @ W_r.T), log_softmax(x @ W_c.T)
+    rows = np.arange(x.shape[0])[:, None]
+    S = p_r[rows, idx // N_c] + p_c[rows, idx % N_c]
+    g = np.exp(S - S.max(axis=1, keepdims=True))
+    g /= g.sum(axis=1, keepdims=True)
+    h = np.einsum("td,tkd->tk", x, W[idx])
+    a = h / (1.0 + np.exp(-h))
+    return np.einsum("tk,tkd->td", g * a, V[idx])
+
+
+def test_backward_matches_finite_differences():
+    """Every gradient of the oracle's backward (expert and router parts,
+    through gates, LogSoftmax and both projections) against central finite
+    differences of an independent fp64 forward, the selection held fixed."""
+    rng = np.random.default_rng(7)
+    L, d, N_r, N_c, K = 3, 8, 5, 4, 6
+    xu, x = _bf16_values(rng, (L, d), 1.0)
+    Wu, W = _bf16_values(rng, (N_r * N_c, d), 0.6)
+    Vu, V = _bf16_values(rng, (N_r * N_c, d), 0.6)
+    Wru, W_r = _bf16_values(rng, (N_r, d), 0.5)
+    Wcu, W_c = _bf16_values(rng, (N_c, d), 0.5)
+    dy = rng.normal(0.0, 1.0, size=(L, d)).astype(np.float32)
+    p_r, p_c = oracle.router_logprobs(xu, Wru, Wcu)
+    idx, _, gate = oracle.topk_from_logprobs(p_r, p_c, K)
+    grads = oracle.routed_bwd(xu, Wu, Vu, Wru, Wcu, p_r, p_c, idx, gate, dy)
+    params = dict(x=x, W=W, V=V, W_r=W_r, W_c=W_c)
+    names = dict(x="dx", W="dW", V="dV", W_r="dW_r", W_c="dW_c")
+    dy64 = dy.astype(np.float64)
+    eps = 1e-6
+    for pname, P in params.items():
+        fd = np.zeros_like(P)
+        for pos in np.ndindex(P.shape):
+            keep = P[pos]
+            P[pos] = keep + eps
+            up = (_np_forward(**params, idx=idx, N_c=N_c) * dy64).sum()
+            P[pos] = keep - eps
+            dn = (_np_forward(**params, idx=idx, N_c=N_c) * dy64).sum()
+            P[pos] = keep
+            fd[pos] = (up - dn) / (2 * eps)
+        got = grads[names[pname]]
+        scale = np.abs(fd).max()
+        assert scale > 1e-3, pname                      # the check is not vacuous
+        # the oracle runs on fp32 gates and log-probabilities (as the GPU does)
+        np.testing.assert_allclose(got, fd, rtol=0, atol=2e-5 * scale, err_msg=pname)
+
+
+def test_backward_single_expert_has_no_router_gradient():
+    """K = 1: the gate is softmax of one score, identically 1, so nothing
+    reaches the router; the expert part reduces to one SiLU unit."""
+    rng = np.random.default_rng(8)
+    L, d, N_r, N_c = 4, 16, 6, 6
+    xu, x = _bf16_values(rng, (L, d), 1.0)
+    Wu, W = _bf16_values(rng, (N_r * N_c, d), 0.4)
+    Vu, V = _bf16_values(rng, (N_r * N_c, d), 0.4)
+    Wru, _ = _bf16_values(rng, (N_r, d), 0.5)
+    Wcu, _ = _bf16_values(rng, (N_c, d), 0.5)
+    dy = rng.normal(0.0, 1.0, size=(L, d)).astype(np.float32)
+    p_r, p_c = oracle.router_logprobs(xu, Wru, Wcu)
+    idx, _, gate = oracle.topk_from_logprobs(p_r, p_c, 1)
+    assert np.all(gate == 1.0)
+    g = oracle.routed_bwd(xu, Wu, Vu, Wru, Wcu, p_r, p_c, idx, gate, dy)
+    assert np.abs(g["dW_r"]).max() < 1e-12 and np.abs(g["dW_c"]).max() < 1e-12
+    for t in range(L):
+        e = idx[t, 0]
+        h = x[t] @ W[e]
+        s = 1.0 / (1.0 + np.exp(-h))
+        c = dy[t].astype(np.float64) @ V[e]
+        np.testing.assert_allclose(g["dgate"][t, 0], h * s * c, rtol=1e-12)
+        np.testing.assert_allclose(g["dx"][t], c * s * (1 + h * (1 - s)) * W[e], rtol=1e-10,
+                                   atol=1e-14)
