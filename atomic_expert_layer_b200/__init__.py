@@ -14,7 +14,8 @@ from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_TOPK_BLOCKWIS
                    OMNI_Y_ACCUMULATE,
                    OmniError, load,
                    expert_workspace, omni_expert_workspace_size, omni_get_device_status,
-                   omni_grouped_expert_fwd, omni_grouped_expert_fwd_noalloc, omni_routed_fwd,
+                   omni_grouped_expert_fwd, omni_grouped_expert_fwd_noalloc, omni_routed_bwd,
+                   omni_routed_fwd,
                    omni_router_topk,
                    omni_router_workspace_size, omni_schedule, omni_schedule_workspace_size,
                    omni_selftest_wait_timeout,
@@ -24,7 +25,7 @@ __all__ = [
     "load", "OmniError", "OMNI_ROUTER_LOGPROBS_IN", "OMNI_Y_ACCUMULATE", "OMNI_TOKEN_ORDER", "OMNI_TOPK_BLOCKWISE",
     "omni_workspace_size", "omni_router_topk", "omni_schedule", "omni_grouped_expert_fwd",
     "omni_routed_fwd", "omni_get_device_status", "workspace", "omni_grouped_expert_fwd_noalloc",
-    "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd",
+    "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd", "omni_routed_bwd", "routed_bwd",
 ]
 
 
@@ -98,3 +99,24 @@ def routed_fwd(x, W, V, W_r, W_c, K, B, y=None, ws=None, want_routing=False, acc
     flags = (OMNI_Y_ACCUMULATE if accumulate else 0) | (OMNI_TOKEN_ORDER if token_order else 0)
     omni_routed_fwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, B, y, idx, gate, flags, ws, stream)
     return (y, idx, gate) if want_routing else y
+
+
+def routed_bwd(x, W, V, W_r, W_c, idx, gate, dy, dW=None, dV=None, dW_r=None, dW_c=None,
+               ws=None, stream=None):
+    """Backward of the routed branch with the forward's routing (idx, gate)
+    fixed.  Returns dx (new) and the weight gradients, accumulated into the
+    given fp32 buffers (new zeroed ones if None)."""
+    L, d = x.shape
+    N_r, N_c = W_r.shape[0], W_c.shape[0]
+    K = idx.shape[1]
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    dx = torch.empty((L, d), **f32)
+    dW = torch.zeros(W.shape, **f32) if dW is None else dW
+    dV = torch.zeros(V.shape, **f32) if dV is None else dV
+    dW_r = torch.zeros(W_r.shape, **f32) if dW_r is None else dW_r
+    dW_c = torch.zeros(W_c.shape, **f32) if dW_c is None else dW_c
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev) if ws is None else ws
+    omni_routed_bwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, idx, gate, dy, dx, dW, dV, dW_r, dW_c,
+                    0, ws, stream)
+    return dict(dx=dx, dW=dW, dV=dV, dW_r=dW_r, dW_c=dW_c)

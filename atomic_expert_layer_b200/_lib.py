@@ -40,6 +40,8 @@ SIGNATURES = {
                                  _U, _P, _Z, _P], _I),
     "omni_routed_fwd": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _U, _P, _Z, _P],
                         _I),
+    "omni_routed_bwd": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                         _U, _P, _Z, _P], _I),
     "omni_get_device_status": ([_P, _Z, _P, ctypes.POINTER(ctypes.c_int)], _I),
     "omni_selftest_wait_timeout": ([_P, _Z, _I, _P], _I),
     "omni_grouped_expert_fwd_noalloc": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
@@ -169,6 +171,15 @@ def omni_routed_fwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, B, y, idx_out, gate_ou
                                 K, B, _ptr(y), _ptr(idx_out), _ptr(gate_out), flags, _ptr(ws),
                                 ws.numel(), _stream(stream))
     _check("omni_routed_fwd", rc)
+
+
+def omni_routed_bwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, idx, gate, dy, dx, dW, dV, dW_r, dW_c,
+                    flags, ws, stream=None):
+    rc = load().omni_routed_bwd(_ptr(x), _ptr(W), _ptr(V), _ptr(W_r), _ptr(W_c), L, d, N_r, N_c,
+                                K, _ptr(idx), _ptr(gate), _ptr(dy), _ptr(dx), _ptr(dW), _ptr(dV),
+                                _ptr(dW_r), _ptr(dW_c), flags, _ptr(ws), ws.numel(),
+                                _stream(stream))
+    _check("omni_routed_bwd", rc)
 
 
 def omni_get_device_status(ws, stream=None) -> int:

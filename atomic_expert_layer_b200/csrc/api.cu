@@ -347,6 +347,31 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     return OMNI_OK;
 }
 
+int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
+                    const omni_bf16 *W_r, const omni_bf16 *W_c, int L, int d, int N_r, int N_c,
+                    int K, const int32_t *idx, const float *gate, const float *dy, float *dx,
+                    float *dW, float *dV, float *dW_r, float *dW_c, unsigned flags, void *ws,
+                    size_t ws_bytes, omni_stream_t stream) {
+    Sizes sz;
+    int rc = check_common(L, d, N_r, N_c, K, 1, true, &sz);
+    if (rc) return rc;
+    if (flags != 0) return OMNI_ERR_INVALID_ARG;
+    if (!x || !W || !V || !W_r || !W_c || !idx || !gate || !dy || !dx || !dW || !dV || !dW_r ||
+        !dW_c || !ws)
+        return OMNI_ERR_INVALID_ARG;
+    if (d % 256 != 0 || d > OMNI_MAX_D) return OMNI_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(V) || !aligned16(W_r) || !aligned16(W_c) ||
+        !aligned16(dy) || !aligned16(dx) || !aligned16(dW) || !aligned16(dV) ||
+        !aligned16(dW_r) || !aligned16(dW_c))
+        return OMNI_ERR_INVALID_ARG;
+    if (ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return OMNI_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return OMNI_ERR_CUDA;
+    return cuda_rc(launch_routed_bwd(x, W, V, W_r, W_c, sz, idx, gate, dy, dx, dW, dV, dW_r,
+                                     dW_c, ws_at<int>(ws, 0), st));
+}
+
 int omni_selftest_wait_timeout(void *ws, size_t ws_bytes, int limit_ms, omni_stream_t stream) {
     if (!ws || ws_bytes < sizeof(WsHeader) || limit_ms < 1 || limit_ms > 10000)
         return OMNI_ERR_INVALID_ARG;

@@ -97,6 +97,13 @@ cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const ui
                                   float *y, bool accumulate, void *ws, const WsLayout &lay,
                                   cudaStream_t st);
 
+// ---- backward of the routed branch (selection fixed)
+cudaError_t launch_routed_bwd(const uint16_t *x, const uint16_t *W, const uint16_t *V,
+                              const uint16_t *W_r, const uint16_t *W_c, const Sizes &sz,
+                              const int32_t *idx, const float *gate, const float *dy, float *dx,
+                              float *dW, float *dV, float *dW_r, float *dW_c, int *status,
+                              cudaStream_t st);
+
 int device_sm_count();
 
 }  // namespace omni

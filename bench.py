@@ -78,6 +78,10 @@ def barrier(world: int):
         dist.barrier()
 
 
+def peaks_hbm() -> float:
+    return measured_peaks()["hbm_gbs"]
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -350,6 +354,50 @@ def run_omni(args, cfg, world, rank, local):
         del ws_r2, o
 
 
+    # ---- backward of the routed branch (routing of the forward fixed): dx,
+    # and fp32 weight gradients accumulated into resident buffers
+    bwd = None
+    free_b, _ = torch.cuda.mem_get_info(dev)
+    need = 8 * cfg.N * d + 16 * L * d + (64 << 20)
+    if free_b > need + (4 << 30):
+        f32 = dict(dtype=torch.float32, device=dev)
+        g_dW, g_dV = torch.zeros((cfg.N, d), **f32), torch.zeros((cfg.N, d), **f32)
+        g_dWr, g_dWc = torch.zeros((cfg.N_r, d), **f32), torch.zeros((cfg.N_c, d), **f32)
+        g_dx = torch.empty((L, d), **f32)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(11)
+        g_dy = torch.randn((L, d), generator=gen, **f32)
+        ws_b = torch.zeros(256, dtype=torch.uint8, device=dev)
+
+        def bstep():
+            omni.omni_routed_bwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r,
+                                 cfg.N_c, cfg.K, rt["idx"], rt["gate"], g_dy, g_dx, g_dW, g_dV,
+                                 g_dWr, g_dWc, 0, ws_b)
+
+        for _ in range(3):
+            bstep()
+        nb = max(3, min(args.steps, 20))
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(nb)]
+        torch.cuda.synchronize()
+        for i in range(nb):
+            flush.zero_()
+            bev[i][0].record(stream)
+            bstep()
+            bev[i][1].record(stream)
+        torch.cuda.synchronize()
+        if omni.omni_get_device_status(ws_b) != 0:
+            raise RuntimeError("device status set in the backward")
+        bms = float(np.mean([a.elapsed_time(b) for a, b in bev]))
+        # read x, dy and the U distinct W, V rows; read-modify-write their fp32
+        # dW, dV rows; write dx
+        bbytes = 4.0 * d * U + 16.0 * d * U + 2.0 * L * d + 4.0 * L * d + 4.0 * L * d
+        bwd = {"ms_per_step": bms, "value": L / (bms * 1e-3), "unit": "tokens/s",
+               "steps": nb, "algorithmic_bytes": bbytes,
+               "hbm_frac": bbytes / (bms * 1e-3) / (peaks_hbm() * 1e9)}
+        del g_dW, g_dV, g_dWr, g_dWc, g_dx, g_dy, ws_b
+        torch.cuda.empty_cache()
+
     # ---- end to end: host buffers, copies inside the timed region.  Every
     # step copies its token batch in from pinned host memory and its y out to
     # pinned host memory.  Steps are pipelined over three streams (copy-in of
@@ -451,6 +499,7 @@ def run_omni(args, cfg, world, rank, local):
         "graph": graph,
         "ablation": ablation,
         "topk_compare": topk_cmp,
+        "backward": bwd,
         "clocks": clocks,
     }
     del t, ws, flush

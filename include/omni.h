@@ -206,6 +206,34 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                     unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
 
 /*
+ * Backward of the routed branch.  The pages give the forward only; this is
+ * its derivative with the forward's top-K selection held fixed (a selection
+ * has no gradient).  Per task (t, k), e = idx[t,k], g = gate[t,k]:
+ *   h = x_t . w_e, a = SiLU(h), c = dy_t . v_e,  dgate = a c,
+ *   dV[e] += g a dy_t,  dW[e] += g c SiLU'(h) x_t,  dx_t += g c SiLU'(h) w_e;
+ * through the gate softmax dS_k = g_k (dgate_k - sum_j g_j dgate_j), through
+ * S = p_r[i] + p_c[j] and the LogSoftmax (whose dense term vanishes because
+ * the selected gates sum to 1) the router gradient is sparse:
+ *   dx_t += dS_k (W_r[i] + W_c[j]),  dW_r[i] += dS_k x_t,  dW_c[j] += dS_k x_t.
+ *   x [L, d], W, V [N, d], W_r [N_r, d], W_c [N_c, d]  bf16 (the forward's)
+ *   idx [L, K] int32, gate [L, K] fp32  the forward's routing (omni_router_topk,
+ *                                       or omni_routed_fwd's idx_out / gate_out)
+ *   dy [L, d] fp32     gradient of the loss with respect to y
+ *   dx [L, d] fp32     output, overwritten
+ *   dW, dV [N, d] fp32 accumulated (+=) in the rows of the experts used
+ *   dW_r [N_r, d], dW_c [N_c, d] fp32  accumulated (+=)
+ * The weight gradients are sums of fp32 reductions: their last bits vary
+ * between runs.  ws: at least 256 bytes (the status word).  All fp32 arrays
+ * 16-byte aligned.  Limits: d % 256 == 0, d <= OMNI_MAX_D, K <= OMNI_MAX_K.
+ */
+int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
+                    const omni_bf16 *W_r, const omni_bf16 *W_c,
+                    int L, int d, int N_r, int N_c, int K,
+                    const int32_t *idx, const float *gate, const float *dy,
+                    float *dx, float *dW, float *dV, float *dW_r, float *dW_c,
+                    unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
+
+/*
  * omni_grouped_expert_fwd without a workspace, for callers that cannot
  * allocate device memory when they run the layer (a serving runtime whose
  * memory is planned once at start-up, code where cudaMalloc is not allowed).
