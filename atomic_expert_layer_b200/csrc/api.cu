@@ -157,13 +157,23 @@ int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c
     } else {
         float *s_r = ws_at<float>(ws, lay.s_r), *s_c = ws_at<float>(ws, lay.s_c);
         float *part_r = ws_at<float>(ws, lay.part_r), *part_c = ws_at<float>(ws, lay.part_c);
-        e = launch_router_gemm(x, W_r, W_c, sz.L, sz.d, sz.N_r, sz.N_c, s_r, s_c, part_r, part_c,
-                               status, st);
+        if (router_small_ok(sz.L, sz.d)) {
+            // a handful of tokens: streamed projection, LogSoftmax in the axis kernels
+            e = launch_router_small(x, W_r, W_c, sz.L, sz.d, sz.N_r, sz.N_c, s_r, s_c, st);
+            part_r = part_c = nullptr;
+        } else {
+            e = launch_router_gemm(x, W_r, W_c, sz.L, sz.d, sz.N_r, sz.N_c, s_r, s_c, part_r,
+                                   part_c, status, st);
+        }
         if (e != cudaSuccess) return OMNI_ERR_CUDA;
         e = launch_axis_topk(s_r, s_c, true, part_r, part_c, p_r, p_c, sz.L, sz.N_r, sz.N_c,
                              sz.K, row_val, row_idx, col_val, col_idx, row_flags, status, st);
-        dead_r = s_r;                      // the logits are dead after the axis kernels
-        dead_c = s_c;
+        // the logits are dead after the axis kernels; large ones are dropped
+        // from L2 unwritten (small ones cost more to drop than to keep)
+        if ((size_t)4 * sz.L * (sz.N_r + sz.N_c) >= ((size_t)16 << 20)) {
+            dead_r = s_r;
+            dead_c = s_c;
+        }
     }
     if (e != cudaSuccess) return OMNI_ERR_CUDA;
     e = launch_merge_topk(row_val, row_idx, col_val, col_idx, sz.L, sz.N_c, sz.K, sz.Kr, sz.Kc,

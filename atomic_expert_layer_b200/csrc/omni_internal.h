@@ -59,6 +59,12 @@ cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *W_r, const uin
                                float *part_r, float *part_c, int *status, cudaStream_t st);
 constexpr int kGemmPartCols = 64;          // columns per LogSoftmax partial
 
+// ---- router projection for a handful of tokens (no LogSoftmax partials)
+bool router_small_ok(int L, int d);
+cudaError_t launch_router_small(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c,
+                                int L, int d, int N_r, int N_c, float *s_r, float *s_c,
+                                cudaStream_t st);
+
 // ---- per-axis LogSoftmax (optional) + top-K; then grid merge + gates
 // With part_r / part_c (from the router GEMM) the LogSoftmax uses the
 // per-tile partials; without them it computes max and sum itself.

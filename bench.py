@@ -513,14 +513,24 @@ def profile_stage(args, cfg):
     dev = torch.device("cuda", 0)
     omni.load()
     t = inputs.make_inputs(cfg, dev, seed=0,
-                           with_experts=args.profile_stage in ("expert", "all"))
+                           with_experts=args.profile_stage in ("expert", "all", "backward"))
     L, d = cfg.L, cfg.d
     rt = omni.router_topk(t["x"], t["W_r"], t["W_c"], cfg.K)
     sc = omni.schedule(rt["idx"], rt["gate"], cfg.N, cfg.B)
     ws = omni.workspace(L, d, cfg.N_r, cfg.N_c, cfg.K, cfg.B, dev)
     y = torch.zeros((L, d), dtype=torch.float32, device=dev)
+    if args.profile_stage == "backward":
+        f32 = dict(dtype=torch.float32, device=dev)
+        g = dict(dx=torch.empty((L, d), **f32), dW=torch.zeros((cfg.N, d), **f32),
+                 dV=torch.zeros((cfg.N, d), **f32), dW_r=torch.zeros((cfg.N_r, d), **f32),
+                 dW_c=torch.zeros((cfg.N_c, d), **f32))
+        dy = torch.ones((L, d), **f32)
     for _ in range(args.warmup + args.steps):
-        if args.profile_stage == "router":
+        if args.profile_stage == "backward":
+            omni.omni_routed_bwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r,
+                                 cfg.N_c, cfg.K, rt["idx"], rt["gate"], dy, g["dx"], g["dW"],
+                                 g["dV"], g["dW_r"], g["dW_c"], 0, ws)
+        elif args.profile_stage == "router":
             omni.omni_router_topk(t["x"], t["W_r"], t["W_c"], L, d, cfg.N_r, cfg.N_c, cfg.K,
                                   rt["p_r"], rt["p_c"], rt["idx"], rt["score"], rt["gate"], 0, ws)
         elif args.profile_stage == "schedule":
@@ -575,7 +585,7 @@ def timeline(args, cfg):
                   if e.device_type == torch.autograd.DeviceType.CUDA)
     steps, cur = [], None
     for a, b, n in rows:
-        if "router_gemm" in n:
+        if "router_gemm" in n or "router_small" in n:      # a step's first kernel
             cur = []
             steps.append(cur)
         if cur is not None and "omni::" in n:
@@ -683,7 +693,7 @@ def main():
                     help="workload name: " + ", ".join(c.name for c in configs.ALL))
     ap.add_argument("--impl", choices=["omni", "reference"], default="omni")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-stage", choices=["router", "schedule", "expert", "all"],
+    ap.add_argument("--profile-stage", choices=["router", "schedule", "expert", "all", "backward"],
                     help="run only this stage W + K times (for profiler captures; no JSON)")
     ap.add_argument("--timeline", action="store_true",
                     help="print the in-stream kernel timeline of the last of K steps (no JSON)")

@@ -111,9 +111,13 @@ def test_router_full_tiny_against_oracle():
 
 
 @pytest.mark.parametrize("L,d,N_r,N_c", [(1, 256, 64, 64), (130, 768, 100, 37),
-                                          (257, 2048, 1304, 1304), (64, 200, 16, 300)])
+                                          (257, 2048, 1304, 1304), (64, 200, 16, 300),
+                                          (16, 2048, 1304, 1304), (7, 200, 100, 37),
+                                          (3, 512, 8, 2000), (17, 1024, 1304, 1304)])
 def test_router_gemm_logprobs_shapes(L, d, N_r, N_c):
-    """Ragged L, N_r, N_c and d (d = 200 is not a multiple of the 64-wide K step)."""
+    """Ragged L, N_r, N_c and d (d = 200 is not a multiple of the 64-wide K step);
+    L <= 4 takes the streamed projection with LogSoftmax in the axis kernels,
+    larger L the tensor-core GEMM with fused partials."""
     cfg = configs.LayerConfig("t", L, d, N_r, N_c, 4, 4)
     t = inputs.make_inputs(cfg, DEV, seed=5, with_experts=False)
     u = {k: host(v) for k, v in t.items()}
@@ -374,4 +378,7 @@ def test_routed_bwd_accumulates():
                            dW_r=out["dW_r"].clone(), dW_c=out["dW_c"].clone())
     np.testing.assert_allclose(host(out2["dx"]), host(out["dx"]), rtol=0, atol=1e-6)
     for k in ("dW", "dV", "dW_r", "dW_c"):
-        np.testing.assert_allclose(host(out2[k]), 2 * host(out[k]), rtol=1e-5, atol=1e-7)
+        # fp32 reductions land in a run-dependent order: compare at fp32 scale
+        ref = 2 * host(out[k])
+        np.testing.assert_allclose(host(out2[k]), ref, rtol=0,
+                                   atol=1e-5 * float(np.abs(ref).max()))
