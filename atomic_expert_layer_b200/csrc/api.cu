@@ -8,6 +8,7 @@
 
 #include "omni_common.cuh"
 #include "omni_internal.h"
+#include "sched_token.cuh"
 
 namespace omni {
 
@@ -138,13 +139,14 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? OMNI_OK : OMNI_ERR_CUDA; 
 
 // Clears the status word and the counters the call's kernels accumulate into.
 int reset_workspace(void *ws, const WsLayout &lay, cudaStream_t st) {
+    first_launch_in_call();             // the next kernel follows this memset
     return cuda_rc(cudaMemsetAsync(ws, 0, lay.zero_end, st));
 }
 
 int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c,
                      const Sizes &sz, float *p_r, float *p_c, int32_t *idx, float *score,
                      float *gate, unsigned flags, void *ws, const WsLayout &lay,
-                     cudaStream_t st) {
+                     cudaStream_t st, const SchedPrep *prep = nullptr) {
     int *status = ws_at<int>(ws, lay.hdr);
     float *row_val = ws_at<float>(ws, lay.row_val), *col_val = ws_at<float>(ws, lay.col_val);
     int *row_idx = ws_at<int>(ws, lay.row_idx), *col_idx = ws_at<int>(ws, lay.col_idx);
@@ -177,7 +179,7 @@ int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c
     }
     if (e != cudaSuccess) return OMNI_ERR_CUDA;
     e = launch_merge_topk(row_val, row_idx, col_val, col_idx, sz.L, sz.N_c, sz.K, sz.Kr, sz.Kc,
-                          sz.C, idx, score, gate, dead_r, dead_c, sz.N_r, st);
+                          sz.C, idx, score, gate, dead_r, dead_c, sz.N_r, prep, st);
     return cuda_rc(e);
 }
 
@@ -327,10 +329,14 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     if ((rc = reset_workspace(ws, lay, st))) return rc;
     int32_t *idx = ws_at<int32_t>(ws, lay.idx);
     float *score = ws_at<float>(ws, lay.score), *gate = ws_at<float>(ws, lay.gate);
+    const bool token_order = (flags & OMNI_TOKEN_ORDER) || L <= kTokenOrderMaxL;
+    // scheduled path: the merge kernel also runs the schedule's per-token step
+    const SchedPrep prep = sched_prep_of(sz, ws, lay);
     rc = router_topk_impl(x, W_r, W_c, sz, nullptr, nullptr, idx, score, gate,
-                          flags & ~OMNI_ROUTER_LOGPROBS_IN, ws, lay, st);
+                          flags & ~OMNI_ROUTER_LOGPROBS_IN, ws, lay, st,
+                          token_order ? nullptr : &prep);
     if (rc) return rc;
-    if ((flags & OMNI_TOKEN_ORDER) || L <= kTokenOrderMaxL) {
+    if (token_order) {
         // tasks in token order, read straight from the routing (no schedule)
         if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, nullptr, idx, gate, y,
                                                 (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st))))
@@ -342,7 +348,7 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
         int32_t *gact = ws_at<int32_t>(ws, lay.g_act), *nact = ws_at<int32_t>(ws, lay.n_act);
         int32_t *ndist = ws_at<int32_t>(ws, lay.n_dist);
         if ((rc = cuda_rc(launch_schedule(idx, gate, sz, tt, te, tg, goff, gcnt, gact, nact,
-                                          ndist, ws, lay, st))))
+                                          ndist, ws, lay, st, /*prepared=*/true))))
             return rc;
         if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, tt, te, tg, y,
                                                 (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st))))
@@ -377,6 +383,7 @@ int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     if (ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
         return OMNI_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    first_launch_in_call();
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return OMNI_ERR_CUDA;
     return cuda_rc(launch_routed_bwd(x, W, V, W_r, W_c, sz, idx, gate, dy, dx, dW, dV, dW_r,
                                      dW_c, ws_at<int>(ws, 0), st));

@@ -90,6 +90,7 @@ extern "C" int omni_grouped_expert_fwd_noalloc(
     lay.zero_end = kOffCount + 4 * (size_t)L;
     lay.total = kNoAllocBytes;
     // status word and this call's slot counters
+    first_launch_in_call();
     if (cudaMemsetAsync(scratch, 0, lay.zero_end, st) != cudaSuccess) return OMNI_ERR_CUDA;
     const cudaError_t e = launch_grouped_expert(x, W, V, sz, task_token, task_expert, task_gate,
                                                 y, (flags & OMNI_Y_ACCUMULATE) != 0, scratch, lay,

@@ -141,9 +141,9 @@ __device__ __forceinline__ int warp_iscan(int v) {
 }
 
 // ------------------------------------------- programmatic dependent launch
-// Every kernel of the library is launched with programmatic stream
-// serialisation (launch() below): its CTAs may be scheduled while the
-// previous kernel in the stream is still finishing.  Each kernel therefore
+// Kernels of the library are launched with programmatic stream serialisation
+// (launch() below): their CTAs may be scheduled while the previous kernel in
+// the stream is still finishing.  Each kernel therefore
 // calls grid_dependency_wait() in every thread, before its first access to
 // global memory that earlier work in the stream writes or reads; since every
 // kernel waits, a kernel's completion implies that of all earlier ones.
@@ -155,6 +155,16 @@ __device__ __forceinline__ void grid_dependency_wait() {
 __device__ __forceinline__ void grid_dependents_launch() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+
+//
+// griddepcontrol.wait orders a kernel only after earlier KERNELS; a copy or a
+// memset that precedes it in the stream is not covered.  So only launches
+// whose predecessor is one of this library's kernels use the attribute: every
+// entry point calls first_launch_in_call() after its workspace memset, and
+// the next launch() then goes out with ordinary stream ordering.
+inline thread_local bool t_plain_next_launch = false;
+
+inline void first_launch_in_call() { t_plain_next_launch = true; }
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
@@ -168,7 +178,8 @@ inline cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = t_plain_next_launch ? 0 : 1;
+    t_plain_next_launch = false;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 

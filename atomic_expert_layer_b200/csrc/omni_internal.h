@@ -75,10 +75,14 @@ cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftm
                              int *flags, int *status, cudaStream_t st);
 // dead_r / dead_c: the router GEMM's logits in the workspace, dropped from
 // L2 once read (null: nothing is dropped, e.g. caller-owned log-probabilities)
+// prep (may be null): run the schedule's per-token step (sched_token.cuh)
+// on the merged selection too
+struct SchedPrep;
 cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
                               const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
                               int32_t *idx, float *score, float *gate, const float *dead_r,
-                              const float *dead_c, int N_r, cudaStream_t st);
+                              const float *dead_c, int N_r, const SchedPrep *prep,
+                              cudaStream_t st);
 
 // ---- the pages' blockwise grid top-K (alternative to axis + merge); its
 // candidates need L * blockwise_bands(...) * K * 16 bytes at `cand`
@@ -92,7 +96,10 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
                             int32_t *task_token, int32_t *task_expert, float *task_gate,
                             int32_t *group_offsets, int32_t *group_counts,
                             int32_t *active_groups, int32_t *num_active, int32_t *num_distinct,
-                            void *ws, const WsLayout &lay, cudaStream_t st);
+                            void *ws, const WsLayout &lay, cudaStream_t st, bool prepared = false);
+int sched_pass_width(const Sizes &sz);
+uint32_t sched_pass_mask(const Sizes &sz, int p);
+SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay);
 
 // ---- grouped expert stage (expects the per-token slot counters zeroed).
 // task_token == nullptr: the tasks are in token order, task m belongs to

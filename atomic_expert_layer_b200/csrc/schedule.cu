@@ -22,6 +22,7 @@
 //      digits of its output, then one scan of that histogram.
 #include "omni_common.cuh"
 #include "omni_internal.h"
+#include "sched_token.cuh"
 
 namespace omni {
 namespace {
@@ -31,7 +32,7 @@ constexpr int kItemsPerWarp = kSortTile / (kScatterThreads / 32);   // 256
 
 // ------------------------------------------------------------ radix digits
 __device__ __forceinline__ uint32_t digit_of(int32_t e, int B, int shift, uint32_t dmask) {
-    return ((uint32_t)(e / B) >> shift) & dmask;
+    return sched_digit(e, B, shift, dmask);
 }
 
 // ---------------------------------------------------------- 1. prepare
@@ -63,31 +64,14 @@ __global__ void sched_prepare_kernel(const int32_t *__restrict__ idx,
         e_s[k] = e;
     }
     __syncwarp();
-    for (int u0 = 0; u0 < K; u0 += 32) {
-        const int u = u0 + (int)lane;
-        bool fresh = false;
-        if (u < K) {
-            const int32_t eu = e_s[u];
-            int r = 0;
-            for (int v = 0; v < K; ++v) {
-                const int32_t ev = e_s[v];
-                r += (ev < eu) | ((ev == eu) & (v < u));
-            }
-            const int32_t raw = idx[row + u];
-            const float g = (raw < 0 || raw >= N) ? 0.f : gate[row + u];
-            const size_t pos = row + r;
-            a_tok[pos] = t;
-            a_exp[pos] = eu;
-            a_gate[pos] = g;
-            atomicAdd(&counts[eu / B], 1);
-            const uint32_t bit = 1u << (eu & 31);
-            fresh = (atomicOr(&bitmap[eu >> 5], bit) & bit) == 0u;   // first task of expert eu
-            if (hist0)
-                atomicAdd(&hist0[(int64_t)digit_of(eu, B, 0, dmask0) * ntiles + pos / kSortTile], 1);
-        }
-        const int nf = __popc(__ballot_sync(0xffffffffu, fresh));
-        if (lane == 0 && nf) atomicAdd(num_distinct, nf);
-    }
+    SchedPrep o;
+    o.a_tok = a_tok; o.a_exp = a_exp; o.a_gate = a_gate;
+    o.counts = counts; o.bitmap = bitmap; o.num_distinct = num_distinct;
+    o.hist0 = hist0; o.ntiles = ntiles; o.dmask0 = dmask0; o.B = B;
+    sched_token(o, t, K, e_s, [&](int u) {
+        const int32_t raw = idx[row + u];
+        return (raw < 0 || raw >= N) ? 0.f : gate[row + u];
+    });
 }
 
 // ------------------------------------------------ block scan (1024 threads)
@@ -392,14 +376,41 @@ __global__ void __launch_bounds__(kScatterThreads) radix_scatter_kernel(
 
 }  // namespace
 
+int sched_pass_width(const Sizes &sz) {
+    return sz.passes ? (sz.qbits + sz.passes - 1) / sz.passes : 0;
+}
+
+uint32_t sched_pass_mask(const Sizes &sz, int p) {
+    const int width = sched_pass_width(sz);
+    const int shift = p * width;
+    const int w = (sz.qbits - shift) < width ? (sz.qbits - shift) : width;
+    return (1u << w) - 1u;
+}
+
+SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay) {
+    SchedPrep o;
+    o.a_tok = ws_at<int32_t>(ws, lay.a_tok);
+    o.a_exp = ws_at<int32_t>(ws, lay.a_exp);
+    o.a_gate = ws_at<float>(ws, lay.a_gate);
+    o.counts = ws_at<int32_t>(ws, lay.z_cnt);
+    o.bitmap = ws_at<uint32_t>(ws, lay.bitmap);
+    o.num_distinct = ws_at<int32_t>(ws, lay.z_ndist);
+    o.hist0 = sz.passes ? ws_at<int32_t>(ws, lay.hist) : nullptr;
+    o.ntiles = sz.ntiles;
+    o.dmask0 = sz.passes ? sched_pass_mask(sz, 0) : 0u;
+    o.B = sz.B;
+    return o;
+}
+
 cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &sz,
                             int32_t *task_token, int32_t *task_expert, float *task_gate,
                             int32_t *group_offsets, int32_t *group_counts,
                             int32_t *active_groups, int32_t *num_active, int32_t *num_distinct,
-                            void *ws, const WsLayout &lay, cudaStream_t st) {
+                            void *ws, const WsLayout &lay, cudaStream_t st, bool prepared) {
     // The caller has zeroed [0, lay.zero_end) of ws: the status word, the
     // group counters, the distinct-expert counter, the bitmap and the radix
-    // histograms.
+    // histograms.  With `prepared`, the per-token step (sched_token.cuh) has
+    // already run inside the router's merge kernel.
     const int64_t M = sz.M, G = sz.G;
     int *status = ws_at<int>(ws, lay.hdr);
     int32_t *a_tok = ws_at<int32_t>(ws, lay.a_tok), *a_exp = ws_at<int32_t>(ws, lay.a_exp);
@@ -415,15 +426,11 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
     cudaError_t e;
 
     // radix passes over q = e / B, digits of at most 8 bits
-    const int nbits = sz.qbits, passes = sz.passes;
-    const int width = passes ? (nbits + passes - 1) / passes : 0;
-    auto pass_mask = [&](int p) -> uint32_t {
-        const int shift = p * width;
-        const int w = (nbits - shift) < width ? (nbits - shift) : width;
-        return (1u << w) - 1u;
-    };
+    const int passes = sz.passes;
+    const int width = sched_pass_width(sz);
+    auto pass_mask = [&](int p) -> uint32_t { return sched_pass_mask(sz, p); };
 
-    {
+    if (!prepared) {
         const int wpb = 8;
         const size_t smem = sizeof(int32_t) * (size_t)sz.K * wpb;
         e = launch(sched_prepare_kernel, dim3((unsigned)((sz.L + wpb - 1) / wpb)), dim3(32 * wpb),
@@ -440,7 +447,9 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
     if (passes == 0) {
         if ((e = cudaMemcpyAsync(task_token, a_tok, 4 * M, cudaMemcpyDeviceToDevice, st))) return e;
         if ((e = cudaMemcpyAsync(task_expert, a_exp, 4 * M, cudaMemcpyDeviceToDevice, st))) return e;
-        return cudaMemcpyAsync(task_gate, a_gate, 4 * M, cudaMemcpyDeviceToDevice, st);
+        e = cudaMemcpyAsync(task_gate, a_gate, 4 * M, cudaMemcpyDeviceToDevice, st);
+        first_launch_in_call();         // a kernel after these copies must not overlap them
+        return e;
     }
     const int32_t *s_tok = a_tok, *s_exp = a_exp;
     const float *s_gate = a_gate;

@@ -30,8 +30,11 @@
 // more candidates than the kernel's capacity, an exact radix select (4
 // passes of 8 bits over order-preserving keys) followed by a rank sort is
 // used instead.
+#include <cstring>
+
 #include "omni_common.cuh"
 #include "omni_internal.h"
+#include "sched_token.cuh"
 
 namespace omni {
 namespace {
@@ -589,7 +592,8 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
                                   const int *__restrict__ col_idx, int L, int N_c, int K, int Kr,
                                   int Kc, int C, int32_t *__restrict__ idx,
                                   float *__restrict__ score, float *__restrict__ gate,
-                                  const float *dead_r, const float *dead_c, int N_r) {
+                                  const float *dead_r, const float *dead_c, int N_r,
+                                  SchedPrep prep) {
     extern __shared__ __align__(16) uint32_t smem_u[];
     grid_dependency_wait();
     grid_dependents_launch();
@@ -755,9 +759,17 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     const float den = warp_sum(part);
     for (int k = lane; k < K; k += 32) {
         const float S = out_S[k];
+        const float g = expf(S - smx) / den;
         idx[(size_t)t * K + k] = (int32_t)out_n[k];
         score[(size_t)t * K + k] = S;
-        gate[(size_t)t * K + k] = expf(S - smx) / den;
+        gate[(size_t)t * K + k] = g;
+        out_S[k] = g;                                 // this lane's entries only
+    }
+    if (prep.a_tok) {
+        // the schedule's per-token step on the selection still on chip
+        __syncwarp();
+        sched_token(prep, t, K, reinterpret_cast<const int32_t *>(out_n),
+                    [&](int u) { return out_S[u]; });
     }
 }
 
@@ -878,7 +890,11 @@ template <int CAP>
 static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, const float *col_val,
                                   const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
                                   int32_t *idx, float *score, float *gate, const float *dead_r,
-                                  const float *dead_c, int N_r, cudaStream_t st) {
+                                  const float *dead_c, int N_r, const SchedPrep *prep,
+                                  cudaStream_t st) {
+    SchedPrep pv;
+    std::memset(&pv, 0, sizeof pv);
+    if (prep) pv = *prep;
     const MergeLayout ml = merge_layout(K, Kr, Kc, C);
     const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
     const size_t per_warp = ml.words * 4;
@@ -894,17 +910,18 @@ static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, cons
     }
     const unsigned grid = (unsigned)((L + wpb - 1) / wpb);
     return launch(merge_topk_kernel<CAP>, dim3(grid), dim3(32 * wpb), smem, st, row_val, row_idx,
-                  col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, dead_r, dead_c, N_r);
+                  col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, dead_r, dead_c, N_r,
+                  pv);
 }
 
 cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const float *col_val,
                               const int *col_idx, int L, int N_c, int K, int Kr, int Kc, int C,
                               int32_t *idx, float *score, float *gate, const float *dead_r,
-                              const float *dead_c, int N_r, cudaStream_t st) {
-    // the candidate keys (4 words each) live in the Cand area (4 words per candidate)
+                              const float *dead_c, int N_r, const SchedPrep *prep,
+                              cudaStream_t st) {
     int cap = fast_capacity(K);
     if (cap > C) cap = C >= K ? (C / 32) * 32 : 0;
-#define OMNI_MG(c) return launch_merge_e<c>(row_val, row_idx, col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, dead_r, dead_c, N_r, st);
+#define OMNI_MG(c) return launch_merge_e<c>(row_val, row_idx, col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, dead_r, dead_c, N_r, prep, st);
     if (cap < K) { OMNI_MG(0) }
     if (cap <= 96) { OMNI_MG(96) }
     if (cap <= 192) { OMNI_MG(192) }

@@ -119,9 +119,11 @@ grid_band_topk_kernel(const float *__restrict__ p_r, const float *__restrict__ p
         const float pr = pr_s[i - r0];
         const uint32_t prk = f2key(pr);
         for (int j0 = 0; j0 < N_c; j0 += kColChunk) {
-            if (cnt + kColChunk > kBandBuf) {            // the same value in every thread
-                const int c = cnt;
-                __syncthreads();
+            // every thread reads the count before any thread appends to it,
+            // so all take the same branch (and meet the same barriers)
+            const int c = cnt;
+            __syncthreads();
+            if (c + kColChunk > kBandBuf) {
                 uint32_t tn = T;
                 const int kept = compact_cells(buf, c, K, &tn);
                 __syncthreads();
@@ -138,12 +140,12 @@ grid_band_topk_kernel(const float *__restrict__ p_r, const float *__restrict__ p
                 const uint32_t sk = f2key(S);
                 if (sk >= thr) {
                     const int pos = atomicAdd(&cnt, 1);
-                    Cell c;
-                    c.skey = sk;
-                    c.prkey = prk;
-                    c.pckey = f2key(pc_s[j]);
-                    c.n = (uint32_t)i * (uint32_t)N_c + (uint32_t)j;
-                    buf[pos] = c;
+                    Cell cell;
+                    cell.skey = sk;
+                    cell.prkey = prk;
+                    cell.pckey = f2key(pc_s[j]);
+                    cell.n = (uint32_t)i * (uint32_t)N_c + (uint32_t)j;
+                    buf[pos] = cell;
                 }
             }
             __syncthreads();
