@@ -23,6 +23,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import tempfile
@@ -595,7 +596,8 @@ def timeline(args, cfg):
     t0, prev_end = last[0][0], last[0][0]
     print(f"{'kernel':44s} {'start us':>9s} {'end us':>9s} {'end delta':>10s}")
     for a, b, n in last:
-        short = n.split("::")[-1].split("(")[0][:44]
+        m = re.search(r"(\w+(?:<[\d, ]+>)?)\((?!anonymous)", n)    # the kernel's own name
+        short = (m.group(1) if m else n)[:44]
         print(f"{short:44s} {a - t0:9.2f} {b - t0:9.2f} {b - prev_end:10.2f}")
         prev_end = max(prev_end, b)
     print(f"first kernel start to last kernel end, per step (us): "
