@@ -109,8 +109,8 @@ def launches_per_step(cfg) -> int:
     reg = cfg.N_r % 4 == 0 and cfg.N_c % 4 == 0 and nmax <= 2048 and 0 < cap <= 320
     router = 1 + (2 if reg else 1) + 1            # GEMM, axis top-K (+ flagged redo), merge
     p = radix_passes(cfg.G)
-    sched = 2 + (p + max(p - 1, 0))               # prepare, scan, scatters, histogram scans
-    if cfg.L <= 16:
+    sched = 1 + (p + max(p - 1, 0))               # scan, scatters, histogram scans (the
+    if cfg.L <= 16:                               # per-token step runs in the merge kernel)
         sched = 0                                 # decode batches run in token order
     return router + sched + 2                     # group pass, token pass
 
