@@ -93,6 +93,24 @@ def test_bad_arguments_rejected_on_host(lib):
     # router: d must be a multiple of 8
     assert lib.omni_router_topk(fake, fake, fake, L, 12, Nr, Nc, K, fake, fake, fake, fake, fake,
                                 0, fake, 1 << 30, None) == -2
+    # blockwise selection: only on caller log-probabilities, and K <= (N_r + N_c) / 4
+    lp_bw = 1 | 8                           # OMNI_ROUTER_LOGPROBS_IN | OMNI_TOPK_BLOCKWISE
+    assert lib.omni_router_topk(fake, fake, fake, L, d, Nr, Nc, K, fake, fake, fake, fake, fake,
+                                8, fake, 1 << 30, None) == -2
+    assert lib.omni_router_topk(None, None, None, L, 0, 8, 8, 16, fake, fake, fake, fake, fake,
+                                lp_bw, fake, 1 << 30, None) == -2
+    # ... and not through the whole forward
+    assert lib.omni_routed_fwd(fake, fake, fake, fake, fake, L, d, Nr, Nc, K, B, fake, None,
+                               None, 8, fake, 1 << 30, None) == -2
+    # backward: null gradient buffer, unknown flag, d off the 256 grid, tiny workspace
+    assert lib.omni_routed_bwd(fake, fake, fake, fake, fake, L, d, Nr, Nc, K, fake, fake, fake,
+                               fake, None, fake, fake, fake, 0, fake, 256, None) == -1
+    assert lib.omni_routed_bwd(fake, fake, fake, fake, fake, L, d, Nr, Nc, K, fake, fake, fake,
+                               fake, fake, fake, fake, fake, 1, fake, 256, None) == -1
+    assert lib.omni_routed_bwd(fake, fake, fake, fake, fake, L, 264, Nr, Nc, K, fake, fake, fake,
+                               fake, fake, fake, fake, fake, 0, fake, 256, None) == -2
+    assert lib.omni_routed_bwd(fake, fake, fake, fake, fake, L, d, Nr, Nc, K, fake, fake, fake,
+                               fake, fake, fake, fake, fake, 0, fake, 64, None) == -3
     # status query needs a workspace
     out = ctypes.c_int(7)
     assert lib.omni_get_device_status(None, 0, None, ctypes.byref(out)) == -1
