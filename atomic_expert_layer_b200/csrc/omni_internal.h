@@ -9,7 +9,6 @@
 namespace omni {
 
 constexpr int kSortTile = 2048;        // tasks per radix-sort tile
-constexpr int kItemTasks = 128;        // sorted tasks per grouped-expert work item
 
 struct Sizes {
     int L, d, N_r, N_c, K, B;

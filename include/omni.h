@@ -75,7 +75,7 @@ typedef enum {
 #define OMNI_DEV_WAIT_TIMEOUT    2  /* a bounded barrier wait ran out (no hang)           */
 #define OMNI_DEV_BAD_SCHEDULE    3  /* schedule arrays inconsistent (offsets/ids)          */
 
-/* Size limits of this build (OMNI_ERR_UNSUPPORTED beyond them). */
+/* Size limits of the library (OMNI_ERR_UNSUPPORTED beyond them). */
 #define OMNI_MAX_AXIS   8192        /* N_r, N_c                                   */
 #define OMNI_MAX_K      512         /* K                                          */
 #define OMNI_MAX_B      1024        /* B                                          */
