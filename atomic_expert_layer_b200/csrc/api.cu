@@ -330,8 +330,10 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     int32_t *idx = ws_at<int32_t>(ws, lay.idx);
     float *score = ws_at<float>(ws, lay.score), *gate = ws_at<float>(ws, lay.gate);
     const bool token_order = (flags & OMNI_TOKEN_ORDER) || L <= kTokenOrderMaxL;
-    // scheduled path: the merge kernel also runs the schedule's per-token step
-    const SchedPrep prep = sched_prep_of(sz, ws, lay);
+    // scheduled path: the merge kernel also runs the schedule's per-token step;
+    // nothing here reads the distinct-expert count, so it is not kept
+    SchedPrep prep = sched_prep_of(sz, ws, lay);
+    prep.bitmap = nullptr;
     rc = router_topk_impl(x, W_r, W_c, sz, nullptr, nullptr, idx, score, gate,
                           flags & ~OMNI_ROUTER_LOGPROBS_IN, ws, lay, st,
                           token_order ? nullptr : &prep);

@@ -25,7 +25,7 @@ struct SchedPrep {          // where the per-token step writes (all in the works
     int32_t *a_tok, *a_exp;
     float *a_gate;
     int32_t *counts;        // [G], zeroed by the caller
-    uint32_t *bitmap;       // [ceil(N / 32)], zeroed
+    uint32_t *bitmap;       // [ceil(N / 32)], zeroed; null: distinct experts not counted
     int32_t *num_distinct;  // [1], zeroed
     int32_t *hist0;         // [digits][ntiles] of the first pass, zeroed; null: no radix pass
     int64_t ntiles;
@@ -58,14 +58,16 @@ __device__ __forceinline__ void sched_token(const SchedPrep &o, int t, int K, co
             o.a_exp[pos] = eu;
             o.a_gate[pos] = gate_of(u);
             atomicAdd(&o.counts[eu / o.B], 1);
-            const uint32_t bit = 1u << (eu & 31);
-            fresh = (atomicOr(&o.bitmap[eu >> 5], bit) & bit) == 0u;   // first task of expert eu
+            if (o.bitmap) {
+                const uint32_t bit = 1u << (eu & 31);
+                fresh = (atomicOr(&o.bitmap[eu >> 5], bit) & bit) == 0u;   // first task of eu
+            }
             if (o.hist0)
                 atomicAdd(&o.hist0[(int64_t)sched_digit(eu, o.B, 0, o.dmask0) * o.ntiles +
                                    (int64_t)(pos / kSortTile)], 1);
         }
         const int nf = __popc(__ballot_sync(0xffffffffu, fresh));
-        if (lane == 0 && nf) atomicAdd(o.num_distinct, nf);
+        if (lane == 0 && nf) atomicAdd(o.num_distinct, nf);     // nf = 0 without a bitmap
     }
 }
 
