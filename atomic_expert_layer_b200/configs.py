@@ -59,5 +59,12 @@ def sweep(L: int) -> LayerConfig:
 # with W and V of 512 MB each (N = 512^2) instead of 3.5 GB.
 PROFILE = LayerConfig("profile_L4096_d1024_N262144_K64_B20", 4096, 1024, 512, 512, 64, 20)
 
+def mlp_hidden(d: int) -> int:
+    """Hidden width F of the shared dense MLP beside a layer of width d: 8d/3
+    rounded up to a multiple of 64 (the width at which a gated MLP has the
+    weights of a plain two-matrix MLP of width 4d)."""
+    return -(-8 * d // (3 * 64)) * 64
+
+
 ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L] + [PROFILE]
 BY_NAME = {c.name: c for c in ALL}

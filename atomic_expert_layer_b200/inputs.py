@@ -9,6 +9,10 @@ Recipe (per tensor, its own generator seeded with seed * 16 + tensor index):
   V   [N, d]    ~ N(0, 1/d)
   W_r [N_r, d]  ~ N(0, 1/d)   (one routing vector per grid row)
   W_c [N_c, d]  ~ N(0, 1/d)
+Shared dense MLP weights (make_mlp_weights), hidden width F:
+  W_g [F, d]    ~ N(0, 1/d)   (gate projection, one row per hidden unit)
+  W_u [F, d]    ~ N(0, 1/d)   (up projection)
+  W_d [d, F]    ~ N(0, 1/F)   (down projection, one row per output feature)
 Large tensors are drawn in row chunks of CHUNK_ROWS from the same generator.
 With zipf=True (skewed routing), feature d-1 of every token is set to 1 and
 W_r[i, d-1] = -1.1 * ln(rank_r(i)), W_c[j, d-1] = -1.1 * ln(rank_c(j)), where
@@ -26,7 +30,7 @@ import torch
 from .configs import LayerConfig
 
 CHUNK_ROWS = 1 << 16
-TENSOR_INDEX = {"x": 0, "W": 1, "V": 2, "W_r": 3, "W_c": 4}
+TENSOR_INDEX = {"x": 0, "W": 1, "V": 2, "W_r": 3, "W_c": 4, "W_g": 7, "W_u": 8, "W_d": 9}
 
 
 def _gen(device: torch.device, seed: int, which: str) -> torch.Generator:
@@ -70,6 +74,16 @@ def make_inputs(cfg: LayerConfig, device="cpu", seed: int = 0, with_experts: boo
         out["W_r"][:, cfg.d - 1] = _zipf_bias(cfg.N_r, seed, 5).to(device=device, dtype=torch.bfloat16)
         out["W_c"][:, cfg.d - 1] = _zipf_bias(cfg.N_c, seed, 6).to(device=device, dtype=torch.bfloat16)
     return out
+
+
+def make_mlp_weights(d: int, F: int, device="cpu", seed: int = 0):
+    """Return a dict of bf16 tensors W_g, W_u [F, d] and W_d [d, F] on `device`."""
+    device = torch.device(device)
+    return {
+        "W_g": _normal_bf16(F, d, 1.0 / math.sqrt(d), device, _gen(device, seed, "W_g")),
+        "W_u": _normal_bf16(F, d, 1.0 / math.sqrt(d), device, _gen(device, seed, "W_u")),
+        "W_d": _normal_bf16(d, F, 1.0 / math.sqrt(F), device, _gen(device, seed, "W_d")),
+    }
 
 
 def to_u16(t: torch.Tensor) -> np.ndarray:

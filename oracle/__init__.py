@@ -54,6 +54,7 @@ def _load():
         lib.oracle_expert_fwd_expert_centric.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, I, P]
         lib.oracle_expert_bwd.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P]
         lib.oracle_router_bwd.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P]
+        lib.oracle_shared_mlp.argtypes = [P, P, P, P, I, I, P, I, P, I]
         lib.oracle_max_threads.argtypes = []
         for f in (lib.oracle_router_logprobs, lib.oracle_topk_from_logprobs, lib.oracle_schedule,
                   lib.oracle_expert_fwd_token_centric, lib.oracle_expert_fwd_expert_centric,
@@ -148,6 +149,26 @@ def expert_fwd_token_centric(x, W, V, idx, gate, tokens=None, nthreads: int = 0)
                                                    _p(tok), n, _p(y), nthreads),
            "expert_fwd_token_centric")
     return y
+
+
+def shared_mlp(x, W_g, W_u, W_d, tokens=None, nthreads: int = 0):
+    """fp64 MLP(x) = (SiLU(x W_g^T) * (x W_u^T)) W_d^T for the given tokens
+    (all if None).  W_g, W_u: [F, d]; W_d: [d, F]; bf16 bit patterns."""
+    x, W_g, W_u, W_d = (_c(a, np.uint16) for a in (x, W_g, W_u, W_d))
+    d = x.shape[1]
+    F = W_g.shape[0]
+    if W_g.shape != (F, d) or W_u.shape != (F, d) or W_d.shape != (d, F):
+        raise ValueError("shared_mlp: W_g, W_u must be [F, d] and W_d [d, F]")
+    if tokens is None:
+        n = x.shape[0]
+        tok = None
+    else:
+        tok = _c(tokens, np.int32)
+        n = tok.shape[0]
+    out = np.empty((n, d), np.float64)
+    _check(_load().oracle_shared_mlp(_p(x), _p(W_g), _p(W_u), _p(W_d), d, F, _p(tok), n, _p(out),
+                                     nthreads), "shared_mlp")
+    return out
 
 
 def expert_fwd_expert_centric(x, W, V, sched, B: int):

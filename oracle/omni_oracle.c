@@ -8,7 +8,7 @@
  *   [R]  "OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at Scale",
  *        review at paper.rainbus.top, method paragraph.  Step 1: atomic expert
  *        E_i(x) = sigma(x w_in_i^T) w_out_i, global matrices W, V, retrieval
- *        w_x = W[I_x], assembly y = (g_x . sigma(x w_x^T)) v_x (+ MLP, not here).
+ *        w_x = W[I_x], assembly y = (g_x . sigma(x w_x^T)) v_x + MLP(x).
  *        Step 2: Cartesian product router s_r = x W_r, s_c = x W_c, LogSoftmax
  *        to p_r, p_c, implicit score S_ij = p_r[i] + p_c[j], global top-K.
  *        Step 3: expert-centric scheduling: M = L*K tasks, sorted by expert id,
@@ -16,7 +16,9 @@
  *        per active group O_q = (G_q . sigma(X_q W_q^T)) V_q.
  *   [G]  same title, gist.science summary (German edition), section 2.2
  *        "Experten-zentriertes Scheduling": groups are contiguous ranges of
- *        expert ids, tokens sorted inside each group.
+ *        expert ids, tokens sorted inside each group.  Section 2.1
+ *        "Kernkomponenten": a standard dense MLP branch, active for every
+ *        input, runs beside the routed one.
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *   - sigma is SiLU, z / (1 + exp(-z)) (each expert has a single w_in, so the
@@ -30,6 +32,8 @@
  *     by (token, e).
  *   - W_r is stored as N_r rows of d (the transpose of the d x N_r matrix of
  *     [R]), likewise W_c, so s_r[i] = sum_k x[k] * W_r[i][k].
+ *   - the shared MLP is the gated (SwiGLU) form with hidden width F:
+ *     MLP(x) = (SiLU(x W_g^T) * (x W_u^T)) W_d^T.
  *
  * Floating point: everything is fp64 except where the method fixes fp32 (the
  * log-probabilities that selection runs on, S, and the returned gates).  bf16
@@ -458,5 +462,48 @@ int oracle_router_bwd(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_
     }
     free(dp_r);
     free(dp_c);
+    return 0;
+}
+
+/* ---- The shared dense MLP of [R] step 1 / [G] section 2.1 ----------------
+ * The pages call it a standard dense MLP and give no form; the reading here is
+ * the gated one, SwiGLU being the activation [R] names for the layer:
+ *   a_f = x_t . W_g[f],  b_f = x_t . W_u[f]            (f < F)
+ *   h_f = SiLU(a_f) * b_f
+ *   out[r, c] = sum_f h_f * W_d[c][f]                   (c < d)
+ * W_g and W_u are F rows of d, W_d is d rows of F (each the K-major operand of
+ * its product).  fp64 over the exact bf16 inputs; row r is token
+ * t = tokens[r] (r itself when tokens is NULL).                            */
+int oracle_shared_mlp(const uint16_t *x, const uint16_t *W_g, const uint16_t *W_u,
+                      const uint16_t *W_d, int d, int F, const int32_t *tokens, int n_tokens,
+                      double *out, int nthreads) {
+    if (d <= 0 || F <= 0 || n_tokens < 0) return -1;
+    set_threads(nthreads);
+    #pragma omp parallel
+    {
+        double *xr = (double *)malloc(sizeof(double) * (size_t)d);
+        double *h = (double *)malloc(sizeof(double) * (size_t)F);
+        #pragma omp for schedule(dynamic, 4)
+        for (int r = 0; r < n_tokens; ++r) {
+            const int64_t t = tokens ? tokens[r] : r;
+            for (int c = 0; c < d; ++c) xr[c] = bf16_to_double(x[(size_t)t * d + c]);
+            for (int f = 0; f < F; ++f) {
+                double a = 0.0, b = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    a += xr[c] * bf16_to_double(W_g[(size_t)f * d + c]);
+                    b += xr[c] * bf16_to_double(W_u[(size_t)f * d + c]);
+                }
+                h[f] = silu(a) * b;
+            }
+            double *o = out + (size_t)r * d;
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int f = 0; f < F; ++f) acc += h[f] * bf16_to_double(W_d[(size_t)c * F + f]);
+                o[c] = acc;
+            }
+        }
+        free(xr);
+        free(h);
+    }
     return 0;
 }

@@ -345,3 +345,61 @@ def test_backward_single_expert_has_no_router_gradient():
         np.testing.assert_allclose(g["dgate"][t, 0], h * s * c, rtol=1e-12)
         np.testing.assert_allclose(g["dx"][t], c * s * (1 + h * (1 - s)) * W[e], rtol=1e-10,
                                    atol=1e-14)
+
+
+# ------------------------------------------------------ shared dense MLP
+@pytest.mark.parametrize("case", GOLDEN["mlp"], ids=lambda c: c["name"])
+def test_shared_mlp_hand_examples(case):
+    out = oracle.shared_mlp(bf16_u16(case["x"]), bf16_u16(case["W_g"]), bf16_u16(case["W_u"]),
+                            bf16_u16(case["W_d"]))
+    np.testing.assert_allclose(out, np.array(case["y"]), rtol=1e-14, atol=1e-15)
+
+
+def test_shared_mlp_one_hot_weights_reduce_to_library_silu():
+    """One-hot rows turn every product into a lookup: with W_g[f] = 2 e_{pg(f)},
+    W_u[f] = e_{pu(f)} and W_d[c] = e_{pd(c)}, MLP(x)[c] = silu(2 x[pg(pd(c))])
+    * x[pu(pd(c))], with torch's silu.  The index maps reach every input
+    feature and both ends of the hidden range, and d != F, so a transposed
+    operand, swapped gate and up roles or a dropped term all change the result."""
+    d, F, L = 16, 24, 5
+    pg = (5 * np.arange(F) + 3) % d
+    pu = (3 * np.arange(F) + 7) % d
+    pd = (7 * np.arange(d) + 2) % F
+    assert set(pg) == set(range(d)) and set(pu) == set(range(d)) and {0, F - 1} <= set(pd)
+    W_g = np.zeros((F, d)); W_g[np.arange(F), pg] = 2.0
+    W_u = np.zeros((F, d)); W_u[np.arange(F), pu] = 1.0
+    W_d = np.zeros((d, F)); W_d[np.arange(d), pd] = 1.0
+    rng = np.random.default_rng(11)
+    xu, x = _bf16_values(rng, (L, d), 1.5)
+    out = oracle.shared_mlp(xu, bf16_u16(W_g), bf16_u16(W_u), bf16_u16(W_d))
+    xt = torch.tensor(x, dtype=torch.float64)
+    want = torch.nn.functional.silu(2.0 * xt[:, pg[pd]]) * xt[:, pu[pd]]
+    np.testing.assert_allclose(out, want.numpy(), rtol=1e-14, atol=0)
+
+
+def test_shared_mlp_linear_in_down_projection_and_zero_gate():
+    """MLP is linear in W_d (exact small bf16 values, so W_d1 + W_d2 is exact
+    too), and a zero gate projection gives SiLU(0) = 0 everywhere."""
+    rng = np.random.default_rng(12)
+    d, F, L = 8, 12, 6
+    xu, _ = _bf16_values(rng, (L, d), 1.0)
+    W_g = bf16_u16(rng.integers(-4, 5, size=(F, d)) / 8.0)
+    W_u = bf16_u16(rng.integers(-4, 5, size=(F, d)) / 8.0)
+    D1 = rng.integers(-4, 5, size=(d, F)) / 8.0
+    D2 = rng.integers(-4, 5, size=(d, F)) / 8.0
+    o1 = oracle.shared_mlp(xu, W_g, W_u, bf16_u16(D1))
+    o2 = oracle.shared_mlp(xu, W_g, W_u, bf16_u16(D2))
+    o12 = oracle.shared_mlp(xu, W_g, W_u, bf16_u16(D1 + D2))
+    assert np.abs(o1).max() > 0.1 and np.abs(o2).max() > 0.1
+    np.testing.assert_allclose(o12, o1 + o2, rtol=1e-13, atol=1e-13)
+    zero = oracle.shared_mlp(xu, bf16_u16(np.zeros((F, d))), W_u, bf16_u16(D1))
+    assert np.all(zero == 0.0)
+
+
+def test_shared_mlp_token_subset_matches_full():
+    w = inputs.make_mlp_weights(64, 128, seed=3)
+    x = inputs.make_inputs(configs.TINY, with_experts=False)["x"][:40, :64].contiguous()
+    args = [inputs.to_u16(t) for t in (x, w["W_g"], w["W_u"], w["W_d"])]
+    full = oracle.shared_mlp(*args)
+    tok = np.array([39, 0, 17, 17, 5], np.int32)
+    np.testing.assert_array_equal(oracle.shared_mlp(*args, tokens=tok), full[tok])
