@@ -3,8 +3,9 @@
 The computation lives in libomni.so (hand-written CUDA, C ABI in
 include/omni.h).  This package only loads it and marshals torch tensors:
   - ``omni_*`` functions mirror the C entry points argument for argument;
-  - ``router_topk``, ``schedule``, ``grouped_expert_fwd``, ``routed_fwd``
-    allocate the output tensors and a workspace, then call them.
+  - ``router_topk``, ``schedule``, ``grouped_expert_fwd``, ``routed_fwd``,
+    ``routed_bwd``, ``shared_mlp_fwd`` and ``layer_fwd`` allocate the output
+    tensors and a workspace, then call them.
 """
 from __future__ import annotations
 
@@ -18,7 +19,8 @@ from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_TOPK_BLOCKWIS
                    omni_routed_fwd,
                    omni_router_topk,
                    omni_router_workspace_size, omni_schedule, omni_schedule_workspace_size,
-                   omni_selftest_wait_timeout,
+                   omni_selftest_wait_timeout, omni_shared_mlp_fwd,
+                   omni_shared_mlp_workspace_size, shared_mlp_workspace,
                    omni_workspace_size, router_workspace, schedule_workspace, workspace)
 
 __all__ = [
@@ -26,6 +28,7 @@ __all__ = [
     "omni_workspace_size", "omni_router_topk", "omni_schedule", "omni_grouped_expert_fwd",
     "omni_routed_fwd", "omni_get_device_status", "workspace", "omni_grouped_expert_fwd_noalloc",
     "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd", "omni_routed_bwd", "routed_bwd",
+    "omni_shared_mlp_workspace_size", "omni_shared_mlp_fwd", "shared_mlp_fwd", "layer_fwd",
 ]
 
 
@@ -120,3 +123,23 @@ def routed_bwd(x, W, V, W_r, W_c, idx, gate, dy, dW=None, dV=None, dW_r=None, dW
     omni_routed_bwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, idx, gate, dy, dx, dW, dV, dW_r, dW_c,
                     0, ws, stream)
     return dict(dx=dx, dW=dW, dV=dV, dW_r=dW_r, dW_c=dW_c)
+
+
+def shared_mlp_fwd(x, W_g, W_u, W_d, y=None, accumulate=False, ws=None, stream=None):
+    """MLP(x) = (SiLU(x W_g^T) * (x W_u^T)) W_d^T into y (fp32), or added to
+    it with accumulate=True.  W_g, W_u: [F, d]; W_d: [d, F]; all bf16."""
+    L, d = x.shape
+    F = W_g.shape[0]
+    y = torch.empty((L, d), dtype=torch.float32, device=x.device) if y is None else y
+    ws = shared_mlp_workspace(L, d, F, x.device) if ws is None else ws
+    omni_shared_mlp_fwd(x, W_g, W_u, W_d, L, d, F, y, OMNI_Y_ACCUMULATE if accumulate else 0, ws,
+                        stream)
+    return y
+
+
+def layer_fwd(x, W, V, W_r, W_c, W_g, W_u, W_d, K, B, y=None, ws=None, mlp_ws=None,
+              stream=None):
+    """The whole layer: y = routed(x) + MLP(x), as omni_routed_fwd followed by
+    omni_shared_mlp_fwd with OMNI_Y_ACCUMULATE on the same stream."""
+    y = routed_fwd(x, W, V, W_r, W_c, K, B, y=y, ws=ws, stream=stream)
+    return shared_mlp_fwd(x, W_g, W_u, W_d, y=y, accumulate=True, ws=mlp_ws, stream=stream)

@@ -42,6 +42,8 @@ SIGNATURES = {
                         _I),
     "omni_routed_bwd": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                          _U, _P, _Z, _P], _I),
+    "omni_shared_mlp_workspace_size": ([_I, _I, _I], _Z),
+    "omni_shared_mlp_fwd": ([_P, _P, _P, _P, _I, _I, _I, _P, _U, _P, _Z, _P], _I),
     "omni_get_device_status": ([_P, _Z, _P, ctypes.POINTER(ctypes.c_int)], _I),
     "omni_selftest_wait_timeout": ([_P, _Z, _I, _P], _I),
     "omni_grouped_expert_fwd_noalloc": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
@@ -180,6 +182,20 @@ def omni_routed_bwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, idx, gate, dy, dx, dW,
                                 _ptr(dW_r), _ptr(dW_c), flags, _ptr(ws), ws.numel(),
                                 _stream(stream))
     _check("omni_routed_bwd", rc)
+
+
+def omni_shared_mlp_workspace_size(L, d, F) -> int:
+    return int(load().omni_shared_mlp_workspace_size(L, d, F))
+
+
+def shared_mlp_workspace(L, d, F, device="cuda") -> torch.Tensor:
+    return _alloc(omni_shared_mlp_workspace_size(L, d, F), device)
+
+
+def omni_shared_mlp_fwd(x, W_g, W_u, W_d, L, d, F, y, flags, ws, stream=None):
+    rc = load().omni_shared_mlp_fwd(_ptr(x), _ptr(W_g), _ptr(W_u), _ptr(W_d), L, d, F, _ptr(y),
+                                    flags, _ptr(ws), ws.numel(), _stream(stream))
+    _check("omni_shared_mlp_fwd", rc)
 
 
 def omni_get_device_status(ws, stream=None) -> int:

@@ -391,6 +391,32 @@ int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                                      dW_c, ws_at<int>(ws, 0), st));
 }
 
+size_t omni_shared_mlp_workspace_size(int L, int d, int F) {
+    if (L <= 0 || d <= 0 || F <= 0) return 0;
+    return sizeof(WsHeader) + align256((size_t)L * (size_t)F * 2);
+}
+
+int omni_shared_mlp_fwd(const omni_bf16 *x, const omni_bf16 *W_g, const omni_bf16 *W_u,
+                        const omni_bf16 *W_d, int L, int d, int F, float *y, unsigned flags,
+                        void *ws, size_t ws_bytes, omni_stream_t stream) {
+    if (!x || !W_g || !W_u || !W_d || !y || !ws) return OMNI_ERR_INVALID_ARG;
+    if (L <= 0 || d <= 0 || F <= 0 || (flags & ~OMNI_Y_ACCUMULATE) != 0)
+        return OMNI_ERR_INVALID_ARG;
+    if (d % 64 != 0 || F % 64 != 0) return OMNI_ERR_UNSUPPORTED;
+    if ((int64_t)L * F > INT_MAX || (int64_t)L * d > INT_MAX || (int64_t)F * d > INT_MAX)
+        return OMNI_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(W_g) || !aligned16(W_u) || !aligned16(W_d) || !aligned16(y))
+        return OMNI_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return OMNI_ERR_INVALID_ARG;
+    if (ws_bytes < omni_shared_mlp_workspace_size(L, d, F)) return OMNI_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    first_launch_in_call();
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return OMNI_ERR_CUDA;
+    uint16_t *h = ws_at<uint16_t>(ws, sizeof(WsHeader));
+    return cuda_rc(launch_shared_mlp(x, W_g, W_u, W_d, L, d, F, h, y,
+                                     (flags & OMNI_Y_ACCUMULATE) != 0, ws_at<int>(ws, 0), st));
+}
+
 int omni_selftest_wait_timeout(void *ws, size_t ws_bytes, int limit_ms, omni_stream_t stream) {
     if (!ws || ws_bytes < sizeof(WsHeader) || limit_ms < 1 || limit_ms > 10000)
         return OMNI_ERR_INVALID_ARG;

@@ -116,6 +116,11 @@ cudaError_t launch_routed_bwd(const uint16_t *x, const uint16_t *W, const uint16
                               float *dW, float *dV, float *dW_r, float *dW_c, int *status,
                               cudaStream_t st);
 
+// ---- shared dense MLP (two tile GEMMs; h is [L, F] bf16 scratch)
+cudaError_t launch_shared_mlp(const uint16_t *x, const uint16_t *W_g, const uint16_t *W_u,
+                              const uint16_t *W_d, int L, int d, int F, uint16_t *h, float *y,
+                              bool accumulate, int *status, cudaStream_t st);
+
 int device_sm_count();
 
 }  // namespace omni

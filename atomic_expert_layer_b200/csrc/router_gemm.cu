@@ -18,15 +18,14 @@
 // of the next.  Ragged edges (L,
 // N_r, N_c, d not multiples of the tile) read as zeros through TMA
 // out-of-bounds fill and are masked on store.
-#include <cuda.h>
-
 #include "omni_common.cuh"
 #include "omni_internal.h"
+#include "tcgen05.cuh"
 
 namespace omni {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 64, STAGES = 6;
+constexpr int BM = 128, BN = 128, BK = kSwK, STAGES = 6;
 constexpr int kTileBytesA = BM * BK * 2;     // 16 KB
 constexpr int kTileBytesB = BN * BK * 2;     // 16 KB
 constexpr uint32_t kTmemCols = 2 * BN;       // two fp32 accumulators
@@ -44,72 +43,7 @@ struct __align__(1024) GemmSmem {
     int abort;
 };
 
-// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
-// (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits
-// 17-22, M >> 4 at bits 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-
-// Shared-memory matrix descriptor for a K-major tile written by TMA with
-// 128-byte swizzle: rows of 128 bytes, 8-row core groups 1024 bytes apart
-// (stride byte offset), leading byte offset unused for this layout, version 1
-// (bit 46), layout SWIZZLE_128B (value 2 at bits 61-63).  Tile bases are
-// 1024-byte aligned, so the base offset field is 0.
-__device__ __forceinline__ uint64_t sw128_desc(const void *tile) {
-    const uint32_t addr = smem_u32(tile);
-    uint64_t d = 0;
-    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)1 << 16;                 // LBO (ignored), encoded 1
-    d |= (uint64_t)(1024 >> 4) << 32;       // SBO
-    d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
-    return d;
-}
-
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, int c0, int c1,
-                                            uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(smem_u32(dst)), "l"(tm), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
+constexpr uint32_t kIdesc = umma_idesc_bf16(BM, BN);
 
 __global__ void __launch_bounds__(kThreads, 1)
 router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
@@ -208,7 +142,7 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
                         // advance 16 bf16 = 32 bytes along K inside the swizzle atom
-                        umma_bf16(acc, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k),
+                        umma_bf16(acc, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), kIdesc,
                                   (kb > 0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit(&sm.empty[s]);
@@ -302,40 +236,6 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
                      ::"r"(tmem), "r"(kTmemCols));
     }
-}
-
-// ---------------------------------------------------------- tensor maps
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// rows x d bf16 matrix, box {BK, box_rows}, 128-byte swizzle, OOB reads zero
-bool make_map(CUtensorMap *tm, const uint16_t *ptr, int rows, int d, int box_rows) {
-    EncodeTiledFn enc = get_encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(ptr), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------- few tokens (L <= 4)
@@ -463,8 +363,8 @@ cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *W_r, const uin
                                int L, int d, int N_r, int N_c, float *s_r, float *s_c,
                                float *part_r, float *part_c, int *status, cudaStream_t st) {
     CUtensorMap tm_x, tm_wr, tm_wc;
-    if (!make_map(&tm_x, x, L, d, BM) || !make_map(&tm_wr, W_r, N_r, d, BN) ||
-        !make_map(&tm_wc, W_c, N_c, d, BN))
+    if (!make_sw128_map(&tm_x, x, L, d, BM) || !make_sw128_map(&tm_wr, W_r, N_r, d, BN) ||
+        !make_sw128_map(&tm_wc, W_c, N_c, d, BN))
         return cudaErrorInvalidValue;
     const int smem = (int)sizeof(GemmSmem) + 1024;   // slack for base alignment
     cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel,

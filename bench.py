@@ -399,6 +399,48 @@ def run_omni(args, cfg, world, rank, local):
         del g_dW, g_dV, g_dWr, g_dWc, g_dx, g_dy, ws_b
         torch.cuda.empty_cache()
 
+    # ---- the shared dense MLP beside the routed branch (gated form, hidden
+    # width F = mlp_hidden(d)) alone, and the whole layer y = routed(x) + MLP(x)
+    F = configs.mlp_hidden(d)
+    mw = inputs.make_mlp_weights(d, F, dev, seed=0)
+    ws_m = omni.shared_mlp_workspace(L, d, F, dev)
+
+    def mstep():
+        omni.omni_shared_mlp_fwd(t["x"], mw["W_g"], mw["W_u"], mw["W_d"], L, d, F, y,
+                                 omni.OMNI_Y_ACCUMULATE, ws_m)
+
+    def lstep():
+        step()
+        mstep()
+
+    res = {}
+    for name, fn in (("mlp", mstep), ("layer", lstep)):
+        for _ in range(3):
+            fn()
+        mev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            mev[i][0].record(stream)
+            fn()
+            mev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        res[name] = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in mev])), world, dev)
+    if omni.omni_get_device_status(ws_m) != 0:
+        raise RuntimeError("device status set in the shared MLP")
+    mlp_flops = 6.0 * L * d * F                      # x W_g^T, x W_u^T, h W_d^T
+    mlp_tflops = mlp_flops / (res["mlp"] * 1e-3) / 1e12
+    mlp = {"F": F, "ms_per_step": res["mlp"], "value": job_throughput(world, L, res["mlp"]),
+           "unit": "tokens/s", "flops": mlp_flops, "achieved_tflops": mlp_tflops,
+           "peak_tflops": measured_peaks()["bf16_tflops"],
+           "frac": mlp_tflops / measured_peaks()["bf16_tflops"],
+           "layer_ms_per_step": res["layer"],
+           "layer_value": job_throughput(world, L, res["layer"])}
+    del mw, ws_m
+
     # ---- end to end: host buffers, copies inside the timed region.  Every
     # step copies its token batch in from pinned host memory and its y out to
     # pinned host memory.  Steps are pipelined over three streams (copy-in of
@@ -501,6 +543,7 @@ def run_omni(args, cfg, world, rank, local):
         "ablation": ablation,
         "topk_compare": topk_cmp,
         "backward": bwd,
+        "shared_mlp": mlp,
         "clocks": clocks,
     }
     del t, ws, flush
@@ -520,6 +563,10 @@ def profile_stage(args, cfg):
     sc = omni.schedule(rt["idx"], rt["gate"], cfg.N, cfg.B)
     ws = omni.workspace(L, d, cfg.N_r, cfg.N_c, cfg.K, cfg.B, dev)
     y = torch.zeros((L, d), dtype=torch.float32, device=dev)
+    if args.profile_stage == "mlp":
+        F = configs.mlp_hidden(d)
+        mw = inputs.make_mlp_weights(d, F, dev, seed=0)
+        ws_m = omni.shared_mlp_workspace(L, d, F, dev)
     if args.profile_stage == "backward":
         f32 = dict(dtype=torch.float32, device=dev)
         g = dict(dx=torch.empty((L, d), **f32), dW=torch.zeros((cfg.N, d), **f32),
@@ -531,6 +578,9 @@ def profile_stage(args, cfg):
             omni.omni_routed_bwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r,
                                  cfg.N_c, cfg.K, rt["idx"], rt["gate"], dy, g["dx"], g["dW"],
                                  g["dV"], g["dW_r"], g["dW_c"], 0, ws)
+        elif args.profile_stage == "mlp":
+            omni.omni_shared_mlp_fwd(t["x"], mw["W_g"], mw["W_u"], mw["W_d"], L, d, F, y,
+                                     omni.OMNI_Y_ACCUMULATE, ws_m)
         elif args.profile_stage == "router":
             omni.omni_router_topk(t["x"], t["W_r"], t["W_c"], L, d, cfg.N_r, cfg.N_c, cfg.K,
                                   rt["p_r"], rt["p_c"], rt["idx"], rt["score"], rt["gate"], 0, ws)
@@ -695,7 +745,7 @@ def main():
                     help="workload name: " + ", ".join(c.name for c in configs.ALL))
     ap.add_argument("--impl", choices=["omni", "reference"], default="omni")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-stage", choices=["router", "schedule", "expert", "all", "backward"],
+    ap.add_argument("--profile-stage", choices=["router", "schedule", "expert", "all", "backward", "mlp"],
                     help="run only this stage W + K times (for profiler captures; no JSON)")
     ap.add_argument("--timeline", action="store_true",
                     help="print the in-stream kernel timeline of the last of K steps (no JSON)")

@@ -234,6 +234,31 @@ int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                     unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
 
 /*
+ * The shared dense MLP that the layer adds to the routed branch
+ * ("OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at Scale",
+ * rainbus review page, method paragraph, step 1: y = routed(x) + MLP(x);
+ * gist.science summary (German edition), section 2.1 "Kernkomponenten": a
+ * standard dense MLP branch, active for every input).  The pages give no
+ * form; this is the gated one with hidden width F:
+ *   h = SiLU(x W_g^T) * (x W_u^T)      [L, F], held in bf16 in ws
+ *   y = h W_d^T,  or  y += h W_d^T with OMNI_Y_ACCUMULATE
+ * so omni_routed_fwd followed by this call with OMNI_Y_ACCUMULATE gives the
+ * whole layer's output.
+ *   x [L, d] bf16;  W_g, W_u [F, d] bf16 (one row per hidden unit);
+ *   W_d [d, F] bf16 (one row per output feature);  y [L, d] fp32.
+ * Products run on the tensor cores (bf16 in, fp32 accumulate); each y element
+ * is written by one tile, so the result is the same on every run.
+ * ws: omni_shared_mlp_workspace_size(L, d, F) bytes, 256-byte aligned.  All
+ * arrays 16-byte aligned.  flags: 0 or OMNI_Y_ACCUMULATE.
+ * Limits: d % 64 == 0, F % 64 == 0, L * F, L * d and F * d < 2^31
+ * (OMNI_ERR_UNSUPPORTED beyond).
+ */
+size_t omni_shared_mlp_workspace_size(int L, int d, int F);
+int omni_shared_mlp_fwd(const omni_bf16 *x, const omni_bf16 *W_g, const omni_bf16 *W_u,
+                        const omni_bf16 *W_d, int L, int d, int F, float *y, unsigned flags,
+                        void *ws, size_t ws_bytes, omni_stream_t stream);
+
+/*
  * omni_grouped_expert_fwd without a workspace, for callers that cannot
  * allocate device memory when they run the layer (a serving runtime whose
  * memory is planned once at start-up, code where cudaMalloc is not allowed).

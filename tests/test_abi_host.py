@@ -58,6 +58,10 @@ def test_workspace_sizes(lib):
     assert omni.omni_workspace_size(4, 8, 4, 4, 17, 1) == 0         # K > N
     assert omni.omni_workspace_size(4, 8, 4, 4, 4, 2048) == 0       # B above the limit
     assert omni.omni_workspace_size(4, 8, 9000, 4, 4, 4) == 0       # axis above the limit
+    # shared MLP: the status header plus h [L, F] bf16
+    F = configs.mlp_hidden(h.d)
+    assert omni.omni_shared_mlp_workspace_size(h.L, h.d, F) == 256 + 2 * h.L * F
+    assert omni.omni_shared_mlp_workspace_size(0, h.d, F) == 0
 
 
 def _p(v):
@@ -111,6 +115,20 @@ def test_bad_arguments_rejected_on_host(lib):
                                fake, fake, fake, fake, fake, 0, fake, 256, None) == -2
     assert lib.omni_routed_bwd(fake, fake, fake, fake, fake, L, d, Nr, Nc, K, fake, fake, fake,
                                fake, fake, fake, fake, fake, 0, fake, 64, None) == -3
+    # shared MLP: null weight, unknown flag, d or F off the 64 grid, misaligned y, small workspace
+    mlp_ws = omni.omni_shared_mlp_workspace_size(L, d, 128)
+    assert lib.omni_shared_mlp_fwd(fake, None, fake, fake, L, d, 128, fake, 0, fake, mlp_ws,
+                                   None) == -1
+    assert lib.omni_shared_mlp_fwd(fake, fake, fake, fake, L, d, 128, fake, 4, fake, mlp_ws,
+                                   None) == -1
+    assert lib.omni_shared_mlp_fwd(fake, fake, fake, fake, L, 96, 128, fake, 0, fake, mlp_ws,
+                                   None) == -2
+    assert lib.omni_shared_mlp_fwd(fake, fake, fake, fake, L, d, 96, fake, 0, fake, mlp_ws,
+                                   None) == -2
+    assert lib.omni_shared_mlp_fwd(fake, fake, fake, fake, L, d, 128, _p((1 << 20) + 4), 0, fake,
+                                   mlp_ws, None) == -1
+    assert lib.omni_shared_mlp_fwd(fake, fake, fake, fake, L, d, 128, fake, 2, fake, mlp_ws - 1,
+                                   None) == -3
     # status query needs a workspace
     out = ctypes.c_int(7)
     assert lib.omni_get_device_status(None, 0, None, ctypes.byref(out)) == -1
