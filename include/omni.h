@@ -1,6 +1,7 @@
 /*
  * omni.h -- C ABI of the B200 (sm_100a) routed-branch forward of an OmniMoE
- * layer.  Library: atomic_expert_layer_b200/libomni.so.
+ * layer (with its backward, and the shared dense MLP the layer adds to it).
+ * Library: atomic_expert_layer_b200/libomni.so.
  *
  * Sources, cited by page title and section:
  *   [R] "OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at Scale",
@@ -23,7 +24,8 @@
  *   - All array arguments are DEVICE pointers to caller-owned, contiguous,
  *     row-major buffers.  The library never allocates or frees device memory;
  *     scratch comes from the caller's workspace `ws` of `ws_bytes` bytes, at
- *     least omni_workspace_size(...) for the same sizes, 256-byte aligned.
+ *     least omni_workspace_size(...) for the same sizes (or the size function
+ *     named at the call), 256-byte aligned.
  *     One workspace must not be used by two calls that overlap in time.
  *   - bf16 values are passed as their 16-bit patterns (omni_bf16).
  *   - W_r is stored as N_r rows of d (row i is the routing vector of grid row
