@@ -8,7 +8,7 @@
 //
 // One persistent launch computes both.  Tiles are 128 x 128 (n-tiles of W_r
 // first, then those of W_c), K step 64 (one 128-byte swizzle atom of bf16).
-// Warp roles: warp 0 issues TMA tile loads (no multicast) into a 6-stage
+// Warp roles: warp 0 issues TMA tile loads (each CTA its own) into a 6-stage
 // shared-memory ring; warp 1 issues tcgen05.mma kind::f16 (bf16 in, fp32
 // accumulate) into one of two 128-column TMEM accumulators; warps 2-9 drain
 // the other accumulator with tcgen05.ld (two warps per TMEM lane quarter,

@@ -12,7 +12,7 @@
 // with W_g, W_u stored as F rows of d and W_d as d rows of F (all K-major).
 //
 // One persistent tile GEMM, launched twice.  Tiles are 128 x 256 with a K
-// step of 64; warp 0 issues TMA loads (no multicast) into a 4-stage ring,
+// step of 64; warp 0 issues TMA loads (each CTA its own) into a 4-stage ring,
 // warp 1 issues tcgen05.mma kind::f16 into one of two 256-column TMEM
 // accumulators (all 512 columns), warps 2-9 drain the other one.
 //   up:   the B tile is 128 rows of W_g stacked on the same 128 rows of W_u,

@@ -41,7 +41,7 @@ __device__ __forceinline__ uint64_t sw128_desc(const void *tile) {
     return d;
 }
 
-// One box of a 2-D tensor map into shared memory (no multicast); completion
+// One box of a 2-D tensor map into this CTA's shared memory; completion
 // is counted on `bar` in bytes.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, int c0, int c1,
                                             uint64_t *bar) {
