@@ -1,0 +1,51 @@
+"""Host logic of bench.py (CPU only): the launch count it claims, the radix
+pass count, the clock-sample parsing and the traffic lookup that is only
+trusted while the profiled kernel source is unchanged."""
+import os
+
+import pytest
+
+import bench
+from atomic_expert_layer_b200 import configs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.parametrize("G,passes", [(1, 0), (2, 1), (256, 1), (257, 2), (13285, 2),
+                                      (65536, 2), (65537, 3)])
+def test_radix_passes(G, passes):
+    assert bench.radix_passes(G) == passes
+
+
+def test_launches_per_step_matches_the_profiled_step():
+    # the headline step in the committed launch list: GEMM, two axis kernels,
+    # merge, scan, two radix scatters, histogram scan, group pass, token pass
+    assert bench.launches_per_step(configs.HEADLINE) == 10
+    # decode batches skip the schedule: router (4) + the two expert passes
+    assert bench.launches_per_step(configs.sweep(16)) == 6
+    assert bench.launches_per_step(configs.sweep(1)) == 6
+
+
+def test_clock_summary_reads_reasons_and_load_median(tmp_path):
+    s = bench.ClockSampler(0)
+    s.path = str(tmp_path / "clocks.csv")
+    with open(s.path, "w") as f:
+        f.write("0, 1965, 1965, 120.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+        f.write("0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n")
+        f.write("0, 1700, 1965, 1000.0, 0x4, Not Active, Not Active, Not Active, Active\n")
+        f.write("garbage line\n")
+    out = s.summary()
+    assert out["samples"] == 3 and out["samples_under_load"] == 2
+    assert out["sm_mhz"] == pytest.approx(1750.0)           # median of the loaded samples
+    assert out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"]
+    assert not os.path.exists(s.path)                         # the sample file is removed
+
+
+def test_traffic_only_for_the_profiled_source(tmp_path):
+    src = os.path.join(ROOT, "atomic_expert_layer_b200", "csrc", "expert.cu")
+    got = bench.traffic_from_profile(src)
+    assert got is not None and got > 1e9                      # the committed headline capture
+    other = tmp_path / "expert.cu"
+    other.write_bytes(open(src, "rb").read() + b"\n// changed\n")
+    assert bench.traffic_from_profile(str(other)) is None
