@@ -100,12 +100,29 @@ def test_router_matches_library_log_softmax():
     (64, 64, 16, None, 0), (8, 64, 16, None, 1), (64, 8, 33, None, 2), (1, 50, 7, None, 3),
     (50, 1, 7, None, 4), (5, 7, 35, None, 5), (16, 16, 64, 2.0 ** -4, 6), (40, 24, 20, 0.25, 7),
     (12, 12, 1, None, 8), (3, 3, 9, 1.0, 9),
+    # both axes at least K, at the K of the full-size layers (64 and 128), so
+    # the pruned (a+1)(b+1) <= K block is the whole argument, as on the GPU
+    (160, 160, 64, None, 10), (200, 150, 128, None, 11), (130, 130, 128, 2.0 ** -4, 12),
+    (128, 256, 64, 0.25, 13), (300, 260, 128, 2.0 ** -3, 14),
 ])
 def test_topk_matches_bruteforce(N_r, N_c, K, quantum, seed):
     L = 24
     p_r = inputs.random_logprobs(L, N_r, seed, quantum)
     p_c = inputs.random_logprobs(L, N_c, seed + 100, quantum)
     idx, score, gate = oracle.topk_from_logprobs(p_r, p_c, K)
+    bidx, bsc = brute_force_topk(p_r, p_c, K)
+    np.testing.assert_array_equal(idx, bidx)
+    np.testing.assert_array_equal(score, bsc)
+
+
+@pytest.mark.parametrize("K,quantum", [(64, None), (128, 2.0 ** -4)])
+def test_topk_matches_bruteforce_headline_grid(K, quantum):
+    # the 1304 x 1304 grid of the headline layer (1.7M cells per token),
+    # brute force over every cell for a few tokens
+    L, n = 3, 1304
+    p_r = inputs.random_logprobs(L, n, 21 + K, quantum)
+    p_c = inputs.random_logprobs(L, n, 22 + K, quantum)
+    idx, score, _ = oracle.topk_from_logprobs(p_r, p_c, K)
     bidx, bsc = brute_force_topk(p_r, p_c, K)
     np.testing.assert_array_equal(idx, bidx)
     np.testing.assert_array_equal(score, bsc)
