@@ -12,10 +12,12 @@ from __future__ import annotations
 import torch
 
 from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_TOPK_BLOCKWISE,  # noqa: F401
-                   OMNI_Y_ACCUMULATE,
+                   OMNI_Y_ACCUMULATE, OMNI_EXPERT_DENSE, OMNI_EXPERT_SPARSE,
+                   omni_workspace_size_flags, omni_expert_workspace_size_flags,
                    OmniError, load,
                    expert_workspace, omni_expert_workspace_size, omni_get_device_status,
-                   omni_grouped_expert_fwd, omni_grouped_expert_fwd_noalloc, omni_routed_bwd,
+                   omni_grouped_expert_fwd, omni_grouped_expert_fwd_noalloc,
+                   omni_noalloc_get_device_status, omni_routed_bwd,
                    omni_routed_fwd,
                    omni_router_topk,
                    omni_router_workspace_size, omni_schedule, omni_schedule_workspace_size,
@@ -25,8 +27,11 @@ from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_TOPK_BLOCKWIS
 
 __all__ = [
     "load", "OmniError", "OMNI_ROUTER_LOGPROBS_IN", "OMNI_Y_ACCUMULATE", "OMNI_TOKEN_ORDER", "OMNI_TOPK_BLOCKWISE",
+    "OMNI_EXPERT_DENSE", "OMNI_EXPERT_SPARSE", "omni_workspace_size_flags",
+    "omni_expert_workspace_size_flags",
     "omni_workspace_size", "omni_router_topk", "omni_schedule", "omni_grouped_expert_fwd",
     "omni_routed_fwd", "omni_get_device_status", "workspace", "omni_grouped_expert_fwd_noalloc",
+    "omni_noalloc_get_device_status",
     "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd", "omni_routed_bwd", "routed_bwd",
     "omni_shared_mlp_workspace_size", "omni_shared_mlp_fwd", "shared_mlp_fwd", "layer_fwd",
 ]
@@ -77,29 +82,37 @@ def schedule(idx, gate, N, B, ws=None, stream=None):
     return out
 
 
-def grouped_expert_fwd(x, W, V, sched, K, B, y=None, accumulate=False, ws=None, stream=None):
+_EXPERT_MODE = {"auto": 0, "dense": OMNI_EXPERT_DENSE, "sparse": OMNI_EXPERT_SPARSE}
+
+
+def grouped_expert_fwd(x, W, V, sched, K, B, y=None, accumulate=False, ws=None, stream=None,
+                       expert_mode="auto"):
+    """expert_mode: "auto" (the library's size rule), "dense" (always try the
+    tensor-core tiles for dense experts) or "sparse" (task by task only)."""
     L, d = x.shape
     N = W.shape[0]
+    mode = _EXPERT_MODE[expert_mode]
     y = torch.empty((L, d), dtype=torch.float32, device=x.device) if y is None else y
-    ws = expert_workspace(L, d, K, N, B, x.device) if ws is None else ws
+    ws = expert_workspace(L, d, K, N, B, x.device, mode) if ws is None else ws
     omni_grouped_expert_fwd(x, W, V, L, d, K, N, B, sched["task_token"], sched["task_expert"],
                             sched["task_gate"], sched["group_offsets"], sched["active_groups"],
-                            sched["num_active"], y, OMNI_Y_ACCUMULATE if accumulate else 0, ws,
-                            stream)
+                            sched["num_active"], y, (OMNI_Y_ACCUMULATE if accumulate else 0) | mode,
+                            ws, stream)
     return y
 
 
 def routed_fwd(x, W, V, W_r, W_c, K, B, y=None, ws=None, want_routing=False, accumulate=False,
-               token_order=False, stream=None):
+               token_order=False, stream=None, expert_mode="auto"):
     L, d = x.shape
     N_r, N_c = W_r.shape[0], W_c.shape[0]
+    mode = _EXPERT_MODE[expert_mode]
+    flags = (OMNI_Y_ACCUMULATE if accumulate else 0) | (OMNI_TOKEN_ORDER if token_order else 0) | mode
     y = torch.empty((L, d), dtype=torch.float32, device=x.device) if y is None else y
-    ws = workspace(L, d, N_r, N_c, K, B, x.device) if ws is None else ws
+    ws = workspace(L, d, N_r, N_c, K, B, x.device, flags) if ws is None else ws
     idx = gate = None
     if want_routing:
         idx = torch.empty((L, K), dtype=torch.int32, device=x.device)
         gate = torch.empty((L, K), dtype=torch.float32, device=x.device)
-    flags = (OMNI_Y_ACCUMULATE if accumulate else 0) | (OMNI_TOKEN_ORDER if token_order else 0)
     omni_routed_fwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, B, y, idx, gate, flags, ws, stream)
     return (y, idx, gate) if want_routing else y
 

@@ -20,6 +20,8 @@ OMNI_ROUTER_LOGPROBS_IN = 1
 OMNI_Y_ACCUMULATE = 2
 OMNI_TOKEN_ORDER = 4
 OMNI_TOPK_BLOCKWISE = 8
+OMNI_EXPERT_DENSE = 16
+OMNI_EXPERT_SPARSE = 32
 
 STATUS = {0: "OMNI_OK", -1: "OMNI_ERR_INVALID_ARG", -2: "OMNI_ERR_UNSUPPORTED",
           -3: "OMNI_ERR_WORKSPACE", -4: "OMNI_ERR_CUDA", -5: "OMNI_ERR_DEVICE"}
@@ -31,9 +33,11 @@ SIGNATURES = {
     "omni_status_string": ([_I], ctypes.c_char_p),
     "omni_device_status_string": ([_I], ctypes.c_char_p),
     "omni_workspace_size": ([_I, _I, _I, _I, _I, _I], _Z),
+    "omni_workspace_size_flags": ([_I, _I, _I, _I, _I, _I, _U], _Z),
     "omni_router_workspace_size": ([_I, _I, _I, _I], _Z),
     "omni_schedule_workspace_size": ([_I, _I, _I, _I], _Z),
     "omni_expert_workspace_size": ([_I, _I, _I, _I, _I], _Z),
+    "omni_expert_workspace_size_flags": ([_I, _I, _I, _I, _I, _U], _Z),
     "omni_router_topk": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _U, _P, _Z, _P], _I),
     "omni_schedule": ([_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "omni_grouped_expert_fwd": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
@@ -48,6 +52,7 @@ SIGNATURES = {
     "omni_selftest_wait_timeout": ([_P, _Z, _I, _P], _I),
     "omni_grouped_expert_fwd_noalloc": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                                          _P, _U, _P], _I),
+    "omni_noalloc_get_device_status": ([_P, ctypes.POINTER(ctypes.c_int)], _I),
 }
 
 _lib = None
@@ -105,6 +110,10 @@ def omni_workspace_size(L, d, N_r, N_c, K, B) -> int:
     return int(load().omni_workspace_size(L, d, N_r, N_c, K, B))
 
 
+def omni_workspace_size_flags(L, d, N_r, N_c, K, B, flags) -> int:
+    return int(load().omni_workspace_size_flags(L, d, N_r, N_c, K, B, flags))
+
+
 def omni_router_workspace_size(L, N_r, N_c, K) -> int:
     return int(load().omni_router_workspace_size(L, N_r, N_c, K))
 
@@ -117,15 +126,20 @@ def omni_expert_workspace_size(L, d, K, N, B) -> int:
     return int(load().omni_expert_workspace_size(L, d, K, N, B))
 
 
+def omni_expert_workspace_size_flags(L, d, K, N, B, flags) -> int:
+    return int(load().omni_expert_workspace_size_flags(L, d, K, N, B, flags))
+
+
 def _alloc(n: int, device) -> torch.Tensor:
     if n == 0:
         raise ValueError("invalid sizes")
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def workspace(L, d, N_r, N_c, K, B, device="cuda") -> torch.Tensor:
-    """Workspace for omni_routed_fwd (and any of the stage calls) at these sizes."""
-    return _alloc(omni_workspace_size(L, d, N_r, N_c, K, B), device)
+def workspace(L, d, N_r, N_c, K, B, device="cuda", flags=0) -> torch.Tensor:
+    """Workspace for omni_routed_fwd (and any of the stage calls) at these
+    sizes, for calls made with `flags`."""
+    return _alloc(omni_workspace_size_flags(L, d, N_r, N_c, K, B, flags), device)
 
 
 def router_workspace(L, N_r, N_c, K, device="cuda") -> torch.Tensor:
@@ -136,8 +150,8 @@ def schedule_workspace(L, K, N, B, device="cuda") -> torch.Tensor:
     return _alloc(omni_schedule_workspace_size(L, K, N, B), device)
 
 
-def expert_workspace(L, d, K, N, B, device="cuda") -> torch.Tensor:
-    return _alloc(omni_expert_workspace_size(L, d, K, N, B), device)
+def expert_workspace(L, d, K, N, B, device="cuda", flags=0) -> torch.Tensor:
+    return _alloc(omni_expert_workspace_size_flags(L, d, K, N, B, flags), device)
 
 
 def omni_router_topk(x, W_r, W_c, L, d, N_r, N_c, K, p_r, p_c, idx, score, gate, flags, ws,
@@ -220,3 +234,13 @@ def omni_grouped_expert_fwd_noalloc(x, W, V, L, d, K, N, B, task_token, task_exp
         _ptr(task_gate), _ptr(group_offsets), _ptr(active_groups), _ptr(num_active), _ptr(y),
         flags, _stream(stream))
     _check("omni_grouped_expert_fwd_noalloc", rc)
+
+
+def omni_noalloc_get_device_status(stream=None) -> int:
+    """Status word of the no-workspace call's array on the current device
+    (synchronises the stream, then clears the word)."""
+    out = ctypes.c_int(0)
+    rc = load().omni_noalloc_get_device_status(_stream(stream), ctypes.byref(out))
+    if rc not in (0, -5):
+        raise OmniError("omni_noalloc_get_device_status", rc)
+    return int(out.value)

@@ -43,10 +43,18 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
              "-I", os.path.join(ROOT, "include"), *ARCH] + list(extra or [])
     if verbose:
         flags += ["-Xptxas", "-v"]
-    for src in sorted(glob.glob(os.path.join(CSRC, "*.cu"))):
+    srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+    def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         cmd = [nvcc(), *flags, "-c", src, "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, subprocess.run(cmd, capture_output=True, text=True)
+
+    # one nvcc per source file, several at a time
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as pool:
+        results = list(pool.map(compile_one, srcs))
+    for src, obj, r in results:
         if verbose or r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode != 0:

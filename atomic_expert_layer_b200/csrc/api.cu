@@ -3,6 +3,7 @@
 // no host synchronisation except in omni_get_device_status.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cstring>
 
@@ -23,16 +24,18 @@ bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 }  // namespace
 
 int device_sm_count() {
-    static int cached[64] = {0};
+    // filled once per device; several host threads may race to fill an entry,
+    // and all of them store the same value
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 bool make_sizes(int L, int d, int N_r, int N_c, int K, int B, Sizes *sz) {
@@ -52,6 +55,34 @@ bool make_sizes(int L, int d, int N_r, int N_c, int K, int B, Sizes *sz) {
     return true;
 }
 
+void set_dense(Sizes *sz, unsigned flags) {
+    sz->dense = false;
+    sz->dense_thr = 0;
+    sz->dense_cap = 0;
+    if (flags & OMNI_EXPERT_SPARSE) return;
+    // By default the tensor-core path is considered only for large expert
+    // stages (tasks x width >= 2^31): its fixed cost (six more launches) is
+    // then a small share of the stage, and below that size an expert rarely
+    // reaches the threshold.
+    const bool want = (flags & OMNI_EXPERT_DENSE) || sz->M * (int64_t)sz->d >= ((int64_t)1 << 31);
+    if (!want) return;
+    // An expert joins the tile GEMMs when >= thr tasks use it: its column
+    // costs 4 L d tensor-core flops, against a gathered W and V row per task
+    // on the CUDA-core path (break-even near L / 96 tasks at d = 2048).
+    int thr = (sz->L + 95) / 96;
+    if (thr < 32) thr = 32;
+    int64_t most = sz->M / thr;                  // experts that can reach thr
+    if (most > sz->N) most = sz->N;
+    if (most == 0) return;
+    int64_t cap = (most + 255) / 256 * 256;
+    if (cap > 4096) cap = 4096;
+    // G (fp32) and P (bf16) take 6 bytes per token and column: at most 768 MB
+    while (cap > 256 && 6 * (int64_t)sz->L * cap > ((int64_t)768 << 20)) cap -= 256;
+    sz->dense = true;
+    sz->dense_thr = thr;
+    sz->dense_cap = (int)cap;
+}
+
 WsLayout make_layout(const Sizes &sz, unsigned regions) {
     WsLayout w;
     std::memset(&w, 0, sizeof w);
@@ -67,6 +98,12 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.hist = take(4 * 256 * (size_t)sz.ntiles * (size_t)sz.passes);   // one per radix pass
     }
     if (regions & kRegExpert) w.tok_count = take(4 * L);
+    const bool dense = (regions & kRegDense) && sz.dense;
+    if (dense) {
+        w.dz_bits = take(4 * (size_t)((sz.N + 31) / 32));
+        w.dz_ghot = take(4 * (G + 1));
+        w.dz_ccount = take(8);
+    }
     w.zero_end = o;
     if (regions & kRegRouter) {
         w.s_r = take(4 * L * sz.N_r);
@@ -95,6 +132,18 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.n_dist = take(4);
     }
     if (regions & kRegExpert) w.tok_slots = take(8 * M);
+    if (dense) {
+        const size_t cap = (size_t)sz.dense_cap, d = (size_t)sz.d;
+        w.d_ehot = take(4);
+        w.d_list = take(4 * cap);
+        w.d_whot = take(2 * cap * d);
+        w.d_vt = take(2 * d * cap);
+        w.d_G = take(4 * L * cap);
+        w.d_P = take(2 * L * cap);
+        w.d_ctok = take(4 * M);
+        w.d_cexp = take(4 * M);
+        w.d_cgate = take(4 * M);
+    }
     w.total = o;
     return w;
 }
@@ -183,6 +232,27 @@ int router_topk_impl(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c
     return cuda_rc(e);
 }
 
+// The expert stage on a sorted schedule.  With the tensor-core path, the
+// dense experts' tasks go through the tile GEMMs (which add into y after
+// the CUDA-core passes wrote it) and the rest through the CUDA-core passes.
+cudaError_t expert_stage(const uint16_t *x, const uint16_t *W, const uint16_t *V, const Sizes &sz,
+                         const int32_t *tt, const int32_t *te, const float *tg,
+                         const int32_t *goff, const int32_t *gact, const int32_t *nact, float *y,
+                         bool accumulate, void *ws, const WsLayout &lay, cudaStream_t st,
+                         bool check_offsets) {
+    if (!sz.dense)
+        return launch_grouped_expert(x, W, V, sz, tt, te, tg, y, accumulate, ws, lay, st,
+                                     check_offsets ? goff : nullptr);
+    int *status = ws_at<int>(ws, lay.hdr);
+    const DenseWs o = dense_ws_of(sz, ws, lay);
+    cudaError_t e = launch_dense_prepare(W, V, sz, tt, te, tg, goff, gact, nact, o, status, st);
+    if (e != cudaSuccess) return e;
+    e = launch_grouped_expert(x, W, V, sz, o.c_tok, o.c_exp, o.c_gate, y, accumulate, ws, lay, st,
+                              nullptr, o.ccount);
+    if (e != cudaSuccess) return e;
+    return launch_dense_gemms(x, sz, o, y, status, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -211,10 +281,16 @@ const char *omni_device_status_string(int s) {
     }
 }
 
-size_t omni_workspace_size(int L, int d, int N_r, int N_c, int K, int B) {
+size_t omni_workspace_size_flags(int L, int d, int N_r, int N_c, int K, int B, unsigned flags) {
     Sizes sz;
     if (check_common(L, d, N_r, N_c, K, B, true, &sz) != OMNI_OK) return 0;
+    if (flags & OMNI_TOKEN_ORDER) return make_layout(sz, kRegRouter | kRegExpert).total;
+    set_dense(&sz, flags);
     return make_layout(sz, kRegAll).total;
+}
+
+size_t omni_workspace_size(int L, int d, int N_r, int N_c, int K, int B) {
+    return omni_workspace_size_flags(L, d, N_r, N_c, K, B, 0u);
 }
 
 size_t omni_router_workspace_size(int L, int N_r, int N_c, int K) {
@@ -229,10 +305,15 @@ size_t omni_schedule_workspace_size(int L, int K, int N, int B) {
     return make_layout(sz, kRegSched).total;
 }
 
-size_t omni_expert_workspace_size(int L, int d, int K, int N, int B) {
+size_t omni_expert_workspace_size_flags(int L, int d, int K, int N, int B, unsigned flags) {
     Sizes sz;
     if (N <= 0 || check_common(L, d, N, 1, K, B, false, &sz) != OMNI_OK) return 0;
-    return make_layout(sz, kRegExpert).total;
+    set_dense(&sz, flags);
+    return make_layout(sz, kRegExpert | kRegDense).total;
+}
+
+size_t omni_expert_workspace_size(int L, int d, int K, int N, int B) {
+    return omni_expert_workspace_size_flags(L, d, K, N, B, 0u);
 }
 
 int omni_router_topk(const omni_bf16 *x, const omni_bf16 *W_r, const omni_bf16 *W_c, int L,
@@ -302,12 +383,14 @@ int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_b
     if (d % 256 != 0 || d > OMNI_MAX_D) return OMNI_ERR_UNSUPPORTED;
     if (!aligned16(x) || !aligned16(W) || !aligned16(V) || !aligned16(y))
         return OMNI_ERR_INVALID_ARG;
+    set_dense(&sz, flags);
     WsLayout lay;
-    if ((rc = check_ws(sz, kRegExpert, ws, ws_bytes, &lay))) return rc;
+    if ((rc = check_ws(sz, kRegExpert | kRegDense, ws, ws_bytes, &lay))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = reset_workspace(ws, lay, st))) return rc;
-    return cuda_rc(launch_grouped_expert(x, W, V, sz, task_token, task_expert, task_gate, y,
-                                         (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st));
+    return cuda_rc(expert_stage(x, W, V, sz, task_token, task_expert, task_gate, group_offsets,
+                                active_groups, num_active, y, (flags & OMNI_Y_ACCUMULATE) != 0,
+                                ws, lay, st, /*check_offsets=*/true));
 }
 
 int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
@@ -323,13 +406,16 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     if (!aligned16(x) || !aligned16(W) || !aligned16(V) || !aligned16(W_r) || !aligned16(W_c) ||
         !aligned16(y))
         return OMNI_ERR_INVALID_ARG;
+    const bool token_order = (flags & OMNI_TOKEN_ORDER) || L <= kTokenOrderMaxL;
+    if (!token_order) set_dense(&sz, flags);
     WsLayout lay;
-    if ((rc = check_ws(sz, kRegAll, ws, ws_bytes, &lay))) return rc;
+    if ((rc = check_ws(sz, token_order ? (unsigned)(kRegRouter | kRegExpert) : (unsigned)kRegAll,
+                       ws, ws_bytes, &lay)))
+        return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = reset_workspace(ws, lay, st))) return rc;
     int32_t *idx = ws_at<int32_t>(ws, lay.idx);
     float *score = ws_at<float>(ws, lay.score), *gate = ws_at<float>(ws, lay.gate);
-    const bool token_order = (flags & OMNI_TOKEN_ORDER) || L <= kTokenOrderMaxL;
     // scheduled path: the merge kernel also runs the schedule's per-token step;
     // nothing here reads the distinct-expert count, so it is not kept
     SchedPrep prep = sched_prep_of(sz, ws, lay);
@@ -352,8 +438,9 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
         if ((rc = cuda_rc(launch_schedule(idx, gate, sz, tt, te, tg, goff, gcnt, gact, nact,
                                           ndist, ws, lay, st, /*prepared=*/true))))
             return rc;
-        if ((rc = cuda_rc(launch_grouped_expert(x, W, V, sz, tt, te, tg, y,
-                                                (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st))))
+        if ((rc = cuda_rc(expert_stage(x, W, V, sz, tt, te, tg, goff, gact, nact, y,
+                                       (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st,
+                                       /*check_offsets=*/false))))
             return rc;
     }
     if (idx_out &&

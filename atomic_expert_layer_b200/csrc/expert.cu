@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(32 * GateCfg<VPL>::kWarps)
 group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W, int L, int N,
                   int K, int M, int per_warp, const int32_t *__restrict__ task_token,
                   const int32_t *__restrict__ task_expert, const float *__restrict__ task_gate,
-                  int *__restrict__ tok_count, int2 *__restrict__ tok_slots, int *status) {
+                  int *__restrict__ tok_count, int2 *__restrict__ tok_slots, int *status,
+                  const int32_t *__restrict__ group_off, int B, const int32_t *__restrict__ dyn_M) {
     using Cfg = GateCfg<VPL>;
     constexpr int D = 256 * VPL;
     constexpr int S = Cfg::kStages;
@@ -129,6 +130,14 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
     uint8_t *xring = wring + S * RB;
     grid_dependency_wait();
     grid_dependents_launch();
+    if (dyn_M) {
+        // the compacted task list of the tensor-core path: its length is on
+        // the device; spread it over every warp of the grid
+        M = *dyn_M;
+        const int64_t warps = (int64_t)gridDim.x * Cfg::kWarps;
+        per_warp = (int)((M + warps - 1) / warps);
+        if (per_warp < 1) per_warp = 1;
+    }
 
     const int64_t gw = (int64_t)blockIdx.x * Cfg::kWarps + warp;
     const int64_t a0 = gw * per_warp;
@@ -150,6 +159,11 @@ group_gate_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
                 set_status(status, OMNI_DEV_BAD_SCHEDULE);
                 e = e < 0 || e >= N ? 0 : e;
                 t = t < 0 || t >= L ? 0 : t;
+            } else if (group_off) {
+                // the task must lie in its group's range of the sorted order
+                const int q = e / B;
+                const int64_t m = a0 + i;
+                if (m < group_off[q] || m >= group_off[q + 1]) set_status(status, OMNI_DEV_BAD_SCHEDULE);
             }
             slot = atomicAdd(&tok_count[t], 1);
         }
@@ -483,7 +497,7 @@ template <int VPL>
 cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, const Sizes &sz,
                        const int32_t *tt, const int32_t *te, const float *tg, float *y,
                        bool accumulate, int *tok_count, int2 *tok_slots, int *status,
-                       cudaStream_t st) {
+                       cudaStream_t st, const int32_t *group_off, const int32_t *dyn_M) {
     using G = GateCfg<VPL>;
     using C = CombineCfg<VPL>;
     cudaError_t e = cudaFuncSetAttribute(group_gate_kernel<VPL>,
@@ -507,7 +521,7 @@ cudaError_t launch_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V, 
         const int grid = (int)((needed + G::kWarps - 1) / G::kWarps);
         e = launch(group_gate_kernel<VPL>, dim3(grid), dim3(32 * G::kWarps), G::kSmem, st, x, W,
                    sz.L, (int)sz.N, sz.K, (int)sz.M, (int)per_warp, tt, te, tg, tok_count,
-                   tok_slots, status);
+                   tok_slots, status, group_off, sz.B, dyn_M);
         if (e != cudaSuccess) return e;
     }
     if (sz.L <= 4 * sms) {
@@ -536,14 +550,15 @@ cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const ui
                                   const Sizes &sz, const int32_t *task_token,
                                   const int32_t *task_expert, const float *task_gate,
                                   float *y, bool accumulate, void *ws, const WsLayout &lay,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, const int32_t *group_offsets,
+                                  const int32_t *dyn_M) {
     int *status = ws_at<int>(ws, lay.hdr);
     int *tok_count = ws_at<int>(ws, lay.tok_count);
     int2 *tok_slots = ws_at<int2>(ws, lay.tok_slots);
     switch (sz.d / 256) {
 #define OMNI_CASE(n) \
         case n: return launch_vpl<n>(x, W, V, sz, task_token, task_expert, task_gate, y, accumulate, \
-                                     tok_count, tok_slots, status, st);
+                                     tok_count, tok_slots, status, st, group_offsets, dyn_M);
         OMNI_CASE(1) OMNI_CASE(2) OMNI_CASE(3) OMNI_CASE(4)
         OMNI_CASE(5) OMNI_CASE(6) OMNI_CASE(7) OMNI_CASE(8)
 #undef OMNI_CASE

@@ -10,9 +10,13 @@
 // that loads it (about 2 MB, held until the process exits).
 //
 // Host code must not use the array's name as a device address: in host code
-// it names a host-side stand-in.  The device address is looked up once per
-// device with cudaGetSymbolAddress, with that device current, on the first
-// call made on it.
+// it names a host-side stand-in.  The device address is looked up with
+// cudaGetSymbolAddress, with the device current, on the first call made in
+// each CUDA context, and cached under that context's unique id: after a
+// cudaDeviceReset, or in a driver-API context other than the device's primary
+// one, the library image is loaded again at another address, and the new
+// context's id forces a fresh lookup.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -35,23 +39,63 @@ constexpr size_t kNoAllocBytes = kOffSlots + 8 * (size_t)kNoAllocMaxM;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices] = {nullptr};
+struct ScratchEntry {
+    unsigned long long ctx_id;   // unique id of the context the address belongs to
+    void *addr;                  // nullptr: nothing cached
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
 
-// Device address of the scratch array on the current device (set up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context; false when no context
+// is current yet or the driver lacks the query.
+bool current_context_id(unsigned long long *id) {
+    static const CtxGetCurrentFn get_current = []() -> CtxGetCurrentFn {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<CtxGetCurrentFn>(p);
+    }();
+    static const CtxGetIdFn get_id = []() -> CtxGetIdFn {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<CtxGetIdFn>(p);
+    }();
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current context.
 cudaError_t scratch_address(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    unsigned long long id = 0;
+    bool have_id = current_context_id(&id);
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
+    ScratchEntry &c = g_scratch[dev];
+    if (have_id && c.addr && c.ctx_id == id) {
+        *out = c.addr;
+        return cudaSuccess;
     }
-    *out = g_scratch_addr[dev];
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    // the lookup makes the device's primary context current if none was
+    if (!have_id) have_id = current_context_id(&id);
+    c.ctx_id = have_id ? id : 0;
+    c.addr = have_id ? p : nullptr;           // without an id nothing is cached
+    *out = p;
     return cudaSuccess;
 }
 
@@ -96,4 +140,18 @@ extern "C" int omni_grouped_expert_fwd_noalloc(
                                                 y, (flags & OMNI_Y_ACCUMULATE) != 0, scratch, lay,
                                                 st);
     return e == cudaSuccess ? OMNI_OK : OMNI_ERR_CUDA;
+}
+
+extern "C" int omni_noalloc_get_device_status(omni_stream_t stream, int *status_out) {
+    if (!status_out) return OMNI_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    if (scratch_address(&scratch) != cudaSuccess) return OMNI_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int host = 0;
+    if (cudaMemcpyAsync(&host, scratch, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return OMNI_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return OMNI_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, sizeof(int), st) != cudaSuccess) return OMNI_ERR_CUDA;
+    *status_out = host;
+    return host == 0 ? OMNI_OK : OMNI_ERR_DEVICE;
 }

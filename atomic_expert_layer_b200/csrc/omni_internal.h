@@ -17,6 +17,10 @@ struct Sizes {
     int C;               // merge candidates: cells (a, b) with (a+1)(b+1) <= K
     int64_t ntiles;      // radix tiles
     int qbits, passes;   // bits of the largest group id G - 1; radix passes of <= 8 bits
+    // tensor-core path of the expert stage (expert_dense.cu)
+    bool dense;          // laid out and run for this call
+    int dense_thr;       // tasks that make an expert dense
+    int dense_cap;       // dense columns at most (a multiple of 256)
 };
 
 struct WsLayout {
@@ -24,6 +28,9 @@ struct WsLayout {
     size_t a_tok, a_exp, a_gate, b_tok, b_exp, b_gate, t_tok, t_exp, t_gate;
     size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, tok_count, tok_slots;
     size_t z_cnt, z_ndist;   // schedule counters (workspace copies)
+    // tensor-core expert path: zeroed per call (dz_*), then the rest
+    size_t dz_bits, dz_ghot, dz_ccount;
+    size_t d_ehot, d_list, d_whot, d_vt, d_G, d_P, d_ctok, d_cexp, d_cgate;
     size_t zero_end;         // [0, zero_end) must be zero when a call starts
     size_t total;
 };
@@ -38,10 +45,15 @@ enum WsRegion : unsigned {
     kRegSched = 2u,       // sort buffers, expert bitmap, radix histograms
     kRegSchedOut = 4u,    // sorted tasks and group arrays (routed forward only)
     kRegExpert = 8u,      // per-token slots of (expert, p) between the two expert kernels
-    kRegAll = 15u
+    kRegDense = 16u,      // tensor-core expert path (only when Sizes::dense)
+    kRegAll = 31u
 };
 
 bool make_sizes(int L, int d, int N_r, int N_c, int K, int B, Sizes *sz);
+// Decides whether the tensor-core expert path runs for these sizes and flags
+// (OMNI_EXPERT_DENSE / OMNI_EXPERT_SPARSE force it on / off) and sets its
+// threshold and column cap.
+void set_dense(Sizes *sz, unsigned flags);
 WsLayout make_layout(const Sizes &sz, unsigned regions);
 int merge_candidates(int K, int Kr, int Kc);
 
@@ -103,11 +115,43 @@ SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay);
 // ---- grouped expert stage (expects the per-token slot counters zeroed).
 // task_token == nullptr: the tasks are in token order, task m belongs to
 // token m / K (task_expert / task_gate are then the router's idx / gate).
+// group_offsets (nullable): each task is checked to lie in its group's range.
+// dyn_M (nullable): the number of tasks is read from the device (the
+// compacted list of the tensor-core path), M is then an upper bound.
 cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const uint16_t *V,
                                   const Sizes &sz, const int32_t *task_token,
                                   const int32_t *task_expert, const float *task_gate,
                                   float *y, bool accumulate, void *ws, const WsLayout &lay,
-                                  cudaStream_t st);
+                                  cudaStream_t st, const int32_t *group_offsets = nullptr,
+                                  const int32_t *dyn_M = nullptr);
+
+// ---- tensor-core expert path (expert_dense.cu); expects the dz_* regions
+// zeroed.  prepare: dense experts per active group, their columns, W_D and
+// V_D^T, G (gates of their tasks) and the compacted list of the other tasks;
+// gemms: P = G . SiLU(x W_D^T), then y += P V_D.
+struct DenseWs {
+    uint32_t *bits;          // [ceil(N / 32)] dense-expert marks
+    int32_t *ghot;           // [G + 1] dense experts per group, then their first column
+    int32_t *ehot;           // [1] dense experts found (before the cap)
+    int32_t *ccount;         // [2] compacted tasks; tasks covered by the active groups
+    int32_t *list;           // [cap] dense expert ids by column
+    uint16_t *whot, *vt;     // [cap, d], [d, cap] bf16
+    float *G;                // [L, cap]
+    uint16_t *P;             // [L, cap] bf16
+    int32_t *c_tok, *c_exp;  // [M] compacted tasks
+    float *c_gate;
+    int cap, thr;
+};
+DenseWs dense_ws_of(const Sizes &sz, void *ws, const WsLayout &lay);
+cudaError_t launch_dense_prepare(const uint16_t *W, const uint16_t *V, const Sizes &sz,
+                                 const int32_t *task_token, const int32_t *task_expert,
+                                 const float *task_gate, const int32_t *group_offsets,
+                                 const int32_t *active_groups, const int32_t *num_active,
+                                 const DenseWs &o, int *status, cudaStream_t st);
+cudaError_t launch_dense_gemms(const uint16_t *x, const Sizes &sz, const DenseWs &o, float *y,
+                               int *status, cudaStream_t st);
+// exclusive scan of n ints in place (one CTA); the total goes to *total
+cudaError_t launch_exclusive_scan(int32_t *a, int64_t n, int32_t *total, cudaStream_t st);
 
 // ---- backward of the routed branch (selection fixed)
 cudaError_t launch_routed_bwd(const uint16_t *x, const uint16_t *W, const uint16_t *V,

@@ -294,14 +294,15 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(
 }
 
 // --------------------------------------------------- 3. radix passes
-// Exclusive scan of n ints in place, one CTA of 1024 threads.
+// Exclusive scan of n ints in place, one CTA of 1024 threads; with `tail`,
+// the total is written there.
 __global__ void __launch_bounds__(1024) exclusive_scan_kernel(int32_t *__restrict__ a,
-                                                             int64_t n) {
+                                                             int64_t n, int32_t *tail) {
     __shared__ int tile[kScanTile];
     __shared__ int sh32[33];
     grid_dependency_wait();
     grid_dependents_launch();
-    cta_exclusive_scan(a, n, nullptr, tile, sh32);
+    cta_exclusive_scan(a, n, tail, tile, sh32);
 }
 
 constexpr int kRounds = kItemsPerWarp / 32;                       // 8
@@ -375,6 +376,10 @@ __global__ void __launch_bounds__(kScatterThreads) radix_scatter_kernel(
 }
 
 }  // namespace
+
+cudaError_t launch_exclusive_scan(int32_t *a, int64_t n, int32_t *total, cudaStream_t st) {
+    return launch(exclusive_scan_kernel, dim3(1), dim3(1024), 0, st, a, n, total);
+}
 
 int sched_pass_width(const Sizes &sz) {
     return sz.passes ? (sz.qbits + sz.passes - 1) / sz.passes : 0;
@@ -460,7 +465,7 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
         int32_t *h = hist + hstride * p;
         if (p > 0) {
             e = launch(exclusive_scan_kernel, dim3(1), dim3(1024), 0, st, h,
-                       (int64_t)(dmask + 1) * ntiles);
+                       (int64_t)(dmask + 1) * ntiles, (int32_t *)nullptr);
             if (e != cudaSuccess) return e;
         }
         // ping-pong: the last pass writes the caller's arrays

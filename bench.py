@@ -73,6 +73,19 @@ def job_throughput(world: int, tokens_per_rank: int, ms_max: float) -> float:
     return world * tokens_per_rank / (ms_max * 1e-3)
 
 
+def med_ms(pairs) -> float:
+    """Median duration (ms) of (start, end) CUDA event pairs."""
+    return float(np.median([a.elapsed_time(b) for a, b in pairs]))
+
+
+def config_of(cfg, world: int) -> dict:
+    """The workload's `config` object (the same keys on both arms)."""
+    return {"workload": cfg.name, "L": cfg.L, "d": cfg.d, "N_r": cfg.N_r, "N_c": cfg.N_c,
+            "N": cfg.N, "K": cfg.K, "B": cfg.B, "tokens_per_gpu": cfg.L,
+            "parallelism": f"replicas x{world} (token batches)",
+            "l2": "flushed between timed steps (256 MB write)"}
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -232,7 +245,8 @@ def run_omni(args, cfg, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
     clocks = clk.summary()
-    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    ms = med_ms(ev)
+    ms_mean = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     ms_max = reduce_max(ms, world, dev)
 
     # ---- ablation: the same layer with the expert stage in token order and
@@ -254,7 +268,7 @@ def run_omni(args, cfg, world, rank, local):
         aev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    tok_ms = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in aev])), world, dev)
+    tok_ms = reduce_max(med_ms(aev), world, dev)
     ablation = {"token_order_ms_per_step": tok_ms, "expert_centric_ms_per_step": ms_max,
                 "token_order_over_expert_centric": tok_ms / ms_max}
 
@@ -277,7 +291,7 @@ def run_omni(args, cfg, world, rank, local):
             gev[i][1].record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        gms = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in gev])), world, dev)
+        gms = reduce_max(med_ms(gev), world, dev)
         graph = {"value": job_throughput(world, L, gms), "unit": "tokens/s", "ms_per_step": gms}
         del g
 
@@ -321,9 +335,9 @@ def run_omni(args, cfg, world, rank, local):
         staged(sev[i])
     torch.cuda.synchronize()
     barrier(world)
-    st_router = float(np.mean([e[0].elapsed_time(e[1]) for e in sev]))
-    st_sched = float(np.mean([e[1].elapsed_time(e[2]) for e in sev]))
-    st_expert = float(np.mean([e[2].elapsed_time(e[3]) for e in sev]))
+    st_router = med_ms([(e[0], e[1]) for e in sev])
+    st_sched = med_ms([(e[1], e[2]) for e in sev])
+    st_expert = med_ms([(e[2], e[3]) for e in sev])
 
     # ---- the selection (row / column top-K + merge, on the same p) against the
     # pages' blockwise grid scan; a few steps, the scan scores all N cells
@@ -349,7 +363,7 @@ def run_omni(args, cfg, world, rank, local):
                 sel()
                 cev[i][1].record(stream)
             torch.cuda.synchronize()
-            res[name] = float(np.mean([a.elapsed_time(b) for a, b in cev]))
+            res[name] = med_ms(cev)
         topk_cmp = {"pruned_ms": res["pruned"], "blockwise_ms": res["blockwise"],
                     "blockwise_over_pruned": res["blockwise"] / res["pruned"]}
         del ws_r2, o
@@ -389,7 +403,7 @@ def run_omni(args, cfg, world, rank, local):
         torch.cuda.synchronize()
         if omni.omni_get_device_status(ws_b) != 0:
             raise RuntimeError("device status set in the backward")
-        bms = float(np.mean([a.elapsed_time(b) for a, b in bev]))
+        bms = med_ms(bev)
         # read x, dy and the U distinct W, V rows; read-modify-write their fp32
         # dW, dV rows; write dx
         bbytes = 4.0 * d * U + 16.0 * d * U + 2.0 * L * d + 4.0 * L * d + 4.0 * L * d
@@ -428,7 +442,7 @@ def run_omni(args, cfg, world, rank, local):
             mev[i][1].record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        res[name] = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in mev])), world, dev)
+        res[name] = reduce_max(med_ms(mev), world, dev)
     if omni.omni_get_device_status(ws_m) != 0:
         raise RuntimeError("device status set in the shared MLP")
     mlp_flops = 6.0 * L * d * F                      # x W_g^T, x W_u^T, h W_d^T
@@ -516,10 +530,9 @@ def run_omni(args, cfg, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded Gaussian inputs and random-init weights of the layer's shapes)",
-        "config": {"workload": cfg.name, "L": L, "d": d, "N_r": cfg.N_r, "N_c": cfg.N_c,
-                   "N": cfg.N, "K": cfg.K, "B": cfg.B, "tokens_per_gpu": L,
-                   "parallelism": f"replicas x{world} (token batches)",
-                   "l2": "flushed between timed steps (256 MB write)"},
+        "config": config_of(cfg, world),
+        "timing": "median of the timed steps' CUDA-event durations (mean in ms_per_step_mean)",
+        "ms_per_step_mean": ms_mean,
         "stages_ms": {"router_topk": st_router, "schedule": st_sched,
                       "grouped_expert": st_expert},
         "distinct_experts": U,
@@ -726,8 +739,7 @@ def run_reference(args, cfg, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * cfg.L / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "L": cfg.L, "d": cfg.d, "N_r": cfg.N_r,
-                   "N_c": cfg.N_c, "K": cfg.K, "B": cfg.B},
+        "config": config_of(cfg, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,

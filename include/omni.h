@@ -70,6 +70,8 @@ typedef enum {
 #define OMNI_Y_ACCUMULATE       2u  /* y += routed(x) instead of y = routed(x)                           */
 #define OMNI_TOKEN_ORDER        4u  /* omni_routed_fwd: expert stage in token order, no schedule (below)  */
 #define OMNI_TOPK_BLOCKWISE     8u  /* omni_router_topk: the pages' blockwise grid top-K (below)           */
+#define OMNI_EXPERT_DENSE      16u  /* expert stage: always try the tensor-core tiles for dense experts   */
+#define OMNI_EXPERT_SPARSE     32u  /* expert stage: every task on the task-by-task path (no tiles)       */
 
 /* Device status codes written into the workspace status word. */
 #define OMNI_DEV_OK              0
@@ -92,15 +94,26 @@ const char *omni_device_status_string(int dev_status);
 
 /*
  * Bytes of workspace that every entry point needs for these sizes (the same
- * layout serves all four calls).  Returns 0 if the sizes are invalid.
+ * layout serves all four calls) with flags 0.  Returns 0 if the sizes are
+ * invalid.
  */
 size_t omni_workspace_size(int L, int d, int N_r, int N_c, int K, int B);
+
+/*
+ * The same for calls made with `flags`: OMNI_EXPERT_DENSE needs room for
+ * the tensor-core expert path at any size, OMNI_EXPERT_SPARSE none, and
+ * OMNI_TOKEN_ORDER (omni_routed_fwd only) leaves out the schedule and the
+ * tensor-core path.  omni_workspace_size(...) is this with flags 0.
+ */
+size_t omni_workspace_size_flags(int L, int d, int N_r, int N_c, int K, int B, unsigned flags);
 
 /* Smaller workspaces for the three stage calls used on their own (each is at
  * most omni_workspace_size of the same sizes).  0 for invalid sizes. */
 size_t omni_router_workspace_size(int L, int N_r, int N_c, int K);
 size_t omni_schedule_workspace_size(int L, int K, int N, int B);
 size_t omni_expert_workspace_size(int L, int d, int K, int N, int B);
+/* omni_grouped_expert_fwd called with `flags` (OMNI_EXPERT_DENSE needs more). */
+size_t omni_expert_workspace_size_flags(int L, int d, int K, int N, int B, unsigned flags);
 
 /*
  * Cartesian product router, [R] step 2 and [G] section 2.2.
@@ -165,15 +178,34 @@ int omni_schedule(const int32_t *idx, const float *gate, int L, int K, int N, in
  * W_q, V_q and gate matrix G_q (gate of task (t, e), 0 where there is none),
  *   O_q = (G_q . SiLU(X_q W_q^T)) V_q,      y[t] += O_q[t]  for its tokens.
  * sigma is read as SiLU (one w_in per expert leaves SwiGLU without a gate).
- * Only the (token, expert) pairs that are tasks are computed: the zero
- * entries of G_q are skipped, not multiplied.
  *   x [L, d] bf16, W [N, d] bf16, V [N, d] bf16
  *   schedule arrays as produced by omni_schedule for the same L, K, N, B
  *   y [L, d] fp32  output (overwritten, or accumulated with OMNI_Y_ACCUMULATE)
- * Each y row is written once, but the order in which a token's tasks are
- * summed follows the order their slots were claimed (atomic counters), so y
- * may differ in the last bits between runs.  Limits: d % 256 == 0,
- * d <= OMNI_MAX_D, B <= OMNI_MAX_B.
+ * Two execution paths share the work, by how dense G_q is:
+ *   - tensor cores, for the "dense" experts: those that at least
+ *     thr = max(32, ceil(L / 96)) tasks use.  The active groups are walked
+ *     (active_groups, num_active, group_offsets); every group's dense experts
+ *     become columns of one bf16 tile GEMM over all L tokens,
+ *       P = G . SiLU(x W_D^T)  (P rounded to bf16),   y += P V_D,
+ *     with G the gates of their tasks (0 elsewhere).  At most a few thousand
+ *     columns are built (a cap set by L); the experts past it stay on the
+ *     other path.
+ *   - CUDA cores, task by task, for every other task: P = g SiLU(x_t . w_e)
+ *     for the task pairs only (fp32), then y_t = sum of p V[e] per token.
+ *   By default the tensor-core path is tried when L * K * d >= 2^31 (large
+ *   stages; below that an expert rarely reaches thr and its fixed cost is
+ *   not paid).  OMNI_EXPERT_DENSE tries it at any size (the workspace must
+ *   then come from omni_workspace_size_flags with that flag);
+ *   OMNI_EXPERT_SPARSE never does.  When no expert is dense the tiles do no
+ *   work.
+ * Checks on the device (OMNI_DEV_BAD_SCHEDULE): every task must lie in its
+ * group's range of group_offsets; on the tensor-core path also num_active in
+ * [0, G], active group ids in range, offsets non-decreasing within [0, M],
+ * each group's tasks of its own experts, and the active groups covering all
+ * L * K tasks.
+ * Each y row gets the CUDA-core sum in the order slots were claimed (atomic
+ * counters) and the tile sum in a fixed order, so y may differ in the last
+ * bits between runs.  Limits: d % 256 == 0, d <= OMNI_MAX_D, B <= OMNI_MAX_B.
  */
 int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                             int L, int d, int K, int N, int B,
@@ -187,7 +219,9 @@ int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_b
  * The whole routed branch: omni_router_topk, omni_schedule and
  * omni_grouped_expert_fwd back to back on `stream`, with every intermediate in
  * `ws` and no host synchronisation:  y = routed(x)  (the shared dense MLP of
- * [G] section 2.1 is not part of it).
+ * [G] section 2.1 is not part of it).  OMNI_EXPERT_DENSE / OMNI_EXPERT_SPARSE
+ * choose the expert stage's paths as for omni_grouped_expert_fwd (its
+ * schedule is produced here, so its offsets are not re-checked).
  *   x [L, d], W [N, d], V [N, d], W_r [N_r, d], W_c [N_c, d]  bf16
  *   y [L, d] fp32 output;  idx_out [L, K] int32, gate_out [L, K] fp32 are
  *   optional copies of the routing (NULL to skip).
@@ -198,7 +232,8 @@ int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_b
  * rows are fetched changes.  For a few tokens the grouping has nothing to
  * reuse and the schedule's launches are pure latency; for large batches the
  * flag is the token-centric execution the expert-centric schedule replaces
- * (an ablation).
+ * (an ablation); it needs only omni_workspace_size_flags(..., OMNI_TOKEN_ORDER)
+ * bytes and never uses the tensor-core path.
  * Limits: those of the three calls above.
  */
 int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
@@ -274,11 +309,15 @@ int omni_shared_mlp_fwd(const omni_bf16 *x, const omni_bf16 *W_g, const omni_bf1
  *     (different streams, or different host threads) race and must not be
  *     issued; the array keeps the last call's contents, and the call clears
  *     what has to start at zero itself;
- *   - the first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before capturing a stream into a CUDA graph;
+ *   - the array's device address is looked up (cudaGetSymbolAddress) on the
+ *     first call made in each CUDA context, with that context current, and
+ *     kept for later calls in the same context; make that first call before
+ *     capturing a stream into a CUDA graph.  A context created later for the
+ *     same device (after cudaDeviceReset, or a driver-API context other than
+ *     the primary one) gets its own lookup on its first call;
  *   - device-detected problems are recorded in the array's own status word,
- *     which omni_get_device_status cannot read.
+ *     which omni_get_device_status cannot read: read it with
+ *     omni_noalloc_get_device_status.
  * No device memory is allocated or freed.
  */
 int omni_grouped_expert_fwd_noalloc(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
@@ -287,6 +326,15 @@ int omni_grouped_expert_fwd_noalloc(const omni_bf16 *x, const omni_bf16 *W, cons
                                     const float *task_gate, const int32_t *group_offsets,
                                     const int32_t *active_groups, const int32_t *num_active,
                                     float *y, unsigned flags, omni_stream_t stream);
+
+/*
+ * The status word of omni_grouped_expert_fwd_noalloc's array on the current
+ * device: synchronises `stream`, copies the word into *status_out (an
+ * OMNI_DEV_* code, e.g. OMNI_DEV_BAD_SCHEDULE for a task whose expert or
+ * token id is out of range) and clears it.  Allocates nothing.  Returns
+ * OMNI_ERR_DEVICE when the word was set, OMNI_OK when it was clear.
+ */
+int omni_noalloc_get_device_status(omni_stream_t stream, int *status_out);
 
 /*
  * Diagnostic, not part of the layer: launches one CTA that waits on a

@@ -70,6 +70,7 @@ int main(void) {
     /* diagnostics need a workspace */
     EXPECT(omni_selftest_wait_timeout(NULL, 256, 10, NULL) == OMNI_ERR_INVALID_ARG);
     EXPECT(omni_get_device_status(NULL, 0, NULL, &st) == OMNI_ERR_INVALID_ARG);
+    EXPECT(omni_noalloc_get_device_status(NULL, NULL) == OMNI_ERR_INVALID_ARG);
 
     if (failures == 0) printf("abi_check: all expectations held\n");
     return failures == 0 ? 0 : 1;

@@ -58,6 +58,23 @@ def test_workspace_sizes(lib):
     assert omni.omni_workspace_size(4, 8, 4, 4, 17, 1) == 0         # K > N
     assert omni.omni_workspace_size(4, 8, 4, 4, 4, 2048) == 0       # B above the limit
     assert omni.omni_workspace_size(4, 8, 9000, 4, 4, 4) == 0       # axis above the limit
+    # flags: token order needs no schedule; the tensor-core expert path adds
+    # its buffers (gate matrix G fp32 and P bf16 [L, cap], W_D and V_D^T
+    # [cap, d] bf16, the compacted task list) when it is forced, and by
+    # default only for large stages (L * K * d >= 2^31)
+    DENSE, SPARSE, TOKEN = omni.OMNI_EXPERT_DENSE, omni.OMNI_EXPERT_SPARSE, omni.OMNI_TOKEN_ORDER
+    fl = lambda c, f: omni.omni_workspace_size_flags(c.L, c.d, c.N_r, c.N_c, c.K, c.B, f)
+    assert fl(h, 0) == full
+    assert fl(h, SPARSE) == full
+    assert fl(h, TOKEN) < full
+    thr = max(32, -(-h.L // 96))
+    cap = min(4096, -(-(h.M // thr) // 256) * 256)
+    assert fl(h, DENSE) >= full + 6 * h.L * cap + 4 * cap * h.d
+    z = configs.SKEW
+    assert z.M * z.d >= 2 ** 31
+    assert fl(z, 0) == fl(z, DENSE) > fl(z, SPARSE)
+    assert (omni.omni_expert_workspace_size_flags(h.L, h.d, h.K, h.N, h.B, DENSE) >
+            omni.omni_expert_workspace_size(h.L, h.d, h.K, h.N, h.B))
     # shared MLP: the status header plus h [L, F] bf16
     F = configs.mlp_hidden(h.d)
     assert omni.omni_shared_mlp_workspace_size(h.L, h.d, F) == 256 + 2 * h.L * F

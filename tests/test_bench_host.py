@@ -1,6 +1,8 @@
 """Host logic of bench.py (CPU only): the launch count it claims, the radix
 pass count, the clock-sample parsing and the traffic lookup that is only
 trusted while the profiled kernel source is unchanged."""
+import hashlib
+import json
 import os
 
 import pytest
@@ -43,9 +45,16 @@ def test_clock_summary_reads_reasons_and_load_median(tmp_path):
 
 
 def test_traffic_only_for_the_profiled_source(tmp_path):
+    # the committed capture is trusted only for the source whose hash it
+    # records; any other source (e.g. a later edit) gives no traffic figure
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["grouped_expert_stage"]
     src = os.path.join(ROOT, "atomic_expert_layer_b200", "csrc", "expert.cu")
+    cur = open(src, "rb").read()
     got = bench.traffic_from_profile(src)
-    assert got is not None and got > 1e9                      # the committed headline capture
+    if hashlib.sha256(cur).hexdigest() == rec["source_sha256"]:
+        assert got == rec["dram_bytes_per_launch_full_size"] and got > 1e9
+    else:
+        assert got is None
     other = tmp_path / "expert.cu"
-    other.write_bytes(open(src, "rb").read() + b"\n// changed\n")
+    other.write_bytes(cur + b"\n// changed\n")
     assert bench.traffic_from_profile(str(other)) is None

@@ -56,3 +56,31 @@ def test_noalloc_matches_workspace_call_twice(cfg):
     y_ref = oracle.expert_fwd_token_centric(u["x"], u["W"], u["V"], host(rt["idx"]),
                                             host(rt["gate"]), tokens=toks)
     check_y(host(y)[toks], y_ref)
+
+
+@pytest.mark.gpu
+def test_noalloc_reports_bad_schedule_through_its_own_status_word():
+    # a task whose expert id is out of range: the call clamps it (every access
+    # stays in bounds) and records OMNI_DEV_BAD_SCHEDULE in the array's status
+    # word, which only omni_noalloc_get_device_status can read
+    cfg = configs.TINY
+    dev = "cuda"
+    t = inputs.make_inputs(cfg, dev, seed=7)
+    rt = omni.router_topk(t["x"], t["W_r"], t["W_c"], cfg.K)
+    sched = omni.schedule(rt["idx"], rt["gate"], cfg.N, cfg.B)
+    y = torch.zeros((cfg.L, cfg.d), dtype=torch.float32, device=dev)
+
+    def call(task_expert):
+        omni.omni_grouped_expert_fwd_noalloc(
+            t["x"], t["W"], t["V"], cfg.L, cfg.d, cfg.K, cfg.N, cfg.B, sched["task_token"],
+            task_expert, sched["task_gate"], sched["group_offsets"], sched["active_groups"],
+            sched["num_active"], y, 0)
+
+    omni.omni_noalloc_get_device_status()           # clear whatever an earlier call left
+    bad = sched["task_expert"].clone()
+    bad[5] = cfg.N                                  # one past the last expert
+    call(bad)
+    assert omni.omni_noalloc_get_device_status() == 3    # OMNI_DEV_BAD_SCHEDULE
+    assert omni.omni_noalloc_get_device_status() == 0    # the read cleared it
+    call(sched["task_expert"])                      # a clean call leaves it clear
+    assert omni.omni_noalloc_get_device_status() == 0
