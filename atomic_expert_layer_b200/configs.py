@@ -59,6 +59,12 @@ def sweep(L: int) -> LayerConfig:
 # with W and V of 512 MB each (N = 512^2) instead of 3.5 GB.
 PROFILE = LayerConfig("profile_L4096_d1024_N262144_K64_B20", 4096, 1024, 512, 512, 64, 20)
 
+# The skewed layer's router (1024 x 1024 grid, K = 128, Zipf bias) at 4096
+# tokens, for profiler captures of the router stage (which never touches W, V).
+SKEW_ROUTER_PROFILE = LayerConfig("skew_router_profile_L4096_d2048_N1048576_K128_B128_zipf", 4096,
+                                  2048, 1024, 1024, 128, 128, zipf=True)
+
+
 def mlp_hidden(d: int) -> int:
     """Hidden width F of the shared dense MLP beside a layer of width d: 8d/3
     rounded up to a multiple of 64 (the width at which a gated MLP has the
@@ -66,5 +72,5 @@ def mlp_hidden(d: int) -> int:
     return -(-8 * d // (3 * 64)) * 64
 
 
-ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L] + [PROFILE]
+ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L] + [PROFILE, SKEW_ROUTER_PROFILE]
 BY_NAME = {c.name: c for c in ALL}

@@ -100,7 +100,7 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
     if (regions & kRegExpert) w.tok_count = take(4 * L);
     const bool dense = (regions & kRegDense) && sz.dense;
     if (dense) {
-        w.dz_bits = take(4 * (size_t)((sz.N + 31) / 32));
+        w.dz_cnt = take(4 * (size_t)sz.N);
         w.dz_ghot = take(4 * (G + 1));
         w.dz_ccount = take(8);
     }

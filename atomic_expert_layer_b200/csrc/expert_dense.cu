@@ -25,12 +25,13 @@
 // dense experts of every group, so y is written once per element (no atomics).
 //
 // Steps (all on the caller's stream, no host synchronisation, no spin-waits):
-//   1. count:   per active group, tasks per expert; experts with >= thr tasks
-//               are marked in a bitmap and counted per group.
+//   1. count:   tasks per expert over the whole list; then per active group
+//               the number of its experts with >= thr tasks.
 //   2. scan:    exclusive scan of the per-group counts -> each group's first
 //               dense column; the total is E (capped at `cap` columns).
-//   3. list:    per group, the ids of its dense experts in column order; marks
-//               past the cap are cleared (those experts stay task-by-task).
+//   3. list:    per group, the ids of its dense experts in column order; each
+//               one's counter becomes -(column + 1).  Experts past the cap get
+//               no column and stay task by task.
 //   4. gather:  W_D = the dense experts' W rows [cap, d] and V_D^T [d, cap]
 //               (zero past E), and G zeroed over the E_pad columns in use.
 //   5. split:   each task either writes its gate into G (dense expert) or is
@@ -50,75 +51,92 @@ namespace omni {
 namespace {
 
 // ---------------------------------------------------------------- 1. count
-// One CTA per active group (grid-stride over the active list).  Checks the
-// schedule arrays it reads: num_active, the group ids and their offsets, and
-// that every task of a group has an expert of that group; it also adds up
-// the tasks the active groups cover (the split step checks that it is M).
+// (a) Tasks per expert over the whole sorted list (grid-stride, 32
+// consecutive tasks per warp; equal experts inside a warp are added by one
+// atomic).  Checks that every task lies in its group's range of the sorted
+// order (group_offsets).
 __global__ void __launch_bounds__(256)
-dense_count_kernel(const int32_t *__restrict__ task_expert, const int32_t *__restrict__ off,
-                   const int32_t *__restrict__ active, const int32_t *__restrict__ num_active,
-                   int64_t G, int B, int64_t N, int64_t M, int thr, int32_t *__restrict__ ghot,
-                   uint32_t *__restrict__ bits, int32_t *__restrict__ covered, int *status) {
-    extern __shared__ int cnt[];                      // B counters
-    __shared__ int s_hot;
+dense_use_kernel(const int32_t *__restrict__ task_expert, int64_t M,
+                 const int32_t *__restrict__ off, int B, int64_t N, int32_t *__restrict__ cnt,
+                 int *status) {
     grid_dependency_wait();
     grid_dependents_launch();
-    const int tid = threadIdx.x;
+    const unsigned lane = lane_id();
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t base = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32;
+         base < M; base += nwarps * 32) {
+        const int64_t m = base + lane;
+        int32_t key = -1;
+        if (m < M) {
+            const int32_t e = task_expert[m];
+            bool ok = e >= 0 && (int64_t)e < N;
+            if (ok) {
+                const int64_t q = e / B;
+                ok = m >= off[q] && m < off[q + 1];
+            }
+            if (ok)
+                key = e;
+            else
+                set_status(status, OMNI_DEV_BAD_SCHEDULE);
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0 && lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&cnt[key], __popc(peers));
+    }
+}
+
+// (b) Warp per active group: the number of its experts with >= thr tasks.
+// Checks num_active, the group ids and their offsets, and adds up the
+// tasks the active groups cover (the split step checks that it is M).
+__global__ void dense_mark_kernel(const int32_t *__restrict__ cnt, const int32_t *__restrict__ off,
+                                  const int32_t *__restrict__ active,
+                                  const int32_t *__restrict__ num_active, int64_t G, int B,
+                                  int64_t N, int64_t M, int thr, int32_t *__restrict__ ghot,
+                                  int32_t *__restrict__ covered, int *status) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const unsigned lane = lane_id();
+    const int gwarp = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     int nact = *num_active;
     if (nact < 0 || (int64_t)nact > G) {
-        if (tid == 0 && blockIdx.x == 0) set_status(status, OMNI_DEV_BAD_SCHEDULE);
+        if (gwarp == 0 && lane == 0) set_status(status, OMNI_DEV_BAD_SCHEDULE);
         nact = nact < 0 ? 0 : (int)G;
     }
-    for (int i = blockIdx.x; i < nact; i += gridDim.x) {
-        const int32_t q = active[i];                  // the same in every thread
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    for (int i = gwarp; i < nact; i += nwarps) {
+        const int32_t q = active[i];
         if (q < 0 || (int64_t)q >= G) {
-            if (tid == 0) set_status(status, OMNI_DEV_BAD_SCHEDULE);
+            if (lane == 0) set_status(status, OMNI_DEV_BAD_SCHEDULE);
             continue;
         }
         const int32_t o0 = off[q], o1 = off[q + 1];
         if (o0 < 0 || (int64_t)o1 > M || o1 < o0) {
-            if (tid == 0) set_status(status, OMNI_DEV_BAD_SCHEDULE);
+            if (lane == 0) set_status(status, OMNI_DEV_BAD_SCHEDULE);
             continue;
         }
-        if (tid == 0) atomicAdd(covered, o1 - o0);
+        if (lane == 0) atomicAdd(covered, o1 - o0);
         if (o1 - o0 < thr) continue;                  // no expert of q can reach thr
-        for (int j = tid; j < B; j += blockDim.x) cnt[j] = 0;
-        if (tid == 0) s_hot = 0;
-        __syncthreads();
         const int64_t base = (int64_t)q * B;
-        for (int64_t m = o0 + tid; m < o1; m += blockDim.x) {
-            const int64_t j = (int64_t)task_expert[m] - base;
-            if (j >= 0 && j < B)
-                atomicAdd(&cnt[j], 1);
-            else
-                set_status(status, OMNI_DEV_BAD_SCHEDULE);
-        }
-        __syncthreads();
         int nh = 0;
-        for (int j = tid; j < B; j += blockDim.x) {
+        for (int j0 = 0; j0 < B; j0 += 32) {
+            const int j = j0 + (int)lane;
             const int64_t e = base + j;
-            if (cnt[j] >= thr && e < N) {
-                ++nh;
-                atomicOr(&bits[e >> 5], 1u << (e & 31));
-            }
+            nh += __popc(__ballot_sync(0xffffffffu, j < B && e < N && cnt[e] >= thr));
         }
-        if (nh) atomicAdd(&s_hot, nh);
-        __syncthreads();
-        if (tid == 0) ghot[q] = s_hot;
-        __syncthreads();                              // cnt is reused by the next group
+        if (lane == 0) ghot[q] = nh;
     }
 }
 
 // ----------------------------------------------------------------- 3. list
-// Warp per active group with dense experts: their ids in column order.  A
-// column at or past `cap` is not built; its expert's mark is cleared so the
-// split step keeps its tasks on the CUDA-core path.  Clearing only removes the
-// highest columns (the last ones of a group, and every later group), so the
-// columns of the experts that keep their marks do not move.
+// Warp per active group with dense experts: their ids in column order, and
+// each one's counter replaced by -(column + 1), which is how the split step
+// tells a dense expert and finds its column.  Columns at or past `cap` are not
+// built; those experts keep their (positive) counts and stay on the CUDA-core
+// path.  They are the highest columns (the last ones of a group, and every
+// later group), so the columns of the others do not move.
 __global__ void dense_list_kernel(const int32_t *__restrict__ hoff,
                                   const int32_t *__restrict__ active,
                                   const int32_t *__restrict__ num_active, int64_t G, int B,
-                                  int64_t N, int cap, uint32_t *__restrict__ bits,
+                                  int64_t N, int thr, int cap, int32_t *__restrict__ cnt,
                                   int32_t *__restrict__ list) {
     grid_dependency_wait();
     grid_dependents_launch();
@@ -136,14 +154,12 @@ __global__ void dense_list_kernel(const int32_t *__restrict__ hoff,
         for (int j0 = 0; j0 < B; j0 += 32) {
             const int j = j0 + (int)lane;
             const int64_t e = base + j;
-            const bool hot = j < B && e < N && ((bits[e >> 5] >> (e & 31)) & 1u);
+            const bool hot = j < B && e < N && cnt[e] >= thr;
             const unsigned bal = __ballot_sync(0xffffffffu, hot);
             const int h = h0 + run + __popc(bal & lanemask_lt());
-            if (hot) {
-                if (h < cap)
-                    list[h] = (int32_t)e;
-                else
-                    atomicAnd(&bits[e >> 5], ~(1u << (e & 31)));
+            if (hot && h < cap) {
+                list[h] = (int32_t)e;
+                cnt[e] = -(h + 1);
             }
             run += __popc(bal);
         }
@@ -224,20 +240,19 @@ dense_gather_kernel(const uint16_t *__restrict__ W, const uint16_t *__restrict__
 }
 
 // ---------------------------------------------------------------- 5. split
-// Each warp takes chunks of 32 x 32 tasks.  A task of a marked (dense) expert
-// writes its gate into G at (token, column); the column is the group's first
-// dense column plus the number of marked experts of the group below it.  The
-// other tasks are appended, in chunk order, to the compacted list of the
-// CUDA-core path (one atomic per chunk).  Also checks that each task lies in
-// its group's range of the sorted order, and that the active groups cover
-// all M tasks (num_active too small or an active group missing).
+// Each warp takes chunks of 32 x 32 tasks.  A task whose expert has a
+// column (counter < 0) writes its gate into G at (token, column); the other
+// tasks are appended, in chunk order, to the compacted list of the CUDA-core
+// path: lane r keeps the ballot of round r, the warp reserves the chunk's
+// room with one atomic and re-reads only the tasks it appends.  Also checks
+// that the active groups cover all M tasks (num_active too small, or an
+// active group missing or listed twice).
 constexpr int kSplitRounds = 32;
 
 __global__ void __launch_bounds__(256)
 dense_split_kernel(const int32_t *__restrict__ task_token, const int32_t *__restrict__ task_expert,
-                   const float *__restrict__ task_gate, int64_t M, const int32_t *__restrict__ off,
-                   int B, int64_t N, int L, const uint32_t *__restrict__ bits,
-                   const int32_t *__restrict__ hoff, int cap, float *__restrict__ Gm,
+                   const float *__restrict__ task_gate, int64_t M, int64_t N, int L,
+                   const int32_t *__restrict__ cnt, int cap, float *__restrict__ Gm,
                    int32_t *__restrict__ c_tok, int32_t *__restrict__ c_exp,
                    float *__restrict__ c_gate, int32_t *__restrict__ c_count,
                    const int32_t *__restrict__ covered, int *status) {
@@ -250,68 +265,48 @@ dense_split_kernel(const int32_t *__restrict__ task_token, const int32_t *__rest
     const int64_t chunk = 32 * kSplitRounds;
     for (int64_t c0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * chunk;
          c0 < M; c0 += nwarps * chunk) {
-        // pass 1: classify, write the dense gates, count the rest
-        int ncold = 0;
+        unsigned my_mask = 0;                         // lane r: the CUDA-core tasks of round r
+#pragma unroll 4
         for (int r = 0; r < kSplitRounds; ++r) {
             const int64_t m = c0 + r * 32 + lane;
             bool cold = false;
             if (m < M) {
                 int32_t t = task_token[m], e = task_expert[m];
-                const float g = task_gate[m];
-                bool bad = t < 0 || t >= L || e < 0 || (int64_t)e >= N;
-                if (!bad) {
-                    const int64_t q = e / B;
-                    bad = m < off[q] || m >= off[q + 1];
-                }
-                if (bad) {
+                if (t < 0 || t >= L || e < 0 || (int64_t)e >= N) {
                     set_status(status, OMNI_DEV_BAD_SCHEDULE);
                     t = t < 0 || t >= L ? 0 : t;
                     e = e < 0 || (int64_t)e >= N ? 0 : e;
                 }
-                if ((bits[e >> 5] >> (e & 31)) & 1u) {
-                    // rank of e among the marked experts of its group
-                    const int64_t q = e / B;
-                    const int64_t b0 = q * B;
-                    int rank = 0;
-                    for (int64_t w = b0 >> 5; w <= ((int64_t)e >> 5); ++w) {
-                        uint32_t word = bits[w];
-                        const int64_t lo = w << 5;
-                        if (lo < b0) word &= ~0u << (b0 - lo);               // below the group
-                        if (lo + 32 > e) word &= (1u << (e - lo)) - 1u;      // e and above
-                        rank += __popc(word);
-                    }
-                    Gm[(size_t)t * cap + hoff[q] + rank] = g;
-                } else {
+                const int32_t v = cnt[e];
+                if (v < 0)
+                    Gm[(size_t)t * cap + (-v - 1)] = task_gate[m];
+                else
                     cold = true;
-                }
-            }
-            ncold += __popc(__ballot_sync(0xffffffffu, cold));
-        }
-        int base = 0;
-        if (lane == 0 && ncold) base = atomicAdd(c_count, ncold);
-        base = __shfl_sync(0xffffffffu, base, 0);
-        // pass 2: append the CUDA-core tasks in order
-        for (int r = 0; r < kSplitRounds && ncold; ++r) {
-            const int64_t m = c0 + r * 32 + lane;
-            bool cold = false;
-            int32_t t = 0, e = 0;
-            float g = 0.f;
-            if (m < M) {
-                t = task_token[m];
-                e = task_expert[m];
-                g = task_gate[m];
-                t = t < 0 || t >= L ? 0 : t;
-                e = e < 0 || (int64_t)e >= N ? 0 : e;
-                cold = !((bits[e >> 5] >> (e & 31)) & 1u);
             }
             const unsigned bal = __ballot_sync(0xffffffffu, cold);
-            if (cold) {
-                const int at = base + __popc(bal & lanemask_lt());
+            if (lane == (unsigned)r) my_mask = bal;
+        }
+        const int mine = __popc(my_mask);
+        const int incl = warp_iscan(mine);
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (total == 0) continue;
+        int base = 0;
+        if (lane == 0) base = atomicAdd(c_count, total);
+        base = __shfl_sync(0xffffffffu, base, 0) + incl - mine;   // this lane's round starts here
+        for (int r = 0; r < kSplitRounds; ++r) {
+            const unsigned bal = __shfl_sync(0xffffffffu, my_mask, r);
+            const int at0 = __shfl_sync(0xffffffffu, base, r);
+            if (bal == 0) continue;
+            if ((bal >> lane) & 1u) {
+                const int64_t m = c0 + r * 32 + lane;
+                int32_t t = task_token[m], e = task_expert[m];
+                t = t < 0 || t >= L ? 0 : t;
+                e = e < 0 || (int64_t)e >= N ? 0 : e;
+                const int at = at0 + __popc(bal & lanemask_lt());
                 c_tok[at] = t;
                 c_exp[at] = e;
-                c_gate[at] = g;
+                c_gate[at] = task_gate[m];
             }
-            base += __popc(bal);
         }
     }
 }
@@ -547,7 +542,7 @@ cudaError_t launch_dense_gemm(const CUtensorMap &a, const CUtensorMap &b, const 
 // ------------------------------------------------------------------- host
 DenseWs dense_ws_of(const Sizes &sz, void *ws, const WsLayout &lay) {
     DenseWs o;
-    o.bits = ws_at<uint32_t>(ws, lay.dz_bits);
+    o.cnt = ws_at<int32_t>(ws, lay.dz_cnt);
     o.ghot = ws_at<int32_t>(ws, lay.dz_ghot);
     o.ehot = ws_at<int32_t>(ws, lay.d_ehot);
     o.ccount = ws_at<int32_t>(ws, lay.dz_ccount);
@@ -571,41 +566,31 @@ cudaError_t launch_dense_prepare(const uint16_t *W, const uint16_t *V, const Siz
                                  const DenseWs &o, int *status, cudaStream_t st) {
     const int sms = device_sm_count();
     const int64_t G = sz.G;
-    cudaError_t e;
-    {
-        int64_t grid = G < (int64_t)sms * 8 ? G : (int64_t)sms * 8;
-        if (grid < 1) grid = 1;
-        e = launch(dense_count_kernel, dim3((unsigned)grid), dim3(256), (size_t)4 * sz.B, st,
-                   task_expert, group_offsets, active_groups, num_active, G, sz.B, sz.N, sz.M,
-                   o.thr, o.ghot, o.bits, o.ccount + 1, status);
-        if (e != cudaSuccess) return e;
-    }
+    auto grid_for = [&](int64_t warps_needed) {
+        int64_t g = (warps_needed + 7) / 8;               // 8 warps per CTA
+        if (g > (int64_t)sms * 8) g = (int64_t)sms * 8;
+        return (unsigned)(g < 1 ? 1 : g);
+    };
+    cudaError_t e = launch(dense_use_kernel, dim3(grid_for((sz.M + 31) / 32)), dim3(256), 0, st,
+                           task_expert, sz.M, group_offsets, sz.B, sz.N, o.cnt, status);
+    if (e != cudaSuccess) return e;
+    e = launch(dense_mark_kernel, dim3(grid_for(G)), dim3(256), 0, st, (const int32_t *)o.cnt,
+               group_offsets, active_groups, num_active, G, sz.B, sz.N, sz.M, o.thr, o.ghot,
+               o.ccount + 1, status);
+    if (e != cudaSuccess) return e;
     // ghot has G + 1 entries (the last one zero): its scan gives hoff[G] = E
     if ((e = launch_exclusive_scan(o.ghot, G + 1, o.ehot, st)) != cudaSuccess) return e;
-    {
-        int64_t grid = (G + 7) / 8;
-        if (grid > (int64_t)sms * 8) grid = (int64_t)sms * 8;
-        if (grid < 1) grid = 1;
-        e = launch(dense_list_kernel, dim3((unsigned)grid), dim3(256), 0, st,
-                   (const int32_t *)o.ghot, active_groups, num_active, G, sz.B, sz.N, o.cap,
-                   o.bits, o.list);
-        if (e != cudaSuccess) return e;
-    }
+    e = launch(dense_list_kernel, dim3(grid_for(G)), dim3(256), 0, st, (const int32_t *)o.ghot,
+               active_groups, num_active, G, sz.B, sz.N, o.thr, o.cap, o.cnt, o.list);
+    if (e != cudaSuccess) return e;
     e = launch(dense_gather_kernel, dim3((unsigned)(sms * 4)), dim3(kGatherThreads), 0, st, W, V,
                sz.d, sz.L, sz.N, (const int32_t *)o.list, (const int32_t *)o.ehot, o.cap, o.whot,
                o.vt, o.G);
     if (e != cudaSuccess) return e;
-    {
-        const int64_t chunks = (sz.M + 32 * kSplitRounds - 1) / (32 * kSplitRounds);
-        int64_t grid = (chunks + 7) / 8;
-        if (grid > (int64_t)sms * 8) grid = (int64_t)sms * 8;
-        if (grid < 1) grid = 1;
-        e = launch(dense_split_kernel, dim3((unsigned)grid), dim3(256), 0, st, task_token,
-                   task_expert, task_gate, sz.M, group_offsets, sz.B, sz.N, sz.L,
-                   (const uint32_t *)o.bits, (const int32_t *)o.ghot, o.cap, o.G, o.c_tok,
-                   o.c_exp, o.c_gate, o.ccount, (const int32_t *)(o.ccount + 1), status);
-    }
-    return e;
+    const int64_t chunks = (sz.M + 32 * kSplitRounds - 1) / (32 * kSplitRounds);
+    return launch(dense_split_kernel, dim3(grid_for(chunks)), dim3(256), 0, st, task_token,
+                  task_expert, task_gate, sz.M, sz.N, sz.L, (const int32_t *)o.cnt, o.cap, o.G,
+                  o.c_tok, o.c_exp, o.c_gate, o.ccount, (const int32_t *)(o.ccount + 1), status);
 }
 
 cudaError_t launch_dense_gemms(const uint16_t *x, const Sizes &sz, const DenseWs &o, float *y,

@@ -29,7 +29,7 @@ struct WsLayout {
     size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, tok_count, tok_slots;
     size_t z_cnt, z_ndist;   // schedule counters (workspace copies)
     // tensor-core expert path: zeroed per call (dz_*), then the rest
-    size_t dz_bits, dz_ghot, dz_ccount;
+    size_t dz_cnt, dz_ghot, dz_ccount;
     size_t d_ehot, d_list, d_whot, d_vt, d_G, d_P, d_ctok, d_cexp, d_cgate;
     size_t zero_end;         // [0, zero_end) must be zero when a call starts
     size_t total;
@@ -111,6 +111,9 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
 int sched_pass_width(const Sizes &sz);
 uint32_t sched_pass_mask(const Sizes &sz, int p);
 SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay);
+// the radix scatter combines equal histogram increments of a warp (crowded
+// groups, see schedule.cu)
+bool sched_aggregate(const Sizes &sz);
 
 // ---- grouped expert stage (expects the per-token slot counters zeroed).
 // task_token == nullptr: the tasks are in token order, task m belongs to
@@ -130,7 +133,7 @@ cudaError_t launch_grouped_expert(const uint16_t *x, const uint16_t *W, const ui
 // V_D^T, G (gates of their tasks) and the compacted list of the other tasks;
 // gemms: P = G . SiLU(x W_D^T), then y += P V_D.
 struct DenseWs {
-    uint32_t *bits;          // [ceil(N / 32)] dense-expert marks
+    int32_t *cnt;            // [N] tasks per expert, then -(column + 1) for dense ones
     int32_t *ghot;           // [G + 1] dense experts per group, then their first column
     int32_t *ehot;           // [1] dense experts found (before the cap)
     int32_t *ccount;         // [2] compacted tasks; tasks covered by the active groups

@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(kScatterThreads) radix_scatter_kernel(
     const float *__restrict__ src_gate, int64_t M, int B, int shift, uint32_t dmask,
     int64_t ntiles, const int32_t *__restrict__ hist_scanned, int32_t *__restrict__ dst_tok,
     int32_t *__restrict__ dst_exp, float *__restrict__ dst_gate,
-    int32_t *__restrict__ hist_next, int next_shift, uint32_t next_dmask) {
+    int32_t *__restrict__ hist_next, int next_shift, uint32_t next_dmask, int agg) {
     __shared__ int wcount[kScatterThreads / 32][256];
     grid_dependency_wait();
     grid_dependents_launch();
@@ -360,14 +360,26 @@ __global__ void __launch_bounds__(kScatterThreads) radix_scatter_kernel(
         const bool valid = e[j] >= 0;
         const uint32_t dg = valid ? digit_of(e[j], B, shift, dmask) : 0xffffffffu;
         const unsigned peers = __match_any_sync(0xffffffffu, dg);
+        int pos = -1;
         if (valid) {
-            const int pos = wcount[warp][dg] + __popc(peers & lanemask_lt());
+            pos = wcount[warp][dg] + __popc(peers & lanemask_lt());
             dst_tok[pos] = tk[j];
             dst_exp[pos] = e[j];
             dst_gate[pos] = g[j];
-            if (hist_next)
-                atomicAdd(&hist_next[(int64_t)digit_of(e[j], B, next_shift, next_dmask) * ntiles +
-                                     pos / kSortTile], 1);
+        }
+        if (hist_next) {
+            // the next pass's (digit, output tile) counter; with `agg` (crowded
+            // groups put many tasks on one counter) lanes with the same key
+            // share one atomic
+            const uint32_t hk = valid ? digit_of(e[j], B, next_shift, next_dmask) * (uint32_t)ntiles +
+                                            (uint32_t)(pos / kSortTile)
+                                      : 0xffffffffu;
+            if (agg) {
+                const unsigned hp = __match_any_sync(0xffffffffu, hk);
+                if (valid && lane == (unsigned)(__ffs(hp) - 1)) atomicAdd(&hist_next[hk], __popc(hp));
+            } else if (valid) {
+                atomicAdd(&hist_next[hk], 1);
+            }
         }
         __syncwarp();
         if (valid && (lanemask_lt() & peers) == 0) wcount[warp][dg] += __popc(peers);
@@ -390,6 +402,13 @@ uint32_t sched_pass_mask(const Sizes &sz, int p) {
     const int shift = p * width;
     const int w = (sz.qbits - shift) < width ? (sz.qbits - shift) : width;
     return (1u << w) - 1u;
+}
+
+bool sched_aggregate(const Sizes &sz) {
+    // crowded groups (64 tasks or more per group on average): the radix
+    // histogram atomics would pile up on a few addresses, so warps combine
+    // equal ones first
+    return sz.M >= 64 * sz.G;
 }
 
 SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay) {
@@ -481,7 +500,7 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
         e = launch(radix_scatter_kernel, dim3((unsigned)ntiles), dim3(kScatterThreads), 0, st,
                    s_tok, s_exp, s_gate, M, sz.B, shift, dmask, ntiles, (const int32_t *)h, d_tok,
                    d_exp, d_gate, last ? nullptr : hist + hstride * (p + 1), (p + 1) * width,
-                   last ? 0u : pass_mask(p + 1));
+                   last ? 0u : pass_mask(p + 1), sched_aggregate(sz) ? 1 : 0);
         if (e != cudaSuccess) return e;
         s_tok = d_tok; s_exp = d_exp; s_gate = d_gate;
     }

@@ -548,21 +548,23 @@ __device__ __forceinline__ bool better(const Cand &u, const Cand &v) {
 }
 
 struct MergeLayout {   // offsets (words) inside one warp's region
-    size_t rv, ri, cv, ci, sval, hist, cur, q, out_s, out_n, words;
+    size_t rv, ri, cv, ci, hist, q, out_s, out_n, words;
 };
 
-__host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C) {
+// Per warp: rv, ri [Kr], cv, ci [Kc] (the token's row and column top-K),
+// hist [kNB] (bucket counts, then bucket starts, then bucket ends), the area
+// q of max(4 CAP, C) words (the fast path's 128-bit candidate keys, or the
+// fallback's candidate keys and then the indices it keeps), out_S, out_n [K].
+__host__ __device__ inline MergeLayout merge_layout(int K, int Kr, int Kc, int C, int cap) {
     MergeLayout m;
     size_t o = 0;
     m.rv = o; o += Kr;
     m.ri = o; o += Kr;
     m.cv = o; o += Kc;
     m.ci = o; o += Kc;
-    m.sval = o; o += C;
     m.hist = o; o += kNB;
-    m.cur = o; o += kNB;
-    o = (o + 3) & ~(size_t)3;                 // 16-byte alignment for Cand / u64
-    m.q = o; o += 4 * (size_t)C;               // Cand[C] (fallback) or the candidate keys
+    o = (o + 3) & ~(size_t)3;                 // 16-byte alignment for the u64 keys
+    m.q = o; o += (4 * (size_t)cap > (size_t)C ? 4 * (size_t)cap : (size_t)C);
     m.out_s = o; o += K;
     m.out_n = o; o += K;
     m.words = (o + 3) & ~(size_t)3;
@@ -600,7 +602,7 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     const int wpb = blockDim.x >> 5;
-    const MergeLayout ml = merge_layout(K, Kr, Kc, C);
+    const MergeLayout ml = merge_layout(K, Kr, Kc, C, CAP);
     uint32_t *table = smem_u;                                   // C entries
     int *off = reinterpret_cast<int *>(table + C);               // Kr + 1 entries
     const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
@@ -643,10 +645,8 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     uint32_t *ri = base + ml.ri;
     float *cv = reinterpret_cast<float *>(base + ml.cv);
     uint32_t *ci = base + ml.ci;
-    float *sval = reinterpret_cast<float *>(base + ml.sval);
     uint32_t *hist = base + ml.hist;
-    uint32_t *cur = base + ml.cur;
-    Cand *q = reinterpret_cast<Cand *>(base + ml.q);
+    uint32_t *qw = base + ml.q;
     uint64_t *tmp = reinterpret_cast<uint64_t *>(base + ml.q);
     float *out_S = reinterpret_cast<float *>(base + ml.out_s);
     uint32_t *out_n = base + ml.out_n;
@@ -661,34 +661,52 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     }
     __syncwarp();
     const float smax = __fadd_rn(rv[0], cv[0]);           // cell (0, 0) is the largest
-    if (CAP > 0) {
-        for (int b = lane; b < kNB; b += 32) hist[b] = 0u;
-        __syncwarp();
-    }
-    for (int c = lane; c < C; c += 32) {
+    // S of candidate c (one fp32 addition, recomputed where needed)
+    auto score_of = [&](int c, int *a_out, int *b_out) {
         const uint32_t ab = table[c];
-        const float S = __fadd_rn(rv[ab >> 16], cv[ab & 0xffffu]);
-        sval[c] = S;
-        if (CAP > 0) {
-            const int b = bucket_of(smax, S);
-            if (b < kNB) atomicAdd(&hist[b], 1u);
-        }
-    }
-    __syncwarp();
+        *a_out = (int)(ab >> 16);
+        *b_out = (int)(ab & 0xffffu);
+        return __fadd_rn(rv[*a_out], cv[*b_out]);
+    };
 
     bool done = false;
     if (CAP > 0) {
+        for (int b = lane; b < kNB; b += 32) hist[b] = 0u;
+        __syncwarp();
+        for (int c = lane; c < C; c += 32) {
+            int a, b2;
+            const int b = bucket_of(smax, score_of(c, &a, &b2));
+            if (b < kNB) atomicAdd(&hist[b], 1u);
+        }
+        __syncwarp();
         int bs = 0;
         const int ncand = bucket_find(hist, K, &bs);
         if (ncand >= K && ncand <= CAP) {
-            bucket_starts(hist, cur);
+            // counts -> bucket starts, in place; the scatter below advances
+            // each bucket's entry to its end
+            {
+                constexpr int per = kNB / 32;
+                uint32_t cnt[per];
+                int tot = 0;
+#pragma unroll
+                for (int j = 0; j < per; ++j) {
+                    cnt[j] = hist[lane * per + j];
+                    tot += (int)cnt[j];
+                }
+                int run = warp_iscan(tot) - tot;
+#pragma unroll
+                for (int j = 0; j < per; ++j) {
+                    hist[lane * per + j] = (uint32_t)run;
+                    run += (int)cnt[j];
+                }
+                __syncwarp();
+            }
             for (int c = lane; c < C; c += 32) {
-                const float S = sval[c];
+                int a, bb;
+                const float S = score_of(c, &a, &bb);
                 const int b = bucket_of(smax, S);
                 if (b <= bs) {
-                    const uint32_t pos = atomicAdd(&cur[b], 1u);
-                    const uint32_t ab = table[c];
-                    const int a = (int)(ab >> 16), bb = (int)(ab & 0xffffu);
+                    const uint32_t pos = atomicAdd(&hist[b], 1u);
                     const uint32_t nn = ri[a] * (uint32_t)N_c + ci[bb];
                     tmp[2 * pos] = ((uint64_t)f2key(S) << 32) | f2key(rv[a]);
                     tmp[2 * pos + 1] = ((uint64_t)f2key(cv[bb]) << 32) | (uint64_t)(0xffffffffu - nn);
@@ -696,11 +714,12 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
             }
             __syncwarp();
             // inside a bucket, order by the full key: rank among its peers
+            // (bucket b now spans [end of b - 1, end of b))
             for (int pos = lane; pos < ncand; pos += 32) {
                 const uint64_t kh = tmp[2 * pos], kl = tmp[2 * pos + 1];
                 const int b = bucket_of(smax, key2f((uint32_t)(kh >> 32)));
-                const int s0 = (int)hist[b];
-                const int s1 = b < bs ? (int)hist[b + 1] : ncand;
+                const int s0 = b > 0 ? (int)hist[b - 1] : 0;
+                const int s1 = (int)hist[b];
                 int r = 0;
                 for (int q = s0; q < s1; ++q) {
                     const uint64_t qh = tmp[2 * q], ql = tmp[2 * q + 1];
@@ -716,35 +735,43 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
         }
     }
     if (!done) {
-        // ---- exact fallback: radix select on key(S), rank sort by the full key
-        uint32_t *ckey = reinterpret_cast<uint32_t *>(sval);
-        for (int c = lane; c < C; c += 32) ckey[c] = f2key(sval[c]);
+        // ---- exact fallback: radix select on key(S), then a rank sort by the
+        // full key of the kept candidates (their keys recomputed from the
+        // candidate table, so only their indices are stored)
+        uint32_t *ckey = qw;
+        for (int c = lane; c < C; c += 32) {
+            int a, b;
+            ckey[c] = f2key(score_of(c, &a, &b));
+        }
         __syncwarp();
         int take_eq;
         const uint32_t T = warp_radix_select(ckey, C, K, hist, &take_eq);
+        // keep the candidates with key >= T, compacted in place (a round reads
+        // its 32 keys before any write, and writes only below them)
         int nq = 0;
         for (int c0 = 0; c0 < C; c0 += 32) {
             const int c = c0 + (int)lane;
             const bool in_q = c < C && ckey[c] >= T;
             const unsigned bal = __ballot_sync(0xffffffffu, in_q);
-            if (in_q) {
-                const int pos = nq + __popc(bal & lanemask_lt());
-                const uint32_t ab = table[c];
-                const int a = (int)(ab >> 16), b = (int)(ab & 0xffffu);
-                Cand cd;
-                cd.skey = ckey[c];
-                cd.prkey = f2key(rv[a]);
-                cd.pckey = f2key(cv[b]);
-                cd.n = ri[a] * (uint32_t)N_c + ci[b];
-                q[pos] = cd;
-            }
+            __syncwarp();
+            if (in_q) qw[nq + __popc(bal & lanemask_lt())] = (uint32_t)c;
             nq += __popc(bal);
+            __syncwarp();
         }
-        __syncwarp();
+        auto cand_of = [&](int c) {
+            int a, b;
+            const float S = score_of(c, &a, &b);
+            Cand cd;
+            cd.skey = f2key(S);
+            cd.prkey = f2key(rv[a]);
+            cd.pckey = f2key(cv[b]);
+            cd.n = ri[a] * (uint32_t)N_c + ci[b];
+            return cd;
+        };
         for (int u = lane; u < nq; u += 32) {
-            const Cand cu = q[u];
+            const Cand cu = cand_of((int)qw[u]);
             int r = 0;
-            for (int v = 0; v < nq; ++v) r += better(q[v], cu) ? 1 : 0;
+            for (int v = 0; v < nq; ++v) r += better(cand_of((int)qw[v]), cu) ? 1 : 0;
             if (r < K) {
                 out_S[r] = key2f(cu.skey);
                 out_n[r] = cu.n;
@@ -895,12 +922,27 @@ static cudaError_t launch_merge_e(const float *row_val, const int *row_idx, cons
     SchedPrep pv;
     std::memset(&pv, 0, sizeof pv);
     if (prep) pv = *prep;
-    const MergeLayout ml = merge_layout(K, Kr, Kc, C);
+    const MergeLayout ml = merge_layout(K, Kr, Kc, C, CAP);
     const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
     const size_t per_warp = ml.words * 4;
-    int wpb = (int)((64 * 1024 - head * 4) / per_warp);
-    if (wpb > 8) wpb = 8;
-    if (wpb < 1) wpb = 1;
+    // warps per CTA: the most resident warps per SM (228 KB of shared memory
+    // with 1 KB reserved per CTA, 48 registers per thread, 64 warps), fewest
+    // warps per CTA on a tie
+    int wpb = 1, best = 0;
+    for (int w = 1; w <= 8; ++w) {
+        const size_t smem = head * 4 + per_warp * (size_t)w;
+        if (smem > 227 * 1024) break;
+        int ctas = (int)((228 * 1024) / (smem + 1024));
+        const int by_regs = 65536 / (48 * 32 * w);
+        if (ctas > by_regs) ctas = by_regs;
+        if (ctas > 32) ctas = 32;
+        int warps = ctas * w;
+        if (warps > 64) warps = 64;
+        if (warps > best) {
+            best = warps;
+            wpb = w;
+        }
+    }
     const size_t smem = head * 4 + per_warp * wpb;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel<CAP>,
@@ -924,6 +966,7 @@ cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const fl
 #define OMNI_MG(c) return launch_merge_e<c>(row_val, row_idx, col_val, col_idx, L, N_c, K, Kr, Kc, C, idx, score, gate, dead_r, dead_c, N_r, prep, st);
     if (cap < K) { OMNI_MG(0) }
     if (cap <= 96) { OMNI_MG(96) }
+    if (cap <= 128) { OMNI_MG(128) }
     if (cap <= 192) { OMNI_MG(192) }
     if (cap <= 320) { OMNI_MG(320) }
     if (cap <= 576) { OMNI_MG(576) }

@@ -125,7 +125,10 @@ def launches_per_step(cfg) -> int:
     sched = 1 + (p + max(p - 1, 0))               # scan, scatters, histogram scans (the
     if cfg.L <= 16:                               # per-token step runs in the merge kernel)
         sched = 0                                 # decode batches run in token order
-    return router + sched + 2                     # group pass, token pass
+    # the tensor-core expert path (default for L * K * d >= 2^31): expert use,
+    # dense marks, column scan, column list, gather, split, two tile GEMMs
+    dense = 8 if cfg.L > 16 and cfg.M * cfg.d >= 2 ** 31 else 0
+    return router + sched + 2 + dense             # group pass, token pass
 
 
 class ClockSampler:

@@ -26,6 +26,10 @@ def test_launches_per_step_matches_the_profiled_step():
     # decode batches skip the schedule: router (4) + the two expert passes
     assert bench.launches_per_step(configs.sweep(16)) == 6
     assert bench.launches_per_step(configs.sweep(1)) == 6
+    # the skewed layer adds the tensor-core expert path: 8 launches
+    # (use, mark, scan, list, gather, split, two GEMMs); its 8192 groups need
+    # two radix passes, like the headline
+    assert bench.launches_per_step(configs.SKEW) == 10 + 8
 
 
 def test_clock_summary_reads_reasons_and_load_median(tmp_path):
