@@ -63,12 +63,12 @@ inline T *ws_at(void *ws, size_t off) {
 }
 
 // ---- router GEMM (tcgen05): s_r = x W_r^T, s_c = x W_c^T (fp32)
-// part_r [L, 2 * ceil(N_r/128)] and part_c: per (token, 64 columns) the max
+// part_r [L, 2 * ceil(N_r/224)] and part_c: per (token, tile, column half) the max
 // of s and the sum of exp(s - max), as float pairs ((-inf, 0) if empty).
 cudaError_t launch_router_gemm(const uint16_t *x, const uint16_t *W_r, const uint16_t *W_c,
                                int L, int d, int N_r, int N_c, float *s_r, float *s_c,
                                float *part_r, float *part_c, int *status, cudaStream_t st);
-constexpr int kGemmPartCols = 64;          // columns per LogSoftmax partial
+constexpr int kGemmPartCols = 112;         // columns per LogSoftmax partial (two per 224-column tile)
 
 // ---- router projection for a handful of tokens (no LogSoftmax partials)
 bool router_small_ok(int L, int d);
