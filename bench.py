@@ -272,8 +272,21 @@ def run_omni(args, cfg, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     tok_ms = reduce_max(med_ms(aev), world, dev)
+    # device memory of each path beyond the shared inputs (x, W, V, W_r, W_c)
+    # and the output y: the library allocates nothing, so it is the workspace
+    # each path needs; and what an implementation that materialises every
+    # token's gathered expert rows (W[idx], V[idx] as [L, K, d] bf16) would
+    # allocate for them
+    ws_ec = omni.omni_workspace_size_flags(L, d, cfg.N_r, cfg.N_c, cfg.K, cfg.B, 0)
+    ws_to = omni.omni_workspace_size_flags(L, d, cfg.N_r, cfg.N_c, cfg.K, cfg.B,
+                                           omni.OMNI_TOKEN_ORDER)
+    gathered = 2 * 2 * L * cfg.K * d
     ablation = {"token_order_ms_per_step": tok_ms, "expert_centric_ms_per_step": ms_max,
-                "token_order_over_expert_centric": tok_ms / ms_max}
+                "token_order_over_expert_centric": tok_ms / ms_max,
+                "workspace_bytes_expert_centric": ws_ec,
+                "workspace_bytes_token_order": ws_to,
+                "materialised_gather_bytes": gathered,
+                "materialised_gather_over_expert_centric_workspace": gathered / ws_ec}
 
     # ---- small batches are launch-bound: the same step as one CUDA graph
     graph = None
