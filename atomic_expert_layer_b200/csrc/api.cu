@@ -97,7 +97,10 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.bitmap = take(4 * (size_t)((sz.N + 31) / 32));
         w.hist = take(4 * 256 * (size_t)sz.ntiles * (size_t)sz.passes);   // one per radix pass
     }
-    if (regions & kRegExpert) w.tok_count = take(4 * L);
+    if (regions & kRegExpert) {
+        w.tok_count = take(4 * L);
+        w.dec_bar = take(4);
+    }
     const bool dense = (regions & kRegDense) && sz.dense;
     if (dense) {
         w.dz_cnt = take(4 * (size_t)sz.N);
@@ -420,6 +423,23 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     // nothing here reads the distinct-expert count, so it is not kept
     SchedPrep prep = sched_prep_of(sz, ws, lay);
     prep.bitmap = nullptr;
+    if (L <= kTokenOrderMaxL && decode_fused_ok(L, d, N_r, N_c, K, sz.Kr, sz.Kc, sz.C)) {
+        // a handful of tokens: the whole step in one cooperative launch
+        rc = cuda_rc(launch_decode_fused(
+            x, W, V, W_r, W_c, L, d, N_r, N_c, K, sz.Kr, sz.Kc, sz.C, ws_at<float>(ws, lay.s_r),
+            ws_at<float>(ws, lay.s_c), ws_at<float>(ws, lay.row_val), ws_at<int>(ws, lay.row_idx),
+            ws_at<float>(ws, lay.col_val), ws_at<int>(ws, lay.col_idx), idx, score, gate, y,
+            (flags & OMNI_Y_ACCUMULATE) != 0, ws_at<unsigned>(ws, lay.dec_bar),
+            ws_at<int>(ws, lay.hdr), st));
+        if (rc) return rc;
+        if (idx_out && (rc = cuda_rc(cudaMemcpyAsync(idx_out, idx, 4 * (size_t)sz.M,
+                                                     cudaMemcpyDeviceToDevice, st))))
+            return rc;
+        if (gate_out && (rc = cuda_rc(cudaMemcpyAsync(gate_out, gate, 4 * (size_t)sz.M,
+                                                      cudaMemcpyDeviceToDevice, st))))
+            return rc;
+        return OMNI_OK;
+    }
     rc = router_topk_impl(x, W_r, W_c, sz, nullptr, nullptr, idx, score, gate,
                           flags & ~OMNI_ROUTER_LOGPROBS_IN, ws, lay, st,
                           token_order ? nullptr : &prep);

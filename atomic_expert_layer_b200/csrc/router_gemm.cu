@@ -19,6 +19,7 @@
 // out-of-bounds fill and are masked on store.
 #include "omni_common.cuh"
 #include "omni_internal.h"
+#include "router_small.cuh"
 #include "tcgen05.cuh"
 
 namespace omni {
@@ -282,21 +283,6 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
     }
 }
 
-// ------------------------------------------------- few tokens (L <= 4)
-// The GEMM above walks one 128-row M tile through the whole K loop when a
-// batch has a handful of tokens, which makes it latency-bound.  Then the
-// projection is a streamed read of W_r and W_c: warp w of CTA b takes grid
-// rows (kSmallRows * (kSmallWarps * b + w)) .. + kSmallRows - 1 (W_r rows,
-// then W_c rows) and issues every load of them at once (lane l holds the
-// 8-wide slices l, l + 32, ..., d <= 2048), the batch's x rows sit in shared
-// memory, and each (row, token) dot product is reduced over the warp.  Only
-// s is written; the axis kernels then take LogSoftmax themselves.  Measured
-// on B200 at d = 2048: faster than the tile GEMM at L = 1 (5.7 vs ~14 us),
-// slower by L = 16, so it serves L <= 4.
-constexpr int kSmallRows = 2;          // grid rows per warp
-constexpr int kSmallWarps = 8;
-constexpr int kSmallSlices = 8;        // 8-wide slices per lane: d <= 32 * 8 * 8
-
 template <int LM>
 __global__ void __launch_bounds__(32 * kSmallWarps)
 router_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W_r,
@@ -308,82 +294,17 @@ router_small_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__
     grid_dependents_launch();
     const int d8 = d >> 3;
     const int warp = threadIdx.x >> 5;
-    const unsigned lane = lane_id();
     const int g0 = (blockIdx.x * kSmallWarps + warp) * kSmallRows;
-    const int ntot = N_r + N_c;
-    // this warp's rows, every slice in flight at once
-    uint4 wu[kSmallRows][kSmallSlices];
-#pragma unroll
-    for (int r = 0; r < kSmallRows; ++r) {
-        const int g = g0 + r < ntot ? g0 + r : ntot - 1;     // clamped; not written
-        const uint4 *w4 = reinterpret_cast<const uint4 *>(
-            g < N_r ? W_r + (size_t)g * d : W_c + (size_t)(g - N_r) * d);
-#pragma unroll
-        for (int i = 0; i < kSmallSlices; ++i) {
-            const int c8 = (int)lane + 32 * i;
-            wu[r][i] = c8 < d8 ? w4[c8] : make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
-    // x rows into shared memory, every copy in flight at once
-    for (int i = threadIdx.x; i < L * d8; i += blockDim.x)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-                     ::"r"(smem_u32(xs + i)), "l"(reinterpret_cast<const uint4 *>(x) + i)
-                     : "memory");
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
-    float acc[kSmallRows][LM];
-#pragma unroll
-    for (int r = 0; r < kSmallRows; ++r)
-#pragma unroll
-        for (int t = 0; t < LM; ++t) acc[r][t] = 0.f;
-#pragma unroll
-    for (int i = 0; i < kSmallSlices; ++i) {
-        const int c8 = (int)lane + 32 * i;
-        if (c8 < d8) {
-            float wf[kSmallRows][8];
-#pragma unroll
-            for (int r = 0; r < kSmallRows; ++r) {
-                const uint32_t w4[4] = {wu[r][i].x, wu[r][i].y, wu[r][i].z, wu[r][i].w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    wf[r][2 * q] = __uint_as_float(w4[q] << 16);
-                    wf[r][2 * q + 1] = __uint_as_float(w4[q] & 0xffff0000u);
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < LM; ++t) {
-                if (t < L) {
-                    const uint4 u = xs[(size_t)t * d8 + c8];
-                    const uint32_t x4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float xlo = __uint_as_float(x4[q] << 16);
-                        const float xhi = __uint_as_float(x4[q] & 0xffff0000u);
-#pragma unroll
-                        for (int r = 0; r < kSmallRows; ++r) {
-                            acc[r][t] = fmaf(xlo, wf[r][2 * q], acc[r][t]);
-                            acc[r][t] = fmaf(xhi, wf[r][2 * q + 1], acc[r][t]);
-                        }
-                    }
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < kSmallRows; ++r) {
-        const int g = g0 + r;
-#pragma unroll
-        for (int t = 0; t < LM; ++t) {
-            if (t < L) {
-                const float v = warp_sum(acc[r][t]);
-                if (lane == 0 && g < ntot) {
-                    if (g < N_r) s_r[(size_t)t * N_r + g] = v;
-                    else s_c[(size_t)t * N_c + (g - N_r)] = v;
-                }
-            }
-        }
-    }
+    small_rows_dot<LM>(xs, W_r, W_c, L, d, N_r, N_c, g0, s_r, s_c, [&]() {
+        // x rows into shared memory, every copy in flight at once
+        for (int i = threadIdx.x; i < L * d8; i += blockDim.x)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                         ::"r"(smem_u32(xs + i)), "l"(reinterpret_cast<const uint4 *>(x) + i)
+                         : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+    });
 }
 
 template <int LM>

@@ -34,6 +34,7 @@
 
 #include "omni_common.cuh"
 #include "omni_internal.h"
+#include "router_small.cuh"
 #include "sched_token.cuh"
 
 namespace omni {
@@ -194,34 +195,16 @@ __device__ __forceinline__ void bucket_starts(uint32_t *hist, uint32_t *cur) {
 // Dynamic smem per warp (words): vals[nmax] | hist[kNB] | cur[kNB] |
 // area[max(2 kmax, 2 CAP)], where area is either sel_key[kmax] + sel_idx[kmax]
 // (fallback) or the candidate keys tmp[CAP] (u64)
+// One (token, axis) row, one warp, exact: LogSoftmax (optional; from the
+// GEMM partials when given) and the top kx = min(K, n) of the row by
+// (p desc, index asc) into oval / oidx.  `base` is the warp's shared area of
+// nmax + 2 kNB + 2 kmax (+1) words.
 template <int CAP>
-__global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__restrict__ in_c,
-                                 int logsoftmax, const float2 *__restrict__ part_r,
-                                 const float2 *__restrict__ part_c, float *__restrict__ p_r_out,
-                                 float *__restrict__ p_c_out, int L, int N_r, int N_c, int K,
-                                 float *__restrict__ row_val, int *__restrict__ row_idx,
-                                 float *__restrict__ col_val, int *__restrict__ col_idx,
-                                 int nmax, int kmax, size_t warp_words,
-                                 const int *__restrict__ only) {
-    extern __shared__ __align__(16) uint32_t smem_u[];
-    grid_dependency_wait();
-    grid_dependents_launch();
-    const int warp = threadIdx.x >> 5;
+__device__ void axis_row_exact(const float *__restrict__ in, int n, int kx, int logsoftmax,
+                               const float2 *__restrict__ part, int t, float *__restrict__ pout,
+                               float *__restrict__ oval, int *__restrict__ oidx, int nmax,
+                               int kmax, uint32_t *base) {
     const unsigned lane = lane_id();
-    const int wpb = blockDim.x >> 5;
-    const int64_t prob = (int64_t)blockIdx.x * wpb + warp;
-    if (prob >= 2 * (int64_t)L) return;
-    if (only && only[prob] == 0) return;          // handled by the register kernel
-    const int t = (int)(prob >> 1);
-    const int axis = (int)(prob & 1);
-    const int n = axis ? N_c : N_r;
-    const int kx = K < n ? K : n;
-    const float *in = (axis ? in_c : in_r) + (size_t)t * n;
-    float *pout = axis ? p_c_out : p_r_out;
-    float *oval = (axis ? col_val : row_val) + (size_t)t * kx;
-    int *oidx = (axis ? col_idx : row_idx) + (size_t)t * kx;
-
-    uint32_t *base = smem_u + (size_t)warp * warp_words;
     float *vals = reinterpret_cast<float *>(base);
     uint32_t *hist = base + nmax;
     uint32_t *cur = hist + kNB;
@@ -232,7 +215,6 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
 
     float vmax = -INFINITY;
     bool counted = false;                  // buckets already filled
-    const float2 *part = axis ? part_c : part_r;
     if (logsoftmax && part) {
         float mx;
         const float lse = lse_from_partials(part, t, n, &mx);
@@ -381,6 +363,34 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
         oval[r] = key2f(ku);
         oidx[r] = sel_idx[u];
     }
+}
+
+template <int CAP>
+__global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__restrict__ in_c,
+                                 int logsoftmax, const float2 *__restrict__ part_r,
+                                 const float2 *__restrict__ part_c, float *__restrict__ p_r_out,
+                                 float *__restrict__ p_c_out, int L, int N_r, int N_c, int K,
+                                 float *__restrict__ row_val, int *__restrict__ row_idx,
+                                 float *__restrict__ col_val, int *__restrict__ col_idx,
+                                 int nmax, int kmax, size_t warp_words,
+                                 const int *__restrict__ only) {
+    extern __shared__ __align__(16) uint32_t smem_u[];
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int warp = threadIdx.x >> 5;
+    const int wpb = blockDim.x >> 5;
+    const int64_t prob = (int64_t)blockIdx.x * wpb + warp;
+    if (prob >= 2 * (int64_t)L) return;
+    if (only && only[prob] == 0) return;          // handled by the register kernel
+    const int t = (int)(prob >> 1);
+    const int axis = (int)(prob & 1);
+    const int n = axis ? N_c : N_r;
+    const int kx = K < n ? K : n;
+    axis_row_exact<CAP>((axis ? in_c : in_r) + (size_t)t * n, n, kx, logsoftmax,
+                        axis ? part_c : part_r, t, axis ? p_c_out : p_r_out,
+                        (axis ? col_val : row_val) + (size_t)t * kx,
+                        (axis ? col_idx : row_idx) + (size_t)t * kx, nmax, kmax,
+                        smem_u + (size_t)warp * warp_words);
 }
 
 // ------------------------------------------------- axis top-K, registers
@@ -581,33 +591,11 @@ __device__ __forceinline__ void discard_l2_lines(const float *p, int n) {
         asm volatile("discard.global.L2 [%0], 128;" ::"l"(a) : "memory");
 }
 
-// Shared by the CTA: table[c] = (a << 16) | b for the c-th candidate, a-major.
-// dead_r / dead_c (may be null): the router GEMM's logits s_r [L, N_r] and
-// s_c [L, N_c] in the library's workspace.  Every reader of them has finished
-// when this kernel runs, so each warp drops its token's rows from L2: about
-// 43 MB of dirty lines at 4096 tokens of 2 x 1304 logits that would otherwise
-// be written back to HBM while the expert stage streams its rows.
-template <int CAP>
-__global__ void merge_topk_kernel(const float *__restrict__ row_val,
-                                  const int *__restrict__ row_idx,
-                                  const float *__restrict__ col_val,
-                                  const int *__restrict__ col_idx, int L, int N_c, int K, int Kr,
-                                  int Kc, int C, int32_t *__restrict__ idx,
-                                  float *__restrict__ score, float *__restrict__ gate,
-                                  const float *dead_r, const float *dead_c, int N_r,
-                                  SchedPrep prep) {
-    extern __shared__ __align__(16) uint32_t smem_u[];
-    grid_dependency_wait();
-    grid_dependents_launch();
+// Candidate table (the whole CTA): table[c] = (a << 16) | b for the c-th cell
+// (a, b) with (a+1)(b+1) <= K, a-major; off (Kr + 1 ints) is scratch.
+__device__ void merge_table(int K, int Kr, int Kc, int C, uint32_t *table, int *off) {
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
-    const int wpb = blockDim.x >> 5;
-    const MergeLayout ml = merge_layout(K, Kr, Kc, C, CAP);
-    uint32_t *table = smem_u;                                   // C entries
-    int *off = reinterpret_cast<int *>(table + C);               // Kr + 1 entries
-    const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
-
-    // ---- candidate table (once per CTA): off[a] = sum_{a' < a} nb(a')
     if (warp == 0) {
         int carry = 0;
         for (int a0 = 0; a0 < Kr; a0 += 32) {
@@ -634,13 +622,20 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     }
     __syncthreads();
 
-    const int t = blockIdx.x * wpb + warp;
-    if (t >= L) return;
-    if (dead_r) {
-        discard_l2_lines(dead_r + (size_t)t * N_r, N_r);
-        discard_l2_lines(dead_c + (size_t)t * N_c, N_c);
-    }
-    uint32_t *base = smem_u + head + (size_t)warp * ml.words;
+}
+
+// One token, one warp: the global top-K of S = fl32(p_r[i] + p_c[j]) over the
+// candidate cells from the token's row and column top-K (row_val / row_idx:
+// Kr entries, col_val / col_idx: Kc entries), ranked by (S, p_r, p_c, n), and
+// the gates; idx / score / gate are the token's K outputs.  `base` is the
+// warp's shared area (merge_layout), `table` the CTA's candidate table.
+template <int CAP>
+__device__ void merge_token(const uint32_t *table, uint32_t *base, const MergeLayout &ml,
+                            const float *__restrict__ row_val, const int *__restrict__ row_idx,
+                            const float *__restrict__ col_val, const int *__restrict__ col_idx,
+                            int N_c, int K, int Kr, int Kc, int C, int t, int32_t *idx,
+                            float *score, float *gate, const SchedPrep &prep) {
+    const unsigned lane = lane_id();
     float *rv = reinterpret_cast<float *>(base + ml.rv);
     uint32_t *ri = base + ml.ri;
     float *cv = reinterpret_cast<float *>(base + ml.cv);
@@ -652,12 +647,12 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     uint32_t *out_n = base + ml.out_n;
 
     for (int a = lane; a < Kr; a += 32) {
-        rv[a] = row_val[(size_t)t * Kr + a];
-        ri[a] = (uint32_t)row_idx[(size_t)t * Kr + a];
+        rv[a] = row_val[a];
+        ri[a] = (uint32_t)row_idx[a];
     }
     for (int b = lane; b < Kc; b += 32) {
-        cv[b] = col_val[(size_t)t * Kc + b];
-        ci[b] = (uint32_t)col_idx[(size_t)t * Kc + b];
+        cv[b] = col_val[b];
+        ci[b] = (uint32_t)col_idx[b];
     }
     __syncwarp();
     const float smax = __fadd_rn(rv[0], cv[0]);           // cell (0, 0) is the largest
@@ -787,9 +782,9 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     for (int k = lane; k < K; k += 32) {
         const float S = out_S[k];
         const float g = expf(S - smx) / den;
-        idx[(size_t)t * K + k] = (int32_t)out_n[k];
-        score[(size_t)t * K + k] = S;
-        gate[(size_t)t * K + k] = g;
+        idx[k] = (int32_t)out_n[k];
+        score[k] = S;
+        gate[k] = g;
         out_S[k] = g;                                 // this lane's entries only
     }
     if (prep.a_tok) {
@@ -800,9 +795,234 @@ __global__ void merge_topk_kernel(const float *__restrict__ row_val,
     }
 }
 
+// dead_r / dead_c (may be null): the router GEMM's logits s_r [L, N_r] and
+// s_c [L, N_c] in the library's workspace.  Every reader of them has finished
+// when this kernel runs, so each warp drops its token's rows from L2: about
+// 43 MB of dirty lines at 4096 tokens of 2 x 1304 logits that would otherwise
+// be written back to HBM while the expert stage streams its rows.
+template <int CAP>
+__global__ void merge_topk_kernel(const float *__restrict__ row_val,
+                                  const int *__restrict__ row_idx,
+                                  const float *__restrict__ col_val,
+                                  const int *__restrict__ col_idx, int L, int N_c, int K, int Kr,
+                                  int Kc, int C, int32_t *__restrict__ idx,
+                                  float *__restrict__ score, float *__restrict__ gate,
+                                  const float *dead_r, const float *dead_c, int N_r,
+                                  SchedPrep prep) {
+    extern __shared__ __align__(16) uint32_t smem_u[];
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int warp = threadIdx.x >> 5;
+    const int wpb = blockDim.x >> 5;
+    const MergeLayout ml = merge_layout(K, Kr, Kc, C, CAP);
+    uint32_t *table = smem_u;                                   // C entries
+    int *off = reinterpret_cast<int *>(table + C);               // Kr + 1 entries
+    const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
+    merge_table(K, Kr, Kc, C, table, off);
+    const int t = blockIdx.x * wpb + warp;
+    if (t >= L) return;
+    if (dead_r) {
+        discard_l2_lines(dead_r + (size_t)t * N_r, N_r);
+        discard_l2_lines(dead_c + (size_t)t * N_c, N_c);
+    }
+    merge_token<CAP>(table, smem_u + head + (size_t)warp * ml.words, ml,
+                     row_val + (size_t)t * Kr, row_idx + (size_t)t * Kr,
+                     col_val + (size_t)t * Kc, col_idx + (size_t)t * Kc, N_c, K, Kr, Kc, C, t,
+                     idx + (size_t)t * K, score + (size_t)t * K, gate + (size_t)t * K, prep);
+}
+
 // candidates the fast path takes (the k best plus the boundary bucket); 0 = none
 int fast_capacity(int k) {
     return k <= 1024 ? ((k + 64 + 31) / 32) * 32 : 0;
+}
+
+// ------------------------------------------------------- fused decode step
+// For a handful of tokens the routed forward is latency-bound: six dependent
+// launches, each starting cold, cost about 37 us at L = 1 against a 1.7 us
+// roofline.  Tokens are independent once the router projection is done, so
+// one cooperative launch (every CTA resident) runs the whole step in three
+// phases separated by a grid barrier (a bounded wait):
+//   A. all CTAs: the streamed router projection (small_rows_dot, the
+//      arithmetic of the small-batch projection kernel) into s; y zeroed
+//      unless accumulating;
+//   B. CTA t < L, token t: LogSoftmax and the exact row and column top-K
+//      (warps 0 and 1, axis_row_exact), then the merge and the gates (warp 0,
+//      merge_token): the same selection as the separate kernels;
+//   C. every warp, one task (t, k) at a time in token order: h = x_t . w_e,
+//      p = g SiLU(h), y_t += p v_e (16-byte fp32 reductions; the order in
+//      which a token's K terms land varies from run to run).
+constexpr int kDecodeWarps = 8;
+constexpr int kDecodeCap = 192;            // axis and merge fast-path capacity (K <= 128)
+constexpr int kDecodeSlices = 8;           // 8-wide slices per lane: d <= 2048
+
+struct DecodeArgs {
+    const uint16_t *x, *W, *V, *W_r, *W_c;
+    int L, d, N_r, N_c, K, Kr, Kc, C;
+    int64_t N;
+    float *s_r, *s_c;
+    float *row_val, *col_val;
+    int *row_idx, *col_idx;
+    int32_t *idx;
+    float *score, *gate;
+    float *y;
+    int accumulate;
+    unsigned *bar;                         // zeroed per call
+    int *status;
+    int nmax, kmax;
+    int axis_words;                        // shared words per axis warp
+    int merge_head;                        // candidate table and its scratch
+};
+
+// All CTAs of the grid arrive; the wait gives up after kWaitLimitNs and
+// records OMNI_DEV_WAIT_TIMEOUT (then the CTA returns).
+__device__ bool decode_grid_barrier(unsigned *bar, unsigned target, int *status, int *s_ok) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(bar, 1u);
+        bool ok = true;
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t it = 0;; ++it) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+            if (v >= target) break;
+            if ((it & 63u) == 63u &&
+                (it > kWaitSpinLimit || global_timer_ns() - t0 > kWaitLimitNs)) {
+                set_status(status, OMNI_DEV_WAIT_TIMEOUT);
+                ok = false;
+                break;
+            }
+        }
+        *s_ok = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                 ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+__global__ void __launch_bounds__(32 * kDecodeWarps) decode_fused_kernel(const DecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem_u[];
+    __shared__ int s_ok;
+    const int warp = threadIdx.x >> 5;
+    const unsigned lane = lane_id();
+    const int d8 = a.d >> 3;
+
+    // ---- A. router projection; y zeroed
+    {
+        uint4 *xs = reinterpret_cast<uint4 *>(smem_u);            // [L][d / 8]
+        const int nblk = (a.N_r + a.N_c + kSmallRows - 1) / kSmallRows;
+        bool staged = false;
+        for (int blk0 = blockIdx.x * kDecodeWarps; blk0 < nblk;
+             blk0 += gridDim.x * kDecodeWarps) {                    // the same in every warp
+            small_rows_dot<16>(xs, a.W_r, a.W_c, a.L, a.d, a.N_r, a.N_c,
+                               (blk0 + warp) * kSmallRows, a.s_r, a.s_c, [&]() {
+                if (!staged) {
+                    for (int i = threadIdx.x; i < a.L * d8; i += blockDim.x)
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                                     ::"r"(smem_u32(xs + i)),
+                                     "l"(reinterpret_cast<const uint4 *>(a.x) + i)
+                                     : "memory");
+                    asm volatile("cp.async.commit_group;" ::: "memory");
+                    asm volatile("cp.async.wait_group 0;" ::: "memory");
+                    __syncthreads();
+                    staged = true;
+                }
+            });
+        }
+        if (!a.accumulate) {
+            float4 *y4 = reinterpret_cast<float4 *>(a.y);
+            const int n4 = a.L * (a.d >> 2);
+            for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x)
+                y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    if (!decode_grid_barrier(a.bar, gridDim.x, a.status, &s_ok)) return;
+
+    // ---- B. selection of token t = blockIdx.x
+    if ((int)blockIdx.x < a.L) {
+        const int t = blockIdx.x;
+        uint32_t *table = smem_u;
+        merge_table(a.K, a.Kr, a.Kc, a.C, table, reinterpret_cast<int *>(table + a.C));
+        uint32_t *area = smem_u + a.merge_head;
+        if (warp < 2) {
+            const int axis = warp;
+            const int n = axis ? a.N_c : a.N_r;
+            const int kx = axis ? a.Kc : a.Kr;
+            axis_row_exact<kDecodeCap>((axis ? a.s_c : a.s_r) + (size_t)t * n, n, kx, 1, nullptr, t,
+                                       nullptr, (axis ? a.col_val : a.row_val) + (size_t)t * kx,
+                                       (axis ? a.col_idx : a.row_idx) + (size_t)t * kx, a.nmax,
+                                       a.kmax, area + (size_t)axis * a.axis_words);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const MergeLayout ml = merge_layout(a.K, a.Kr, a.Kc, a.C, kDecodeCap);
+            const SchedPrep none{};
+            merge_token<kDecodeCap>(table, area, ml, a.row_val + (size_t)t * a.Kr,
+                                    a.row_idx + (size_t)t * a.Kr, a.col_val + (size_t)t * a.Kc,
+                                    a.col_idx + (size_t)t * a.Kc, a.N_c, a.K, a.Kr, a.Kc, a.C, t,
+                                    a.idx + (size_t)t * a.K, a.score + (size_t)t * a.K,
+                                    a.gate + (size_t)t * a.K, none);
+        }
+    }
+    if (!decode_grid_barrier(a.bar, 2 * gridDim.x, a.status, &s_ok)) return;
+
+    // ---- C. experts, one task per warp at a time
+    const int nwarps = gridDim.x * kDecodeWarps;
+    for (int m = blockIdx.x * kDecodeWarps + warp; m < a.L * a.K; m += nwarps) {
+        const int t = m / a.K;
+        int64_t e = a.idx[m];
+        const float g = a.gate[m];
+        if (e < 0 || e >= a.N) {
+            set_status(a.status, OMNI_DEV_BAD_EXPERT);
+            e = 0;
+        }
+        const uint4 *x4 = reinterpret_cast<const uint4 *>(a.x) + (size_t)t * d8;
+        const uint4 *w4 = reinterpret_cast<const uint4 *>(a.W) + (size_t)e * d8;
+        const uint4 *v4 = reinterpret_cast<const uint4 *>(a.V) + (size_t)e * d8;
+        uint4 xu[kDecodeSlices], wu[kDecodeSlices], vu[kDecodeSlices];
+#pragma unroll
+        for (int i = 0; i < kDecodeSlices; ++i) {             // every slice in flight at once
+            const int c8 = (int)lane + 32 * i;
+            const bool in = c8 < d8;
+            xu[i] = in ? x4[c8] : make_uint4(0u, 0u, 0u, 0u);
+            wu[i] = in ? w4[c8] : make_uint4(0u, 0u, 0u, 0u);
+            vu[i] = in ? v4[c8] : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < kDecodeSlices; ++i) {
+            const uint32_t xw[4] = {xu[i].x, xu[i].y, xu[i].z, xu[i].w};
+            const uint32_t ww[4] = {wu[i].x, wu[i].y, wu[i].z, wu[i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc = fmaf(__uint_as_float(xw[q] << 16), __uint_as_float(ww[q] << 16), acc);
+                acc = fmaf(__uint_as_float(xw[q] & 0xffff0000u), __uint_as_float(ww[q] & 0xffff0000u),
+                           acc);
+            }
+        }
+        const float h = warp_sum(acc);
+        const float p = g * (h / (1.f + __expf(-h)));
+        float *yr = a.y + (size_t)t * a.d;
+#pragma unroll
+        for (int i = 0; i < kDecodeSlices; ++i) {
+            const int c8 = (int)lane + 32 * i;
+            if (c8 < d8) {
+                const uint32_t vw[4] = {vu[i].x, vu[i].y, vu[i].z, vu[i].w};
+                float f[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    f[2 * q] = p * __uint_as_float(vw[q] << 16);
+                    f[2 * q + 1] = p * __uint_as_float(vw[q] & 0xffff0000u);
+                }
+                red_add_v4(yr + 8 * c8, f[0], f[1], f[2], f[3]);
+                red_add_v4(yr + 8 * c8 + 4, f[4], f[5], f[6], f[7]);
+            }
+        }
+    }
 }
 
 }  // namespace
@@ -972,6 +1192,79 @@ cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const fl
     if (cap <= 576) { OMNI_MG(576) }
     OMNI_MG(1088)
 #undef OMNI_MG
+}
+
+// Shared words of one axis warp of the fused decode step: axis_row_exact's
+// values, two bucket arrays and max(2 kmax, 2 CAP) words of candidates (as
+// the stand-alone axis kernel takes), a multiple of 4.
+static size_t decode_axis_words(int nmax, int kmax) {
+    const size_t area = kmax > kDecodeCap ? 2 * (size_t)kmax : 2 * (size_t)kDecodeCap;
+    const size_t words = (((size_t)nmax + 2 * kNB + 1) & ~(size_t)1) + area;
+    return (words + 3) & ~(size_t)3;
+}
+
+// Shared words of the fused decode step for these sizes (0 if it does not
+// apply): the larger of phase A (x) and phase B (candidate table, two axis
+// warps or the merge warp).
+static size_t decode_smem_bytes(int L, int d, int N_r, int N_c, int K, int Kr, int Kc, int C) {
+    if (L > 16 || K > 128 || d > 32 * 8 * kDecodeSlices || d % 256 != 0) return 0;
+    const int nmax = N_r > N_c ? N_r : N_c;
+    const int kmax = Kr > Kc ? Kr : Kc;
+    const size_t axis_words = decode_axis_words(nmax, kmax);
+    const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
+    const MergeLayout ml = merge_layout(K, Kr, Kc, C, kDecodeCap);
+    const size_t area = 2 * axis_words > ml.words ? 2 * axis_words : ml.words;
+    const size_t b_bytes = 4 * (head + area);
+    const size_t a_bytes = (size_t)L * d * 2;
+    const size_t bytes = a_bytes > b_bytes ? a_bytes : b_bytes;
+    return bytes <= 200 * 1024 ? bytes : 0;
+}
+
+bool decode_fused_ok(int L, int d, int N_r, int N_c, int K, int Kr, int Kc, int C) {
+    return decode_smem_bytes(L, d, N_r, N_c, K, Kr, Kc, C) > 0;
+}
+
+cudaError_t launch_decode_fused(const uint16_t *x, const uint16_t *W, const uint16_t *V,
+                                const uint16_t *W_r, const uint16_t *W_c, int L, int d, int N_r,
+                                int N_c, int K, int Kr, int Kc, int C, float *s_r, float *s_c,
+                                float *row_val, int *row_idx, float *col_val, int *col_idx,
+                                int32_t *idx, float *score, float *gate, float *y,
+                                bool accumulate, unsigned *bar, int *status, cudaStream_t st) {
+    const size_t smem = decode_smem_bytes(L, d, N_r, N_c, K, Kr, Kc, C);
+    if (smem == 0) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel,
+                                                      32 * kDecodeWarps, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm > 2) per_sm = 2;
+    const int grid = device_sm_count() * per_sm;      // every CTA resident (cooperative launch)
+    if (per_sm < 1 || grid < L) return cudaErrorInvalidValue;
+    DecodeArgs a;
+    a.x = x; a.W = W; a.V = V; a.W_r = W_r; a.W_c = W_c;
+    a.L = L; a.d = d; a.N_r = N_r; a.N_c = N_c; a.K = K; a.Kr = Kr; a.Kc = Kc; a.C = C;
+    a.N = (int64_t)N_r * N_c;
+    a.s_r = s_r; a.s_c = s_c; a.row_val = row_val; a.col_val = col_val;
+    a.row_idx = row_idx; a.col_idx = col_idx; a.idx = idx; a.score = score; a.gate = gate;
+    a.y = y; a.accumulate = accumulate ? 1 : 0; a.bar = bar; a.status = status;
+    a.nmax = N_r > N_c ? N_r : N_c;
+    a.kmax = Kr > Kc ? Kr : Kc;
+    a.axis_words = (int)decode_axis_words(a.nmax, a.kmax);
+    a.merge_head = (int)(((size_t)C + Kr + 1 + 3) & ~(size_t)3);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(32 * kDecodeWarps);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    first_launch_in_call();                     // ordinary stream order for what follows it too
+    return cudaLaunchKernelEx(&cfg, decode_fused_kernel, a);
 }
 
 }  // namespace omni

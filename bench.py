@@ -123,8 +123,8 @@ def launches_per_step(cfg) -> int:
     router = 1 + (2 if reg else 1) + 1            # GEMM, axis top-K (+ flagged redo), merge
     p = radix_passes(cfg.G)
     sched = 1 + (p + max(p - 1, 0))               # scan, scatters, histogram scans (the
-    if cfg.L <= 16:                               # per-token step runs in the merge kernel)
-        sched = 0                                 # decode batches run in token order
+    if cfg.L <= 16 and cfg.K <= 128 and cfg.d % 256 == 0 and cfg.d <= 2048:
+        return 1                                  # the fused decode step: one launch
     # the tensor-core expert path (default for L * K * d >= 2^31): expert use,
     # dense marks, column scan, column list, gather, split, two tile GEMMs
     dense = 8 if cfg.L > 16 and cfg.M * cfg.d >= 2 ** 31 else 0
@@ -291,25 +291,29 @@ def run_omni(args, cfg, world, rank, local):
     # ---- small batches are launch-bound: the same step as one CUDA graph
     graph = None
     if L <= GRAPH_MAX_L:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step()
-        for _ in range(3):
-            g.replay()
-        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        barrier(world)
-        torch.cuda.synchronize()
-        for i in range(args.steps):
-            flush.zero_()
-            gev[i][0].record(stream)
-            g.replay()
-            gev[i][1].record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        gms = reduce_max(med_ms(gev), world, dev)
-        graph = {"value": job_throughput(world, L, gms), "unit": "tokens/s", "ms_per_step": gms}
-        del g
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step()
+            for _ in range(3):
+                g.replay()
+            gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            barrier(world)
+            torch.cuda.synchronize()
+            for i in range(args.steps):
+                flush.zero_()
+                gev[i][0].record(stream)
+                g.replay()
+                gev[i][1].record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            gms = reduce_max(med_ms(gev), world, dev)
+            graph = {"value": job_throughput(world, L, gms), "unit": "tokens/s", "ms_per_step": gms}
+            del g
+        except RuntimeError as exc:                   # a step that cannot be captured
+            graph = {"unavailable": str(exc).splitlines()[0]}
+            torch.cuda.synchronize()
 
     # ---- staged loop: the same kernels through the three stage calls, for
     # per-stage times and the grouped-expert kernel's duration
@@ -665,7 +669,7 @@ def timeline(args, cfg):
                   if e.device_type == torch.autograd.DeviceType.CUDA)
     steps, cur = [], None
     for a, b, n in rows:
-        if "router_gemm" in n or "router_small" in n:      # a step's first kernel
+        if "router_gemm" in n or "router_small" in n or "decode_fused" in n:   # a step's first kernel
             cur = []
             steps.append(cur)
         if cur is not None and "omni::" in n:

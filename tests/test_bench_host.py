@@ -23,9 +23,9 @@ def test_launches_per_step_matches_the_profiled_step():
     # the headline step in the committed launch list: GEMM, two axis kernels,
     # merge, scan, two radix scatters, histogram scan, group pass, token pass
     assert bench.launches_per_step(configs.HEADLINE) == 10
-    # decode batches skip the schedule: router (4) + the two expert passes
-    assert bench.launches_per_step(configs.sweep(16)) == 6
-    assert bench.launches_per_step(configs.sweep(1)) == 6
+    # decode batches (L <= 16) run the whole step as one cooperative launch
+    assert bench.launches_per_step(configs.sweep(16)) == 1
+    assert bench.launches_per_step(configs.sweep(1)) == 1
     # the skewed layer adds the tensor-core expert path: 8 launches
     # (use, mark, scan, list, gather, split, two GEMMs); its 8192 groups need
     # two radix passes, like the headline

@@ -382,3 +382,41 @@ def test_routed_bwd_accumulates():
         ref = 2 * host(out[k])
         np.testing.assert_allclose(host(out2[k]), ref, rtol=0,
                                    atol=1e-5 * float(np.abs(ref).max()))
+
+
+# ------------------------------------------------------- fused decode step
+@pytest.mark.parametrize("L,d,N_r,N_c,K", [
+    (1, 2048, 1304, 1304, 64),     # the decode sweep's grid and width
+    (16, 2048, 1304, 1304, 64),
+    (3, 256, 100, 37, 16),         # ragged axes (37: rows not a multiple of 4)
+    (5, 512, 64, 64, 128),         # K = 128 on a small grid (K > N_r)
+    (16, 1024, 512, 512, 128),
+])
+def test_decode_step_against_oracle(L, d, N_r, N_c, K):
+    """L <= 16 runs the whole routed step (projection, selection, gates,
+    token-order expert work) in one cooperative launch: routing against the
+    oracle under the near-tie rule, y on every token against the oracle on
+    the GPU's routing, idx_out / gate_out, and OMNI_Y_ACCUMULATE."""
+    torch.cuda.empty_cache()
+    cfg = configs.LayerConfig("decode", L, d, N_r, N_c, K, 64)
+    t = inputs.make_inputs(cfg, DEV, seed=9)
+    u = {k: host(v) for k, v in t.items() if k in ("x", "W_r", "W_c")}
+    ws = omni.workspace(L, d, N_r, N_c, K, cfg.B)
+    y, idx, gate = omni.routed_fwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], K, cfg.B, ws=ws,
+                                   want_routing=True)
+    assert omni.omni_get_device_status(ws) == 0
+    p_r, p_c = oracle.router_logprobs(u["x"], u["W_r"], u["W_c"])
+    idx_ref, score_ref, _ = oracle.topk_from_logprobs(p_r, p_c, K)
+    check_routing_near_ties(host(idx), idx_ref, score_ref, p_r, p_c, N_c)
+    g = host(gate)
+    np.testing.assert_allclose(g.astype(np.float64).sum(1), 1.0, atol=2e-5)
+    y_ref = oracle_y_rows(t["x"], t["W"], t["V"], idx, gate, np.arange(L))
+    check_y(host(y), y_ref, "decode step")
+    # accumulate adds to what is there
+    base = torch.randn_like(y)
+    y2 = base.clone()
+    omni.routed_fwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], K, cfg.B, y=y2, ws=ws,
+                    accumulate=True)
+    check_y(host(y2), host(base).astype(np.float64) + y_ref, "decode step, accumulate")
+    del t, ws
+    torch.cuda.empty_cache()
