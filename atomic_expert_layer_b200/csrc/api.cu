@@ -99,7 +99,6 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
     }
     if (regions & kRegExpert) {
         w.tok_count = take(4 * L);
-        w.dec_bar = take(4);
     }
     const bool dense = (regions & kRegDense) && sz.dense;
     if (dense) {
@@ -108,6 +107,7 @@ WsLayout make_layout(const Sizes &sz, unsigned regions) {
         w.dz_ccount = take(8);
     }
     w.zero_end = o;
+    if (regions & kRegExpert) w.dec_bar = take(8);      // outside the zeroed prefix
     if (regions & kRegRouter) {
         w.s_r = take(4 * L * sz.N_r);
         w.s_c = take(4 * L * sz.N_c);
@@ -416,20 +416,25 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                        ws, ws_bytes, &lay)))
         return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = reset_workspace(ws, lay, st))) return rc;
+    const bool fused = L <= kTokenOrderMaxL && decode_fused_ok(L, d, N_r, N_c, K, sz.Kr, sz.Kc, sz.C);
+    // the fused step clears its own status word and needs no zeroed counters
+    if (!fused && (rc = reset_workspace(ws, lay, st))) return rc;
     int32_t *idx = ws_at<int32_t>(ws, lay.idx);
     float *score = ws_at<float>(ws, lay.score), *gate = ws_at<float>(ws, lay.gate);
     // scheduled path: the merge kernel also runs the schedule's per-token step;
     // nothing here reads the distinct-expert count, so it is not kept
     SchedPrep prep = sched_prep_of(sz, ws, lay);
     prep.bitmap = nullptr;
-    if (L <= kTokenOrderMaxL && decode_fused_ok(L, d, N_r, N_c, K, sz.Kr, sz.Kc, sz.C)) {
+    if (fused) {
         // a handful of tokens: the whole step in one cooperative launch
+        static std::atomic<unsigned> epochs{0};
+        unsigned epoch = ++epochs;
+        if (epoch == 0) epoch = ++epochs;
         rc = cuda_rc(launch_decode_fused(
             x, W, V, W_r, W_c, L, d, N_r, N_c, K, sz.Kr, sz.Kc, sz.C, ws_at<float>(ws, lay.s_r),
             ws_at<float>(ws, lay.s_c), ws_at<float>(ws, lay.row_val), ws_at<int>(ws, lay.row_idx),
             ws_at<float>(ws, lay.col_val), ws_at<int>(ws, lay.col_idx), idx, score, gate, y,
-            (flags & OMNI_Y_ACCUMULATE) != 0, ws_at<unsigned>(ws, lay.dec_bar),
+            (flags & OMNI_Y_ACCUMULATE) != 0, ws_at<unsigned long long>(ws, lay.dec_bar), epoch,
             ws_at<int>(ws, lay.hdr), st));
         if (rc) return rc;
         if (idx_out && (rc = cuda_rc(cudaMemcpyAsync(idx_out, idx, 4 * (size_t)sz.M,

@@ -27,7 +27,7 @@ struct WsLayout {
     size_t hdr, s_r, s_c, part_r, part_c, flags, row_val, row_idx, col_val, col_idx, idx, score, gate;
     size_t a_tok, a_exp, a_gate, b_tok, b_exp, b_gate, t_tok, t_exp, t_gate;
     size_t g_off, g_cnt, g_act, n_act, n_dist, bitmap, hist, tok_count, tok_slots;
-    size_t dec_bar;          // grid-barrier counter of the fused decode step (zeroed)
+    size_t dec_bar;          // grid-barrier word of the fused decode step (never cleared)
     size_t z_cnt, z_ndist;   // schedule counters (workspace copies)
     // tensor-core expert path: zeroed per call (dz_*), then the rest
     size_t dz_cnt, dz_ghot, dz_ccount;
@@ -105,7 +105,8 @@ cudaError_t launch_decode_fused(const uint16_t *x, const uint16_t *W, const uint
                                 int N_c, int K, int Kr, int Kc, int C, float *s_r, float *s_c,
                                 float *row_val, int *row_idx, float *col_val, int *col_idx,
                                 int32_t *idx, float *score, float *gate, float *y,
-                                bool accumulate, unsigned *bar, int *status, cudaStream_t st);
+                                bool accumulate, unsigned long long *bar, unsigned epoch,
+                                int *status, cudaStream_t st);
 
 // ---- the pages' blockwise grid top-K (alternative to axis + merge); its
 // candidates need L * blockwise_bands(...) * K * 16 bytes at `cand`

@@ -46,13 +46,13 @@ __device__ __forceinline__ void small_rows_dot(const uint4 *xs, const uint16_t *
     uint4 wu[kSmallRows][kSmallSlices];
 #pragma unroll
     for (int r = 0; r < kSmallRows; ++r) {
-        const int g = g0 + r < ntot ? g0 + r : ntot - 1;     // clamped; not written
+        const int g = g0 + r;                            // rows past the end: zeros, not written
         const uint4 *w4 = reinterpret_cast<const uint4 *>(
             g < N_r ? W_r + (size_t)g * d : W_c + (size_t)(g - N_r) * d);
 #pragma unroll
         for (int i = 0; i < kSmallSlices; ++i) {
             const int c8 = (int)lane + 32 * i;
-            wu[r][i] = c8 < d8 ? w4[c8] : make_uint4(0u, 0u, 0u, 0u);
+            wu[r][i] = c8 < d8 && g < ntot ? w4[c8] : make_uint4(0u, 0u, 0u, 0u);
         }
     }
     xs_ready();

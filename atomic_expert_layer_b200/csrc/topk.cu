@@ -191,6 +191,40 @@ __device__ __forceinline__ void bucket_starts(uint32_t *hist, uint32_t *cur) {
     __syncwarp();
 }
 
+// bucket_find and bucket_starts in one pass over the histogram (one warp):
+// the counts become starting positions (written to hist and cur), and the
+// return value / *bstar are those of bucket_find.
+__device__ int bucket_scan(uint32_t *hist, uint32_t *cur, int k, int *bstar) {
+    const unsigned lane = lane_id();
+    constexpr int per = kNB / 32;
+    uint32_t c[per];
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+        c[j] = hist[lane * per + j];
+        tot += (int)c[j];
+    }
+    const int incl = warp_iscan(tot);
+    const int excl = incl - tot;
+    const bool mine = excl < k && k <= incl;
+    const unsigned bal = __ballot_sync(0xffffffffu, mine);
+    int run = excl, bs = 0, through = 0;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+        hist[lane * per + j] = (uint32_t)run;
+        cur[lane * per + j] = (uint32_t)run;
+        run += (int)c[j];
+        if (mine && through == 0 && run >= k) {
+            bs = lane * per + j;
+            through = run;
+        }
+    }
+    if (bal == 0u) return -1;
+    const int src = __ffs(bal) - 1;
+    *bstar = __shfl_sync(0xffffffffu, bs, src);
+    return __shfl_sync(0xffffffffu, through, src);
+}
+
 // ------------------------------------------------------------ axis top-K
 // Dynamic smem per warp (words): vals[nmax] | hist[kNB] | cur[kNB] |
 // area[max(2 kmax, 2 CAP)], where area is either sel_key[kmax] + sel_idx[kmax]
@@ -267,12 +301,21 @@ __device__ void axis_row_exact(const float *__restrict__ in, int n, int kx, int 
         }
         counted = true;
     } else if (logsoftmax) {
-        float mx = -INFINITY;
-        for (int i = lane; i < n; i += 32) {
-            const float v = in[i];
-            vals[i] = v;
-            mx = fmaxf(mx, v);
+        // the row into shared memory with every load in flight (16-byte
+        // vectors when the row allows), then the max over the stored values
+        if ((n & 3) == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0) {
+            const float4 *in4 = reinterpret_cast<const float4 *>(in);
+            float4 *v4 = reinterpret_cast<float4 *>(vals);
+            const int n4 = n >> 2;
+#pragma unroll 8
+            for (int i4 = lane; i4 < n4; i4 += 32) v4[i4] = in4[i4];
+        } else {
+#pragma unroll 8
+            for (int i = lane; i < n; i += 32) vals[i] = in[i];
         }
+        __syncwarp();
+        float mx = -INFINITY;
+        for (int i = lane; i < n; i += 32) mx = fmaxf(mx, vals[i]);
         mx = warp_max(mx);
         float sum = 0.f;
         for (int i = lane; i < n; i += 32) sum += __expf(vals[i] - mx);
@@ -836,23 +879,369 @@ int fast_capacity(int k) {
     return k <= 1024 ? ((k + 64 + 31) / 32) * 32 : 0;
 }
 
+// ------------------------------------------------ block-wide exact selection
+// Used by the fused decode step, where one token's selection is on the
+// critical path: many threads per row instead of one warp.
+
+// Named barrier over `nthreads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Exact radix select of the k largest of the 32-bit keys key(i), i < n, by
+// `nt` threads (thread ht of them, ht < nt) sharing `hist` (kNB words) and
+// `scr` (2 words).  Returns T, the k-th largest key, and sets *take_eq to how
+// many keys equal to T belong to the k largest (every key > T does).
+template <typename KeyOf>
+__device__ uint32_t group_radix_select(KeyOf key_of, int n, int k, int ht, int nt, int bar_id,
+                                       uint32_t *hist, int *scr, int *take_eq) {
+    uint32_t prefix = 0, mask = 0;
+    int krem = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = ht; b < kNB; b += nt) hist[b] = 0u;
+        named_sync(bar_id, nt);
+        // keys that share the prefix crowd a few digits (all log-probabilities
+        // share the top byte): lanes with the same digit add with one atomic
+        for (int i0 = 0; i0 < n; i0 += nt) {
+            const int i = i0 + ht;
+            uint32_t dg = kNB;                                   // no digit
+            if (i < n) {
+                const uint32_t key = key_of(i);
+                if ((key & mask) == prefix) dg = (key >> shift) & 255u;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, dg);
+            if (dg < (uint32_t)kNB && lane_id() == (unsigned)(__ffs(peers) - 1))
+                atomicAdd(&hist[dg], (uint32_t)__popc(peers));
+        }
+        named_sync(bar_id, nt);
+        if (ht < 32) {
+            // lane l owns bins 255-8l down to 248-8l (largest digits first)
+            int c[8], tot = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                c[j] = (int)hist[255 - 8 * ht - j];
+                tot += c[j];
+            }
+            const int incl = warp_iscan(tot);
+            const int excl = incl - tot;
+            const bool mine = excl < krem && krem <= incl;
+            if (mine) {
+                int run = excl;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (run + c[j] >= krem) {
+                        scr[0] = 255 - 8 * ht - j;
+                        scr[1] = run;
+                        break;
+                    }
+                    run += c[j];
+                }
+            }
+        }
+        named_sync(bar_id, nt);
+        const int digit = scr[0], above = scr[1];
+        krem -= above;
+        prefix |= (uint32_t)digit << shift;
+        mask |= 255u << shift;
+        named_sync(bar_id, nt);                      // scr is rewritten by the next pass
+    }
+    *take_eq = krem;
+    return prefix;
+}
+
+// Sum / max of one float per thread over nt threads (warp-level, then
+// through `red` (nt / 32 floats)).
+__device__ __forceinline__ float group_sum(float v, int ht, int nt, int bar_id, float *red) {
+    v = warp_sum(v);
+    if ((ht & 31) == 0) red[ht >> 5] = v;
+    named_sync(bar_id, nt);
+    float t = 0.f;
+    for (int w = 0; w < nt / 32; ++w) t += red[w];
+    named_sync(bar_id, nt);
+    return t;
+}
+__device__ __forceinline__ float group_max(float v, int ht, int nt, int bar_id, float *red) {
+    v = warp_max(v);
+    if ((ht & 31) == 0) red[ht >> 5] = v;
+    named_sync(bar_id, nt);
+    float t = -INFINITY;
+    for (int w = 0; w < nt / 32; ++w) t = fmaxf(t, red[w]);
+    named_sync(bar_id, nt);
+    return t;
+}
+
+// One (token, axis) row by nt threads: p = s - logsumexp(s), and the kx best
+// by (p desc, index asc) into oval / oidx in that order.  The block-wide
+// form of the warp's bucket counting sort: p is counted into value buckets
+// below the row maximum, the bucket b* that holds the kx-th value is found,
+// the candidates (buckets <= b*) are scattered to their bucket's range and
+// each is ranked among its bucket peers only.  When more than tmp_cap values
+// fall in those buckets (or fewer than kx in range), an exact radix select
+// takes over.  Shared: vals (n words), hist, cur (kNB each), tmp
+// (max(tmp_cap, kx) 64-bit keys), scr (8 words).
+__device__ void group_axis_select(const float *__restrict__ in, int n, int kx, int ht, int nt,
+                                  int bar_id, float *vals, uint32_t *hist, uint32_t *cur,
+                                  uint64_t *tmp, int tmp_cap, int *scr, float *oval, int *oidx) {
+    float *red = reinterpret_cast<float *>(scr + 2);
+    for (int b = ht; b < kNB; b += nt) hist[b] = 0u;
+    // the row with every load in flight, its maximum
+    float mx = -INFINITY;
+    if ((n & 3) == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0) {
+        const float4 *in4 = reinterpret_cast<const float4 *>(in);
+        float4 *v4 = reinterpret_cast<float4 *>(vals);
+#pragma unroll 4
+        for (int i4 = ht; i4 < (n >> 2); i4 += nt) {
+            const float4 v = in4[i4];
+            v4[i4] = v;
+            mx = fmaxf(fmaxf(mx, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
+        }
+    } else {
+#pragma unroll 4
+        for (int i = ht; i < n; i += nt) {
+            const float v = in[i];
+            vals[i] = v;
+            mx = fmaxf(mx, v);
+        }
+    }
+    mx = group_max(mx, ht, nt, bar_id, red);
+    float sm_ = 0.f;
+    for (int i = ht; i < n; i += nt) sm_ += __expf(vals[i] - mx);
+    const float lse = mx + __logf(group_sum(sm_, ht, nt, bar_id, red));
+    const float vmax = mx - lse;                 // the p of the largest logit, same rounding
+    for (int i = ht; i < n; i += nt) {
+        const float p = vals[i] - lse;
+        vals[i] = p;
+        const int b = bucket_of(vmax, p);
+        if (b < kNB) atomicAdd(&hist[b], 1u);
+    }
+    named_sync(bar_id, nt);
+    if (ht < 32) {                               // the group's first warp
+        int bs = 0;
+        const int nc = bucket_scan(hist, cur, kx, &bs);
+        const bool fast = nc >= kx && nc <= tmp_cap;
+        if (ht == 0) {
+            scr[0] = fast ? nc : -1;
+            scr[1] = bs;
+        }
+    }
+    named_sync(bar_id, nt);
+    const int ncand = scr[0], bstar = scr[1];
+    if (ncand >= 0) {
+        for (int i = ht; i < n; i += nt) {
+            const float p = vals[i];
+            const int b = bucket_of(vmax, p);
+            if (b <= bstar)
+                tmp[atomicAdd(&cur[b], 1u)] =
+                    ((uint64_t)f2key(p) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
+        }
+        named_sync(bar_id, nt);
+        for (int pos = ht; pos < ncand; pos += nt) {
+            const uint64_t k = tmp[pos];
+            const float p = key2f((uint32_t)(k >> 32));
+            const int b = bucket_of(vmax, p);
+            const int s0 = (int)hist[b], s1 = b < bstar ? (int)hist[b + 1] : ncand;
+            int r = 0;
+            for (int q = s0; q < s1; ++q) r += tmp[q] > k ? 1 : 0;
+            if (s0 + r < kx) {
+                oval[s0 + r] = p;
+                oidx[s0 + r] = (int)(0xffffffffu - (uint32_t)k);
+            }
+        }
+        named_sync(bar_id, nt);
+        return;
+    }
+
+    // ---- exact fallback: radix select on the keys of p
+    for (int i = ht; i < n; i += nt) vals[i] = __uint_as_float(f2key(vals[i]));
+    named_sync(bar_id, nt);
+    auto key_of = [&](int i) { return __float_as_uint(vals[i]); };
+    int take_eq;
+    const uint32_t T = group_radix_select(key_of, n, kx, ht, nt, bar_id, hist, scr, &take_eq);
+    // keys equal to T: the take_eq smallest indices (by radix select on the
+    // inverted index among them, when there are more)
+    int n_eq = 0;
+    for (int i = ht; i < n; i += nt) n_eq += key_of(i) == T ? 1 : 0;
+    n_eq = (int)group_sum((float)n_eq, ht, nt, bar_id, red);
+    uint32_t Tl = 0u;
+    if (n_eq > take_eq) {
+        int tl_eq;
+        Tl = group_radix_select([&](int i) { return key_of(i) == T ? 0xffffffffu - (uint32_t)i : 0u; },
+                                n, take_eq, ht, nt, bar_id, hist, scr, &tl_eq);
+    }
+    // compact the kx selected (64-bit keys: p key, inverted index), one
+    // atomic per warp and round
+    if (ht == 0) scr[0] = 0;
+    named_sync(bar_id, nt);
+    for (int i0 = 0; i0 < n; i0 += nt) {
+        const int i = i0 + ht;
+        bool take = false;
+        uint32_t key = 0u, lo = 0u;
+        if (i < n) {
+            key = key_of(i);
+            lo = 0xffffffffu - (uint32_t)i;
+            take = key > T || (key == T && (n_eq == take_eq || lo >= Tl));
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        int base = 0;
+        if (bal && lane_id() == 0) base = atomicAdd(&scr[0], __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (take) {
+            const int at = base + __popc(bal & lanemask_lt());
+            if (at < kx) tmp[at] = ((uint64_t)key << 32) | lo;
+        }
+    }
+    named_sync(bar_id, nt);
+    // rank sort (keys are distinct)
+    for (int j = ht; j < kx; j += nt) {
+        const uint64_t kj = tmp[j];
+        int r = 0;
+        for (int i = 0; i < kx; ++i) r += tmp[i] > kj;
+        oval[r] = key2f((uint32_t)(kj >> 32));
+        oidx[r] = (int)(0xffffffffu - (uint32_t)kj);
+    }
+    named_sync(bar_id, nt);
+}
+
+// Shared words of the block-wide merge (group_merge) ahead of its candidate
+// keys: hist, cur, the dense ranks of the row and column lists (128 each),
+// 16 words of scratch, out_S and out_n (K each); even, so that the 64-bit
+// keys that follow are aligned.
+__host__ __device__ inline int group_merge_head_words(int K) {
+    return (2 * kNB + 256 + 16 + 2 * K + 1) & ~1;
+}
+
+// The merge of one token by the whole CTA (256 threads): the global top-K of
+// S = fl32(p_r[a] + p_c[b]) over the candidate cells (a, b) of `table`,
+// ranked by (S desc, p_r desc, p_c desc, n asc), and the gates.  Kr, Kc <=
+// 128.  Every cell gets one unique 64-bit key that encodes the whole rule:
+// the key of S, then (dr[a], dc[b], a, b) ascending, where dr / dc are the
+// dense ranks of the row / column list (equal p share a rank; the lists are
+// in (p desc, index asc) order, so among equal p a smaller list position is
+// a smaller index, and (a, b) ascending is n ascending).  The K largest keys
+// are found by the bucket counting sort on S below S(0, 0) (every cell
+// ranked among its bucket peers), or, when fewer than K cells are in range,
+// by ranking every cell against all C.  rv / ri, cv / ci: the token's row and
+// column top-K (shared); `work`: group_merge_head_words(K) + 2 C words.
+__device__ void group_merge(const uint32_t *table, const float *rv, const int *ri, const float *cv,
+                            const int *ci, int N_c, int K, int Kr, int Kc, int C, uint32_t *work,
+                            int32_t *idx, float *score, float *gate) {
+    const int ht = threadIdx.x, nt = blockDim.x;
+    const unsigned lane = lane_id();
+    const int warp = ht >> 5;
+    uint32_t *hist = work, *cur = work + kNB;
+    uint32_t *dr = cur + kNB, *dc = dr + 128;
+    int *scr = reinterpret_cast<int *>(dc + 128);
+    float *out_S = reinterpret_cast<float *>(scr + 16);
+    uint32_t *out_n = reinterpret_cast<uint32_t *>(out_S + K);
+    uint64_t *ckey = reinterpret_cast<uint64_t *>(work + group_merge_head_words(K));
+
+    for (int b = ht; b < kNB; b += nt) hist[b] = 0u;
+    // dense ranks: warps 0-3 the row list, warps 4-7 the column list
+    const bool colw = ht >= 128;
+    const int pos = ht & 127;
+    const int nl = colw ? Kc : Kr;
+    const float *lv = colw ? cv : rv;
+    const bool flag = pos > 0 && pos < nl && f2key(lv[pos]) != f2key(lv[pos - 1]);
+    const unsigned bal = __ballot_sync(0xffffffffu, flag);
+    if (lane == 0) scr[warp] = __popc(bal);
+    const float smax = __fadd_rn(rv[0], cv[0]);          // cell (0, 0) is the largest
+    __syncthreads();
+    {
+        int before = 0;
+        for (int w = colw ? 4 : 0; w < warp; ++w) before += scr[w];
+        if (pos < nl) (colw ? dc : dr)[pos] = (uint32_t)(before + __popc(bal & lanemask_lt()) + (flag ? 1 : 0));
+    }
+    for (int c = ht; c < C; c += nt) {
+        const uint32_t ab = table[c];
+        const int b = bucket_of(smax, __fadd_rn(rv[ab >> 16], cv[ab & 0xffffu]));
+        if (b < kNB) atomicAdd(&hist[b], 1u);
+    }
+    __syncthreads();
+    if (ht < 32) {
+        int bs = 0;
+        const int nc = bucket_scan(hist, cur, K, &bs);
+        const bool fast = nc >= K;
+        if (ht == 0) {
+            scr[8] = fast ? nc : -1;
+            scr[9] = bs;
+        }
+    }
+    __syncthreads();
+    const int ncand = scr[8], bstar = scr[9];
+    auto key_of = [&](uint32_t ab, float S) {
+        const uint32_t a = ab >> 16, b = ab & 0xffffu;
+        const uint32_t sec = (dr[a] << 24) | (dc[b] << 16) | (a << 8) | b;
+        return ((uint64_t)f2key(S) << 32) | (uint64_t)(0xffffffffu - sec);
+    };
+    auto emit = [&](int at, uint64_t k) {
+        const uint32_t sec = 0xffffffffu - (uint32_t)k;
+        out_S[at] = key2f((uint32_t)(k >> 32));
+        out_n[at] = (uint32_t)ri[(sec >> 8) & 255u] * (uint32_t)N_c + (uint32_t)ci[sec & 255u];
+    };
+    if (ncand >= 0) {
+        for (int c = ht; c < C; c += nt) {
+            const uint32_t ab = table[c];
+            const float S = __fadd_rn(rv[ab >> 16], cv[ab & 0xffffu]);
+            const int b = bucket_of(smax, S);
+            if (b <= bstar) ckey[atomicAdd(&cur[b], 1u)] = key_of(ab, S);
+        }
+        __syncthreads();
+        for (int j = ht; j < ncand; j += nt) {
+            const uint64_t k = ckey[j];
+            const int b = bucket_of(smax, key2f((uint32_t)(k >> 32)));
+            const int s0 = (int)hist[b], s1 = b < bstar ? (int)hist[b + 1] : ncand;
+            int r = 0;
+            for (int q = s0; q < s1; ++q) r += ckey[q] > k ? 1 : 0;
+            if (s0 + r < K) emit(s0 + r, k);
+        }
+    } else {
+        for (int c = ht; c < C; c += nt) {
+            const uint32_t ab = table[c];
+            ckey[c] = key_of(ab, __fadd_rn(rv[ab >> 16], cv[ab & 0xffffu]));
+        }
+        __syncthreads();
+        for (int j = ht; j < C; j += nt) {
+            const uint64_t k = ckey[j];
+            int r = 0;
+            for (int q = 0; q < C; ++q) r += ckey[q] > k ? 1 : 0;
+            if (r < K) emit(r, k);
+        }
+    }
+    __syncthreads();
+    // gates: softmax over the K selected S (out_S[0] is the max)
+    if (ht < 32) {
+        const float smx = out_S[0];
+        float part = 0.f;
+        for (int k = ht; k < K; k += 32) part += expf(out_S[k] - smx);
+        const float den = warp_sum(part);
+        for (int k = ht; k < K; k += 32) {
+            const float S = out_S[k];
+            idx[k] = (int32_t)out_n[k];
+            score[k] = S;
+            gate[k] = expf(S - smx) / den;
+        }
+    }
+}
+
 // ------------------------------------------------------- fused decode step
 // For a handful of tokens the routed forward is latency-bound: six dependent
-// launches, each starting cold, cost about 37 us at L = 1 against a 1.7 us
+// launches, each starting cold, cost about 34 us at L = 1 against a 1.7 us
 // roofline.  Tokens are independent once the router projection is done, so
 // one cooperative launch (every CTA resident) runs the whole step in three
 // phases separated by a grid barrier (a bounded wait):
 //   A. all CTAs: the streamed router projection (small_rows_dot, the
 //      arithmetic of the small-batch projection kernel) into s; y zeroed
-//      unless accumulating;
-//   B. CTA t < L, token t: LogSoftmax and the exact row and column top-K
-//      (warps 0 and 1, axis_row_exact), then the merge and the gates (warp 0,
-//      merge_token): the same selection as the separate kernels;
-//   C. every warp, one task (t, k) at a time in token order: h = x_t . w_e,
-//      p = g SiLU(h), y_t += p v_e (16-byte fp32 reductions; the order in
-//      which a token's K terms land varies from run to run).
+//      unless accumulating; the CTAs that select build the merge's
+//      candidate table;
+//   B. CTA gridDim.x - 1 - t, token t: LogSoftmax and the exact row and
+//      column top-K (128 threads per axis, group_axis_select), then the
+//      merge and the gates (the whole CTA, group_merge): the selection of
+//      the separate kernels, with the same ranking rule and results;
+//   C. chunks of up to 8 tasks of one token per CTA: h = x_t . w_e,
+//      p = g SiLU(h) per warp, the chunk's sum of p v_e per CTA, added to
+//      y_t with 16-byte fp32 reductions (the order in which a token's chunks
+//      land varies from run to run).
 constexpr int kDecodeWarps = 8;
-constexpr int kDecodeCap = 192;            // axis and merge fast-path capacity (K <= 128)
 constexpr int kDecodeSlices = 8;           // 8-wide slices per lane: d <= 2048
 
 struct DecodeArgs {
@@ -866,32 +1255,55 @@ struct DecodeArgs {
     float *score, *gate;
     float *y;
     int accumulate;
-    unsigned *bar;                         // zeroed per call
+    unsigned long long *bar;               // grid barrier: (epoch << 32) | arrivals
+    unsigned epoch;                        // this call's tag, never 0, differs from the last call's
+    int rpc;                               // router rows per projecting CTA
+    int nproj;                             // projecting CTAs (the first ones)
     int *status;
     int nmax, kmax;
     int axis_words;                        // shared words per axis warp
     int merge_head;                        // candidate table and its scratch
+    int list_words;                        // the token's row and column top-K (values, indices)
+    int nmax_pad;                          // nmax rounded up to an even word count
+    int tmp_cap;                           // candidates of the axis bucket sort
 };
 
 // All CTAs of the grid arrive; the wait gives up after kWaitLimitNs and
-// records OMNI_DEV_WAIT_TIMEOUT (then the CTA returns).
-__device__ bool decode_grid_barrier(unsigned *bar, unsigned target, int *status, int *s_ok) {
+// records OMNI_DEV_WAIT_TIMEOUT (then the CTA returns).  The barrier word
+// holds (epoch << 32) | arrivals and needs no clearing between calls: CTA 0
+// installs (epoch, 0) with one exchange when the kernel starts, and an
+// arrival that finds another call's epoch (it came before the exchange,
+// which erased it) arrives again once the epoch is there.  Barrier k of the
+// call completes at k * gridDim.x arrivals.
+__device__ bool decode_grid_barrier(unsigned long long *bar, unsigned epoch, unsigned target,
+                                    int *status, int *s_ok) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        atomicAdd(bar, 1u);
+        bool counted = (unsigned)(atomicAdd(bar, 1ull) >> 32) == epoch;
         bool ok = true;
         const uint64_t t0 = global_timer_ns();
+        // relaxed polls with a short back-off, one acquire fence at the end
         for (uint32_t it = 0;; ++it) {
-            unsigned v;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-            if (v >= target) break;
+            unsigned long long w;
+            asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(bar) : "memory");
+            if ((unsigned)(w >> 32) == epoch) {
+                if (!counted) {
+                    counted = (unsigned)(atomicAdd(bar, 1ull) >> 32) == epoch;
+                    continue;
+                }
+                if ((unsigned)w >= target) {
+                    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+                    break;
+                }
+            }
             if ((it & 63u) == 63u &&
                 (it > kWaitSpinLimit || global_timer_ns() - t0 > kWaitLimitNs)) {
                 set_status(status, OMNI_DEV_WAIT_TIMEOUT);
                 ok = false;
                 break;
             }
+            __nanosleep(32);
         }
         *s_ok = ok ? 1 : 0;
     }
@@ -899,39 +1311,217 @@ __device__ bool decode_grid_barrier(unsigned *bar, unsigned target, int *status,
     return *s_ok != 0;
 }
 
+// One 1-D bulk copy global -> this CTA's shared memory, completing on `bar`
+// (16-byte aligned addresses, a multiple of 16 bytes).
+__device__ __forceinline__ void bulk_load_1d(void *dst, const void *src, uint32_t bytes,
+                                             uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// The projection of the CTA's nrow staged router rows with L staged token
+// rows on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+// 16-row tiles of the block by 8-token tiles, the K = d loop split over the
+// CTA's 8 warps, the warps' partial tiles summed through `red` (8 x 16 x 16
+// floats of shared memory).  Rows and tokens past the end read the last
+// staged one and their results are dropped.  A 10-row block is far below
+// the 64-row minimum of a tcgen05 tile, and the warp-level instruction keeps
+// the code short, which matters for a kernel fetched cold once per step.
+__device__ void decode_rows_mma(const uint16_t *xs, const uint16_t *wsm, int nrow, int g0,
+                                float *red, const DecodeArgs &a) {
+    const int warp = threadIdx.x >> 5;
+    const unsigned lane = lane_id();
+    const int kw = a.d / kDecodeWarps;                       // this warp's K range
+    const int k_lo = warp * kw;
+    const int ntile = (a.L + 7) >> 3;
+    for (int m0 = 0; m0 < nrow; m0 += 16) {
+        float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // ldmatrix row addresses: A rows m0 + (lane % 16), B tokens lane % 8
+        const int ar = min(m0 + (int)(lane & 15u), nrow - 1);
+        const uint32_t a_base = smem_u32(wsm + (size_t)ar * a.d + k_lo + ((lane >> 4) << 3));
+        uint32_t b_base[2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int bt = min(nt * 8 + (int)(lane & 7u), a.L - 1);
+            b_base[nt] = smem_u32(xs + (size_t)bt * a.d + k_lo + (((lane >> 3) & 1u) << 3));
+        }
+#pragma unroll 4
+        for (int k = 0; k < kw; k += 16) {
+            uint32_t fa[4];
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(fa[0]), "=r"(fa[1]), "=r"(fa[2]), "=r"(fa[3])
+                         : "r"(a_base + 2u * k));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                if (nt < ntile) {
+                    uint32_t fb[2];
+                    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+                                 : "=r"(fb[0]), "=r"(fb[1]) : "r"(b_base[nt] + 2u * k));
+                    asm volatile(
+                        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+                        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                        : "+f"(c[nt][0]), "+f"(c[nt][1]), "+f"(c[nt][2]), "+f"(c[nt][3])
+                        : "r"(fa[0]), "r"(fa[1]), "r"(fa[2]), "r"(fa[3]), "r"(fb[0]), "r"(fb[1]));
+                }
+            }
+        }
+        // partial tiles -> red[warp][row][token]; then one (row, token) per thread
+        float *rw = red + warp * 256;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int col = nt * 8 + (int)(lane & 3u) * 2;
+            const int row = (int)(lane >> 2);
+            rw[row * 16 + col] = c[nt][0];
+            rw[row * 16 + col + 1] = c[nt][1];
+            rw[(row + 8) * 16 + col] = c[nt][2];
+            rw[(row + 8) * 16 + col + 1] = c[nt][3];
+        }
+        __syncthreads();
+        {
+            const int row = threadIdx.x >> 4, t = threadIdx.x & 15;
+            if (m0 + row < nrow && t < a.L) {
+                float v = 0.f;
+#pragma unroll
+                for (int w = 0; w < kDecodeWarps; ++w) v += red[w * 256 + threadIdx.x];
+                const int g = g0 + m0 + row;
+                if (g < a.N_r) a.s_r[(size_t)t * a.N_r + g] = v;
+                else a.s_c[(size_t)t * a.N_c + (g - a.N_r)] = v;
+            }
+        }
+        __syncthreads();                                    // red is rewritten next
+    }
+}
+
+// The projection of two staged router rows (j0, j0 + 1 of the CTA's block,
+// bf16 [rows][d] in shared memory) with the L <= LM staged token rows:
+// every slice of both rows in registers, each (row, token) dot product
+// reduced over the warp and written to s_r / s_c at grid row g0 + j.  LM is
+// the token count rounded up to a power of two: the token loop is unrolled
+// LM times, and guarded lanes of it still cost issue slots.
+template <int LM>
+__device__ __forceinline__ void decode_rows_dot2(const uint4 *xs, const uint4 *wsm, int j0,
+                                                 int nrow, int g0, const DecodeArgs &a) {
+    const int d8 = a.d >> 3;
+    const unsigned lane = lane_id();
+    uint4 wu[2][kSmallSlices];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int i = 0; i < kSmallSlices; ++i) {
+            const int c8 = (int)lane + 32 * i;
+            wu[r][i] = c8 < d8 && j0 + r < nrow ? wsm[(size_t)(j0 + r) * d8 + c8]
+                                                : make_uint4(0u, 0u, 0u, 0u);
+        }
+    float acc[2][LM];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int t = 0; t < LM; ++t) acc[r][t] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSmallSlices; ++i) {
+        const int c8 = (int)lane + 32 * i;
+        if (c8 < d8) {
+            float wf[2][8];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t w4[4] = {wu[r][i].x, wu[r][i].y, wu[r][i].z, wu[r][i].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    wf[r][2 * q] = __uint_as_float(w4[q] << 16);
+                    wf[r][2 * q + 1] = __uint_as_float(w4[q] & 0xffff0000u);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < LM; ++t) {
+                if (t < a.L) {
+                    const uint4 u = xs[(size_t)t * d8 + c8];
+                    const uint32_t x4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float xlo = __uint_as_float(x4[q] << 16);
+                        const float xhi = __uint_as_float(x4[q] & 0xffff0000u);
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            acc[r][t] = fmaf(xlo, wf[r][2 * q], acc[r][t]);
+                            acc[r][t] = fmaf(xhi, wf[r][2 * q + 1], acc[r][t]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int g = g0 + j0 + r;
+#pragma unroll
+        for (int t = 0; t < LM; ++t) {
+            if (t < a.L) {
+                const float v = warp_sum(acc[r][t]);
+                if (lane == 0 && j0 + r < nrow) {
+                    if (g < a.N_r) a.s_r[(size_t)t * a.N_r + g] = v;
+                    else a.s_c[(size_t)t * a.N_c + (g - a.N_r)] = v;
+                }
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
                  ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
-__global__ void __launch_bounds__(32 * kDecodeWarps) decode_fused_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(32 * kDecodeWarps, 2) decode_fused_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem_u[];
     __shared__ int s_ok;
     const int warp = threadIdx.x >> 5;
     const unsigned lane = lane_id();
     const int d8 = a.d >> 3;
 
-    // ---- A. router projection; y zeroed
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        atomicExch(a.bar, (unsigned long long)a.epoch << 32);     // this call's barrier word
+        *a.status = 0;                                               // no error can precede it
+    }
+
+    // ---- A. router projection: CTA b < nproj takes rows [b rpc, (b + 1) rpc)
+    // of (W_r; W_c); one bulk copy per matrix pulls them, and another the
+    // token rows, into shared memory; each warp then takes two rows at a
+    // time.  y zeroed unless accumulating.
     {
-        uint4 *xs = reinterpret_cast<uint4 *>(smem_u);            // [L][d / 8]
-        const int nblk = (a.N_r + a.N_c + kSmallRows - 1) / kSmallRows;
-        bool staged = false;
-        for (int blk0 = blockIdx.x * kDecodeWarps; blk0 < nblk;
-             blk0 += gridDim.x * kDecodeWarps) {                    // the same in every warp
-            small_rows_dot<16>(xs, a.W_r, a.W_c, a.L, a.d, a.N_r, a.N_c,
-                               (blk0 + warp) * kSmallRows, a.s_r, a.s_c, [&]() {
-                if (!staged) {
-                    for (int i = threadIdx.x; i < a.L * d8; i += blockDim.x)
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-                                     ::"r"(smem_u32(xs + i)),
-                                     "l"(reinterpret_cast<const uint4 *>(a.x) + i)
-                                     : "memory");
-                    asm volatile("cp.async.commit_group;" ::: "memory");
-                    asm volatile("cp.async.wait_group 0;" ::: "memory");
-                    __syncthreads();
-                    staged = true;
+        const int R = a.N_r + a.N_c;
+        const int r0 = (int)blockIdx.x * a.rpc;
+        const int nrow = (int)blockIdx.x < a.nproj ? min(a.rpc, R - r0) : 0;
+        if (nrow > 0) {
+            uint4 *xs = reinterpret_cast<uint4 *>(smem_u);                      // [L][d / 8]
+            uint4 *wsm = xs + (size_t)a.L * d8;                                 // [rpc][d / 8]
+            uint64_t *mb = reinterpret_cast<uint64_t *>(wsm + (size_t)a.rpc * d8);
+            if (threadIdx.x == 0) {
+                mbar_init(mb, 1);
+                fence_barrier_init();
+                const uint32_t row_bytes = (uint32_t)a.d * 2u;
+                const int nr = min(max(a.N_r - r0, 0), nrow);                  // rows of W_r
+                mbar_arrive_expect_tx(mb, (uint32_t)a.L * row_bytes + (uint32_t)nrow * row_bytes);
+                bulk_load_1d(xs, a.x, (uint32_t)a.L * row_bytes, mb);
+                if (nr > 0) bulk_load_1d(wsm, a.W_r + (size_t)r0 * a.d, (uint32_t)nr * row_bytes, mb);
+                if (nrow > nr)
+                    bulk_load_1d(wsm + (size_t)nr * d8, a.W_c + (size_t)(r0 + nr - a.N_r) * a.d,
+                                 (uint32_t)(nrow - nr) * row_bytes, mb);
+            }
+            __syncthreads();
+            mbar_wait(mb, 0u, a.status);
+            if (a.L <= 2) {
+                for (int j0 = 2 * warp; j0 < nrow; j0 += 2 * kDecodeWarps) {
+                    if (a.L == 1) decode_rows_dot2<1>(xs, wsm, j0, nrow, r0, a);
+                    else decode_rows_dot2<2>(xs, wsm, j0, nrow, r0, a);
                 }
-            });
+            } else {
+                decode_rows_mma(reinterpret_cast<const uint16_t *>(xs),
+                                reinterpret_cast<const uint16_t *>(wsm), nrow, r0,
+                                reinterpret_cast<float *>(mb + 2), a);
+            }
+            __syncthreads();
+            if (threadIdx.x == 0)
+                asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(mb)) : "memory");
         }
         if (!a.accumulate) {
             float4 *y4 = reinterpret_cast<float4 *>(a.y);
@@ -940,88 +1530,113 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_fused_kernel(const D
                 y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
-    if (!decode_grid_barrier(a.bar, gridDim.x, a.status, &s_ok)) return;
+    // the candidate table of the merge, built while the projection finishes
+    // elsewhere (the staged x is no longer read)
+    const int t_sel = (int)gridDim.x - 1 - (int)blockIdx.x < a.L ? (int)gridDim.x - 1 - (int)blockIdx.x : -1;
+    if (t_sel >= 0) {
+        __syncthreads();
+        merge_table(a.K, a.Kr, a.Kc, a.C, smem_u, reinterpret_cast<int *>(smem_u + a.C));
+    }
+    if (!decode_grid_barrier(a.bar, a.epoch, gridDim.x, a.status, &s_ok)) return;
 
-    // ---- B. selection of token t = blockIdx.x
-    if ((int)blockIdx.x < a.L) {
-        const int t = blockIdx.x;
-        uint32_t *table = smem_u;
-        merge_table(a.K, a.Kr, a.Kc, a.C, table, reinterpret_cast<int *>(table + a.C));
-        uint32_t *area = smem_u + a.merge_head;
-        if (warp < 2) {
-            const int axis = warp;
+    // ---- B. selection of token t = gridDim.x - 1 - blockIdx.x (the last
+    // CTAs, which the projection reaches last): warps 0-3 the row axis and
+    // warps 4-7 the column axis (named barriers 1 and 2), then the whole CTA
+    // the merge; the row and column top-K pass through shared memory
+    if (t_sel >= 0) {
+        const int t = t_sel;
+        const uint32_t *table = smem_u;
+        float *lists_v = reinterpret_cast<float *>(smem_u + a.merge_head);       // [Kr + Kc]
+        int *lists_i = reinterpret_cast<int *>(lists_v + a.Kr + a.Kc);          // [Kr + Kc]
+        uint32_t *area = smem_u + a.merge_head + a.list_words;
+        {
+            const int axis = threadIdx.x >> 7;                               // 128 threads each
             const int n = axis ? a.N_c : a.N_r;
             const int kx = axis ? a.Kc : a.Kr;
-            axis_row_exact<kDecodeCap>((axis ? a.s_c : a.s_r) + (size_t)t * n, n, kx, 1, nullptr, t,
-                                       nullptr, (axis ? a.col_val : a.row_val) + (size_t)t * kx,
-                                       (axis ? a.col_idx : a.row_idx) + (size_t)t * kx, a.nmax,
-                                       a.kmax, area + (size_t)axis * a.axis_words);
+            uint32_t *h = area + (size_t)axis * a.axis_words;
+            uint32_t *hist = h + a.nmax_pad;
+            group_axis_select((axis ? a.s_c : a.s_r) + (size_t)t * n, n, kx, threadIdx.x & 127, 128,
+                              1 + axis, reinterpret_cast<float *>(h), hist, hist + kNB,
+                              reinterpret_cast<uint64_t *>(hist + 2 * kNB + 8), a.tmp_cap,
+                              reinterpret_cast<int *>(hist + 2 * kNB),
+                              lists_v + (axis ? a.Kr : 0), lists_i + (axis ? a.Kr : 0));
         }
         __syncthreads();
-        if (warp == 0) {
-            const MergeLayout ml = merge_layout(a.K, a.Kr, a.Kc, a.C, kDecodeCap);
-            const SchedPrep none{};
-            merge_token<kDecodeCap>(table, area, ml, a.row_val + (size_t)t * a.Kr,
-                                    a.row_idx + (size_t)t * a.Kr, a.col_val + (size_t)t * a.Kc,
-                                    a.col_idx + (size_t)t * a.Kc, a.N_c, a.K, a.Kr, a.Kc, a.C, t,
-                                    a.idx + (size_t)t * a.K, a.score + (size_t)t * a.K,
-                                    a.gate + (size_t)t * a.K, none);
-        }
+        group_merge(table, lists_v, lists_i, lists_v + a.Kr, lists_i + a.Kr, a.N_c, a.K, a.Kr, a.Kc,
+                    a.C, area, a.idx + (size_t)t * a.K, a.score + (size_t)t * a.K,
+                    a.gate + (size_t)t * a.K);
     }
-    if (!decode_grid_barrier(a.bar, 2 * gridDim.x, a.status, &s_ok)) return;
+    if (!decode_grid_barrier(a.bar, a.epoch, 2 * gridDim.x, a.status, &s_ok)) return;
 
-    // ---- C. experts, one task per warp at a time
-    const int nwarps = gridDim.x * kDecodeWarps;
-    for (int m = blockIdx.x * kDecodeWarps + warp; m < a.L * a.K; m += nwarps) {
-        const int t = m / a.K;
-        int64_t e = a.idx[m];
-        const float g = a.gate[m];
-        if (e < 0 || e >= a.N) {
-            set_status(a.status, OMNI_DEV_BAD_EXPERT);
-            e = 0;
-        }
-        const uint4 *x4 = reinterpret_cast<const uint4 *>(a.x) + (size_t)t * d8;
-        const uint4 *w4 = reinterpret_cast<const uint4 *>(a.W) + (size_t)e * d8;
-        const uint4 *v4 = reinterpret_cast<const uint4 *>(a.V) + (size_t)e * d8;
-        uint4 xu[kDecodeSlices], wu[kDecodeSlices], vu[kDecodeSlices];
-#pragma unroll
-        for (int i = 0; i < kDecodeSlices; ++i) {             // every slice in flight at once
-            const int c8 = (int)lane + 32 * i;
-            const bool in = c8 < d8;
-            xu[i] = in ? x4[c8] : make_uint4(0u, 0u, 0u, 0u);
-            wu[i] = in ? w4[c8] : make_uint4(0u, 0u, 0u, 0u);
-            vu[i] = in ? v4[c8] : make_uint4(0u, 0u, 0u, 0u);
-        }
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < kDecodeSlices; ++i) {
-            const uint32_t xw[4] = {xu[i].x, xu[i].y, xu[i].z, xu[i].w};
-            const uint32_t ww[4] = {wu[i].x, wu[i].y, wu[i].z, wu[i].w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                acc = fmaf(__uint_as_float(xw[q] << 16), __uint_as_float(ww[q] << 16), acc);
-                acc = fmaf(__uint_as_float(xw[q] & 0xffff0000u), __uint_as_float(ww[q] & 0xffff0000u),
-                           acc);
+    // ---- C. experts: CTA b takes chunks of up to 8 tasks of one token
+    // (chunk j of token t: tasks 8 j .. 8 j + 7), one per warp; each warp
+    // stages its v_e row (bf16) and p = g SiLU(x_t . w_e) in shared memory,
+    // then every thread sums the chunk's p v_e over its 8 columns and adds
+    // them to y_t (16-byte fp32 reductions, one per 4 columns and chunk)
+    uint4 *vs = reinterpret_cast<uint4 *>(smem_u);                    // [8][d / 8]
+    float *ps = reinterpret_cast<float *>(vs + kDecodeWarps * d8);   // [8]
+    const int kch = (a.K + kDecodeWarps - 1) / kDecodeWarps;
+    for (int ch = blockIdx.x; ch < a.L * kch; ch += gridDim.x) {
+        const int t = ch / kch, k0 = (ch - t * kch) * kDecodeWarps;
+        const int nw = a.K - k0 < kDecodeWarps ? a.K - k0 : kDecodeWarps;
+        if (warp < nw) {
+            const int m = t * a.K + k0 + warp;
+            int64_t e = a.idx[m];
+            const float g = a.gate[m];
+            if (e < 0 || e >= a.N) {
+                set_status(a.status, OMNI_DEV_BAD_EXPERT);
+                e = 0;
             }
-        }
-        const float h = warp_sum(acc);
-        const float p = g * (h / (1.f + __expf(-h)));
-        float *yr = a.y + (size_t)t * a.d;
+            const uint4 *x4 = reinterpret_cast<const uint4 *>(a.x) + (size_t)t * d8;
+            const uint4 *w4 = reinterpret_cast<const uint4 *>(a.W) + (size_t)e * d8;
+            const uint4 *v4 = reinterpret_cast<const uint4 *>(a.V) + (size_t)e * d8;
+            uint4 xu[kDecodeSlices], wu[kDecodeSlices], vu[kDecodeSlices];
 #pragma unroll
-        for (int i = 0; i < kDecodeSlices; ++i) {
-            const int c8 = (int)lane + 32 * i;
-            if (c8 < d8) {
-                const uint32_t vw[4] = {vu[i].x, vu[i].y, vu[i].z, vu[i].w};
-                float f[8];
+            for (int i = 0; i < kDecodeSlices; ++i) {         // every slice in flight at once
+                const int c8 = (int)lane + 32 * i;
+                const bool in = c8 < d8;
+                xu[i] = in ? x4[c8] : make_uint4(0u, 0u, 0u, 0u);
+                wu[i] = in ? w4[c8] : make_uint4(0u, 0u, 0u, 0u);
+                vu[i] = in ? v4[c8] : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < kDecodeSlices; ++i) {
+                const uint32_t xw[4] = {xu[i].x, xu[i].y, xu[i].z, xu[i].w};
+                const uint32_t ww[4] = {wu[i].x, wu[i].y, wu[i].z, wu[i].w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    f[2 * q] = p * __uint_as_float(vw[q] << 16);
-                    f[2 * q + 1] = p * __uint_as_float(vw[q] & 0xffff0000u);
+                    acc = fmaf(__uint_as_float(xw[q] << 16), __uint_as_float(ww[q] << 16), acc);
+                    acc = fmaf(__uint_as_float(xw[q] & 0xffff0000u),
+                               __uint_as_float(ww[q] & 0xffff0000u), acc);
                 }
-                red_add_v4(yr + 8 * c8, f[0], f[1], f[2], f[3]);
-                red_add_v4(yr + 8 * c8 + 4, f[4], f[5], f[6], f[7]);
             }
+#pragma unroll
+            for (int i = 0; i < kDecodeSlices; ++i) {
+                const int c8 = (int)lane + 32 * i;
+                if (c8 < d8) vs[warp * d8 + c8] = vu[i];
+            }
+            const float h = warp_sum(acc);
+            if (lane == 0) ps[warp] = g * (h / (1.f + __expf(-h)));
         }
+        __syncthreads();
+        float *yr = a.y + (size_t)t * a.d;
+        for (int c8 = threadIdx.x; c8 < d8; c8 += blockDim.x) {
+            float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int w = 0; w < nw; ++w) {
+                const uint4 u = vs[w * d8 + c8];
+                const float p = ps[w];
+                const uint32_t vw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    f[2 * q] = fmaf(p, __uint_as_float(vw[q] << 16), f[2 * q]);
+                    f[2 * q + 1] = fmaf(p, __uint_as_float(vw[q] & 0xffff0000u), f[2 * q + 1]);
+                }
+            }
+            red_add_v4(yr + 8 * c8, f[0], f[1], f[2], f[3]);
+            red_add_v4(yr + 8 * c8 + 4, f[4], f[5], f[6], f[7]);
+        }
+        __syncthreads();                                   // vs and ps are rewritten next
     }
 }
 
@@ -1194,34 +1809,77 @@ cudaError_t launch_merge_topk(const float *row_val, const int *row_idx, const fl
 #undef OMNI_MG
 }
 
-// Shared words of one axis warp of the fused decode step: axis_row_exact's
-// values, two bucket arrays and max(2 kmax, 2 CAP) words of candidates (as
-// the stand-alone axis kernel takes), a multiple of 4.
+// Candidates the axis bucket sort of the fused decode step takes (more go to
+// its radix select).
+static int decode_tmp_cap(int nmax, int kmax) {
+    const int cap = nmax < 1024 ? nmax : 1024;
+    return cap > kmax ? cap : kmax;
+}
+
+// Shared words of one axis half of the fused decode step (group_axis_select):
+// the row (nmax, rounded up to even), hist and cur (kNB each), 8 words of
+// scratch and the 64-bit candidate keys; a multiple of 4.
 static size_t decode_axis_words(int nmax, int kmax) {
-    const size_t area = kmax > kDecodeCap ? 2 * (size_t)kmax : 2 * (size_t)kDecodeCap;
-    const size_t words = (((size_t)nmax + 2 * kNB + 1) & ~(size_t)1) + area;
+    const size_t words = (((size_t)nmax + 1) & ~(size_t)1) + 2 * kNB + 8 +
+                         2 * (size_t)decode_tmp_cap(nmax, kmax);
     return (words + 3) & ~(size_t)3;
 }
 
-// Shared words of the fused decode step for these sizes (0 if it does not
-// apply): the larger of phase A (x) and phase B (candidate table, two axis
-// warps or the merge warp).
-static size_t decode_smem_bytes(int L, int d, int N_r, int N_c, int K, int Kr, int Kc, int C) {
-    if (L > 16 || K > 128 || d > 32 * 8 * kDecodeSlices || d % 256 != 0) return 0;
+// Shared words of the block-wide merge (group_merge): its head and the
+// 64-bit keys of the C candidates.
+static size_t decode_merge_words(int K, int C) {
+    return ((size_t)group_merge_head_words(K) + 2 * (size_t)C + 3) & ~(size_t)3;
+}
+
+// Shared words of a token's row and column top-K lists (values and indices),
+// a multiple of 4.
+static size_t decode_list_words(int Kr, int Kc) {
+    return ((size_t)2 * (Kr + Kc) + 3) & ~(size_t)3;
+}
+
+// The launch shape of the fused decode step for these sizes: two CTAs per SM
+// when their shared memory allows it, else one; the first grid - L CTAs
+// project rpc router rows each (the last L select, one token each).  Shared
+// memory per CTA is the largest of phase A (token rows, router rows, the
+// copy barrier), phase B (candidate table, the token's lists, the axis
+// halves or the merge) and phase C (8 staged v rows and their p).
+struct DecodePlan {
+    int grid, rpc, nproj;
+    size_t smem;
+};
+
+static bool decode_plan(int L, int d, int N_r, int N_c, int K, int Kr, int Kc, int C,
+                        DecodePlan *plan) {
+    if (L < 1 || L > 16 || K > 128 || d > 32 * 8 * kSmallSlices || d % 256 != 0) return false;
     const int nmax = N_r > N_c ? N_r : N_c;
     const int kmax = Kr > Kc ? Kr : Kc;
     const size_t axis_words = decode_axis_words(nmax, kmax);
     const size_t head = ((size_t)C + Kr + 1 + 3) & ~(size_t)3;
-    const MergeLayout ml = merge_layout(K, Kr, Kc, C, kDecodeCap);
-    const size_t area = 2 * axis_words > ml.words ? 2 * axis_words : ml.words;
-    const size_t b_bytes = 4 * (head + area);
-    const size_t a_bytes = (size_t)L * d * 2;
-    const size_t bytes = a_bytes > b_bytes ? a_bytes : b_bytes;
-    return bytes <= 200 * 1024 ? bytes : 0;
+    const size_t mw = decode_merge_words(K, C);
+    const size_t area = 2 * axis_words > mw ? 2 * axis_words : mw;
+    const size_t lists = decode_list_words(Kr, Kc);
+    const size_t b_bytes = 4 * (head + lists + area);
+    const size_t c_bytes = (size_t)kDecodeWarps * d * 2 + 4 * kDecodeWarps;
+    const int sms = device_sm_count();
+    for (int per_sm = 2; per_sm >= 1; --per_sm) {
+        const int grid = sms * per_sm;
+        const int nproj = grid - L;
+        if (nproj < 1) continue;
+        const int rpc = (N_r + N_c + nproj - 1) / nproj;
+        const size_t a_bytes = (size_t)(L + rpc) * d * 2 + 16 + 4 * 256 * kDecodeWarps;
+        size_t bytes = a_bytes > b_bytes ? a_bytes : b_bytes;
+        if (c_bytes > bytes) bytes = c_bytes;
+        if (bytes > 200 * 1024) continue;
+        if (per_sm == 2 && 2 * (bytes + 1024) > 228 * 1024) continue;
+        *plan = {grid, rpc, nproj, bytes};
+        return true;
+    }
+    return false;
 }
 
 bool decode_fused_ok(int L, int d, int N_r, int N_c, int K, int Kr, int Kc, int C) {
-    return decode_smem_bytes(L, d, N_r, N_c, K, Kr, Kc, C) > 0;
+    DecodePlan plan;
+    return decode_plan(L, d, N_r, N_c, K, Kr, Kc, C, &plan);
 }
 
 cudaError_t launch_decode_fused(const uint16_t *x, const uint16_t *W, const uint16_t *V,
@@ -1229,34 +1887,38 @@ cudaError_t launch_decode_fused(const uint16_t *x, const uint16_t *W, const uint
                                 int N_c, int K, int Kr, int Kc, int C, float *s_r, float *s_c,
                                 float *row_val, int *row_idx, float *col_val, int *col_idx,
                                 int32_t *idx, float *score, float *gate, float *y,
-                                bool accumulate, unsigned *bar, int *status, cudaStream_t st) {
-    const size_t smem = decode_smem_bytes(L, d, N_r, N_c, K, Kr, Kc, C);
-    if (smem == 0) return cudaErrorInvalidValue;
+                                bool accumulate, unsigned long long *bar, unsigned epoch,
+                                int *status, cudaStream_t st) {
+    DecodePlan plan;
+    if (!decode_plan(L, d, N_r, N_c, K, Kr, Kc, C, &plan)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)plan.smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel,
-                                                      32 * kDecodeWarps, smem);
+                                                      32 * kDecodeWarps, plan.smem);
     if (e != cudaSuccess) return e;
-    if (per_sm > 2) per_sm = 2;
-    const int grid = device_sm_count() * per_sm;      // every CTA resident (cooperative launch)
-    if (per_sm < 1 || grid < L) return cudaErrorInvalidValue;
+    if (per_sm * device_sm_count() < plan.grid) return cudaErrorInvalidValue;   // not all resident
     DecodeArgs a;
     a.x = x; a.W = W; a.V = V; a.W_r = W_r; a.W_c = W_c;
     a.L = L; a.d = d; a.N_r = N_r; a.N_c = N_c; a.K = K; a.Kr = Kr; a.Kc = Kc; a.C = C;
     a.N = (int64_t)N_r * N_c;
     a.s_r = s_r; a.s_c = s_c; a.row_val = row_val; a.col_val = col_val;
     a.row_idx = row_idx; a.col_idx = col_idx; a.idx = idx; a.score = score; a.gate = gate;
-    a.y = y; a.accumulate = accumulate ? 1 : 0; a.bar = bar; a.status = status;
+    a.y = y; a.accumulate = accumulate ? 1 : 0; a.bar = bar; a.epoch = epoch; a.status = status;
+    a.rpc = plan.rpc; a.nproj = plan.nproj;
     a.nmax = N_r > N_c ? N_r : N_c;
     a.kmax = Kr > Kc ? Kr : Kc;
     a.axis_words = (int)decode_axis_words(a.nmax, a.kmax);
     a.merge_head = (int)(((size_t)C + Kr + 1 + 3) & ~(size_t)3);
+    a.list_words = (int)decode_list_words(Kr, Kc);
+    a.nmax_pad = (a.nmax + 1) & ~1;
+    a.tmp_cap = decode_tmp_cap(a.nmax, a.kmax);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
+    cfg.gridDim = dim3((unsigned)plan.grid);
     cfg.blockDim = dim3(32 * kDecodeWarps);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;

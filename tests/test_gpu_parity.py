@@ -391,17 +391,23 @@ def test_routed_bwd_accumulates():
     (3, 256, 100, 37, 16),         # ragged axes (37: rows not a multiple of 4)
     (5, 512, 64, 64, 128),         # K = 128 on a small grid (K > N_r)
     (16, 1024, 512, 512, 128),
+    (2, 512, 200, 300, 32),        # two tokens (CUDA-core projection), unequal axes
+    (4, 256, 2400, 2400, 32),      # more than 16 router rows per CTA (two row tiles)
 ])
 def test_decode_step_against_oracle(L, d, N_r, N_c, K):
     """L <= 16 runs the whole routed step (projection, selection, gates,
     token-order expert work) in one cooperative launch: routing against the
     oracle under the near-tie rule, y on every token against the oracle on
-    the GPU's routing, idx_out / gate_out, and OMNI_Y_ACCUMULATE."""
+    the GPU's routing, idx_out / gate_out, and OMNI_Y_ACCUMULATE.  The
+    workspace starts filled with 0xff bytes: the step needs no cleared state
+    (its barrier word is tagged per call), and a second call on the same
+    workspace (the accumulating one) still synchronises."""
     torch.cuda.empty_cache()
     cfg = configs.LayerConfig("decode", L, d, N_r, N_c, K, 64)
     t = inputs.make_inputs(cfg, DEV, seed=9)
     u = {k: host(v) for k, v in t.items() if k in ("x", "W_r", "W_c")}
     ws = omni.workspace(L, d, N_r, N_c, K, cfg.B)
+    ws.fill_(0xff)           # the step clears its own status and barrier state
     y, idx, gate = omni.routed_fwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], K, cfg.B, ws=ws,
                                    want_routing=True)
     assert omni.omni_get_device_status(ws) == 0
