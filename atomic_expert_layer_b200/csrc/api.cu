@@ -425,6 +425,9 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     // nothing here reads the distinct-expert count, so it is not kept
     SchedPrep prep = sched_prep_of(sz, ws, lay);
     prep.bitmap = nullptr;
+    // the expert stage needs each group's tasks together, in no particular
+    // order inside the group: no radix pass, so no first-pass digit counts
+    if (sched_unordered(sz)) prep.hist0 = nullptr;
     if (fused) {
         // a handful of tokens: the whole step in one cooperative launch
         static std::atomic<unsigned> epochs{0};
@@ -461,7 +464,8 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
         int32_t *gact = ws_at<int32_t>(ws, lay.g_act), *nact = ws_at<int32_t>(ws, lay.n_act);
         int32_t *ndist = ws_at<int32_t>(ws, lay.n_dist);
         if ((rc = cuda_rc(launch_schedule(idx, gate, sz, tt, te, tg, goff, gcnt, gact, nact,
-                                          ndist, ws, lay, st, /*prepared=*/true))))
+                                          ndist, ws, lay, st, /*prepared=*/true,
+                                          /*any_order=*/true))))
             return rc;
         if ((rc = cuda_rc(expert_stage(x, W, V, sz, tt, te, tg, goff, gact, nact, y,
                                        (flags & OMNI_Y_ACCUMULATE) != 0, ws, lay, st,

@@ -120,13 +120,19 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
                             int32_t *task_token, int32_t *task_expert, float *task_gate,
                             int32_t *group_offsets, int32_t *group_counts,
                             int32_t *active_groups, int32_t *num_active, int32_t *num_distinct,
-                            void *ws, const WsLayout &lay, cudaStream_t st, bool prepared = false);
+                            void *ws, const WsLayout &lay, cudaStream_t st, bool prepared = false,
+                            bool any_order = false);
 int sched_pass_width(const Sizes &sz);
 uint32_t sched_pass_mask(const Sizes &sz, int p);
 SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay);
 // the radix scatter combines equal histogram increments of a warp (crowded
 // groups, see schedule.cu)
 bool sched_aggregate(const Sizes &sz);
+// with any_order, launch_schedule groups the tasks by q without ordering a
+// group's tasks by (token, expert) when the groups are not crowded (one scan
+// and one scatter instead of the radix passes); the per-token step then need
+// not count the first pass's digits
+bool sched_unordered(const Sizes &sz);
 
 // ---- grouped expert stage (expects the per-token slot counters zeroed).
 // task_token == nullptr: the tasks are in token order, task m belongs to

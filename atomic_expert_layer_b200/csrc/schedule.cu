@@ -393,6 +393,56 @@ cudaError_t launch_exclusive_scan(int32_t *a, int64_t n, int32_t *total, cudaStr
     return launch(exclusive_scan_kernel, dim3(1), dim3(1024), 0, st, a, n, total);
 }
 
+namespace {
+// Grouping by q = e / B without ordering inside a group (the routed forward's
+// schedule, where the expert stage needs each group's tasks together but in
+// no particular order): task i of the token-order arrays goes to
+// offsets[q] + (a position counted down from the group's total in counts[q]).
+// Lanes of a warp with the same q (a token's experts of one group are
+// adjacent) share one atomic and keep their order.  A position outside the
+// group's range (counts that do not match the tasks) is reported as
+// OMNI_DEV_BAD_SCHEDULE and not written.
+__global__ void __launch_bounds__(kScatterThreads) group_scatter_kernel(
+    const int32_t *__restrict__ a_tok, const int32_t *__restrict__ a_exp,
+    const float *__restrict__ a_gate, int64_t M, int B, int64_t G,
+    const int32_t *__restrict__ offsets, int32_t *__restrict__ counts, int32_t *__restrict__ d_tok,
+    int32_t *__restrict__ d_exp, float *__restrict__ d_gate, int *status) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const unsigned lane = lane_id();
+    int32_t t = 0, e = 0;
+    float g = 0.f;
+    int64_t q = -1;
+    if (i < M) {
+        t = a_tok[i];
+        e = a_exp[i];
+        g = a_gate[i];
+        q = e >= 0 ? e / B : -1;
+        if (q >= G) q = -1;
+        if (q < 0) set_status(status, OMNI_DEV_BAD_EXPERT);
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, (unsigned)(q + 1));
+    const int leader = __ffs(peers) - 1;
+    const int n = __popc(peers);
+    int base = 0;
+    if (q >= 0 && (int)lane == leader) base = atomicSub(&counts[q], n) - n;
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (q >= 0) {
+        const int r = base + __popc(peers & lanemask_lt());
+        const int64_t o0 = offsets[q], o1 = offsets[q + 1];
+        const int64_t pos = o0 + r;
+        if (r < 0 || pos >= o1) {
+            set_status(status, OMNI_DEV_BAD_SCHEDULE);
+        } else {
+            d_tok[pos] = t;
+            d_exp[pos] = e;
+            d_gate[pos] = g;
+        }
+    }
+}
+}  // namespace
+
 int sched_pass_width(const Sizes &sz) {
     return sz.passes ? (sz.qbits + sz.passes - 1) / sz.passes : 0;
 }
@@ -410,6 +460,8 @@ bool sched_aggregate(const Sizes &sz) {
     // equal ones first
     return sz.M >= 64 * sz.G;
 }
+
+bool sched_unordered(const Sizes &sz) { return sz.passes > 0 && !sched_aggregate(sz); }
 
 SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay) {
     SchedPrep o;
@@ -430,7 +482,8 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
                             int32_t *task_token, int32_t *task_expert, float *task_gate,
                             int32_t *group_offsets, int32_t *group_counts,
                             int32_t *active_groups, int32_t *num_active, int32_t *num_distinct,
-                            void *ws, const WsLayout &lay, cudaStream_t st, bool prepared) {
+                            void *ws, const WsLayout &lay, cudaStream_t st, bool prepared,
+                            bool any_order) {
     // The caller has zeroed [0, lay.zero_end) of ws: the status word, the
     // group counters, the distinct-expert counter, the bitmap and the radix
     // histograms.  With `prepared`, the per-token step (sched_token.cuh) has
@@ -462,6 +515,18 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
                    bitmap, ndist, passes ? hist : nullptr, ntiles, passes ? pass_mask(0) : 0u,
                    status);
         if (e != cudaSuccess) return e;
+    }
+    if (any_order && sched_unordered(sz)) {
+        // grouping only: offsets, then one scatter that counts each group's
+        // tasks down from its total (the counters are not needed after the scan)
+        e = launch(sched_scan_kernel, dim3(1), dim3(1024), 0, st, counts, G, group_counts,
+                   group_offsets, active_groups, num_active, ndist, num_distinct,
+                   (int32_t *)nullptr, (int64_t)0);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = (unsigned)((M + kScatterThreads - 1) / kScatterThreads);
+        return launch(group_scatter_kernel, dim3(grid), dim3(kScatterThreads), 0, st, a_tok, a_exp,
+                      a_gate, M, sz.B, G, (const int32_t *)group_offsets, counts, task_token,
+                      task_expert, task_gate, status);
     }
     e = launch(sched_scan_kernel, dim3(passes ? 2 : 1), dim3(1024), 0, st, counts, G,
                group_counts, group_offsets, active_groups, num_active, ndist, num_distinct, hist,
