@@ -440,20 +440,21 @@ __global__ void axis_topk_kernel(const float *__restrict__ in_r, const float *__
 // Fast path for rows with n % 4 == 0 and n <= 128 * NPL: lane l holds float4
 // number l + 32 j of the row (j < NPL) in registers.  mode 0: the input is
 // p; mode 1: p = s - lse with lse from the GEMM partials; mode 2: p = s - lse
-// computed here.  A row this kernel cannot finish (too few values within 8
-// units of the maximum, or more than CAP candidates) sets flags[row] = 1 and
-// is redone by axis_topk_kernel; every other row gets flags[row] = 0.
-// Shared memory per warp (words): hist[kNB] | cur[kNB] | tmp[CAP] (u64).
+// computed here.  A row the bucket sort cannot finish (too few values within
+// 8 units of the maximum, or more than CAP candidates) is redone by the same
+// warp with the exact radix select of axis_row_exact, which reads the row
+// again.  Shared memory per warp (warp_words, even): hist[kNB] | cur[kNB] |
+// tmp[CAP] (u64), or axis_row_exact's area for nmax, kmax.  Up to 11 float4
+// per lane, at most 96 registers, so that five CTAs share an SM.
 template <int NPL, int CAP>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, NPL <= 11 ? 5 : 4)
 axis_topk_reg_kernel(const float *__restrict__ in_r, const float *__restrict__ in_c, int mode,
                      const float2 *__restrict__ part_r, const float2 *__restrict__ part_c,
                      float *__restrict__ p_r_out, float *__restrict__ p_c_out, int L, int N_r,
                      int N_c, int K, float *__restrict__ row_val, int *__restrict__ row_idx,
-                     float *__restrict__ col_val, int *__restrict__ col_idx,
-                     int *__restrict__ flags) {
+                     float *__restrict__ col_val, int *__restrict__ col_idx, int nmax, int kmax,
+                     int warp_words) {
     extern __shared__ __align__(16) uint32_t smem_u[];
-    constexpr int kWords = 2 * kNB + 2 * CAP;
     grid_dependency_wait();
     grid_dependents_launch();
     const int warp = threadIdx.x >> 5;
@@ -467,7 +468,7 @@ axis_topk_reg_kernel(const float *__restrict__ in_r, const float *__restrict__ i
     const int kx = K < n ? K : n;
     const float4 *in4 = reinterpret_cast<const float4 *>((axis ? in_c : in_r) + (size_t)t * n);
     float *pout = axis ? p_c_out : p_r_out;
-    uint32_t *hist = smem_u + (size_t)warp * kWords;
+    uint32_t *hist = smem_u + (size_t)warp * warp_words;
     uint32_t *cur = hist + kNB;
     uint64_t *tmp = reinterpret_cast<uint64_t *>(cur + kNB);
 
@@ -545,8 +546,13 @@ axis_topk_reg_kernel(const float *__restrict__ in_r, const float *__restrict__ i
     __syncwarp();
     int bs = 0;
     const int ncand = bucket_find(hist, kx, &bs);
+    float *oval = (axis ? col_val : row_val) + (size_t)t * kx;
+    int *oidx = (axis ? col_idx : row_idx) + (size_t)t * kx;
     if (ncand < kx || ncand > CAP) {
-        if (lane == 0) flags[prob] = 1;
+        __syncwarp();
+        axis_row_exact<0>((axis ? in_c : in_r) + (size_t)t * n, n, kx, mode != 0,
+                          mode == 1 ? (axis ? part_c : part_r) : nullptr, t, pout, oval, oidx,
+                          nmax, kmax, hist);
         return;
     }
     bucket_starts(hist, cur);
@@ -566,8 +572,6 @@ axis_topk_reg_kernel(const float *__restrict__ in_r, const float *__restrict__ i
         place(v[j].w, i + 3);
     }
     __syncwarp();
-    float *oval = (axis ? col_val : row_val) + (size_t)t * kx;
-    int *oidx = (axis ? col_idx : row_idx) + (size_t)t * kx;
     for (int pos = lane; pos < ncand; pos += 32) {
         const uint64_t k = tmp[pos];
         const int b = bucket_of(vmax, key2f((uint32_t)(k >> 32)));
@@ -581,7 +585,6 @@ axis_topk_reg_kernel(const float *__restrict__ in_r, const float *__restrict__ i
             oidx[fp] = (int)(0xffffffffu - (uint32_t)k);
         }
     }
-    if (lane == 0) flags[prob] = 0;
 }
 
 // ----------------------------------------------------------- merge top-K
@@ -1683,20 +1686,37 @@ static cudaError_t launch_axis_e(const float *in_r, const float *in_c, bool logs
                   row_val, row_idx, col_val, col_idx, nmax, kmax, words, only);
 }
 
+// Shared words per warp of axis_topk_reg_kernel (even): its bucket sort, or
+// the exact fallback's area (axis_row_exact: the row, hist, cur and the
+// selected keys and indices).
+static int axis_reg_warp_words(int cap, int nmax, int kmax) {
+    const int fast = 2 * kNB + 2 * cap;
+    const int exact = ((nmax + 2 * kNB + 1) & ~1) + 2 * kmax;
+    const int w = fast > exact ? fast : exact;
+    return (w + 1) & ~1;
+}
+
 template <int NPL, int CAP>
 static cudaError_t launch_axis_reg(const float *in_r, const float *in_c, int mode,
                                    const float *part_r, const float *part_c, float *p_r_out,
                                    float *p_c_out, int L, int N_r, int N_c, int K, float *row_val,
-                                   int *row_idx, float *col_val, int *col_idx, int *flags,
-                                   cudaStream_t st) {
+                                   int *row_idx, float *col_val, int *col_idx, cudaStream_t st) {
     constexpr int wpb = 4;
-    const size_t smem = (size_t)wpb * (2 * kNB + 2 * CAP) * 4;
+    const int nmax = N_r > N_c ? N_r : N_c;
+    const int kmax = K < nmax ? K : nmax;
+    const int words = axis_reg_warp_words(CAP, nmax, kmax);
+    const size_t smem = (size_t)wpb * words * 4;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(axis_topk_reg_kernel<NPL, CAP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
     const int64_t probs = 2 * (int64_t)L;
     const unsigned grid = (unsigned)((probs + wpb - 1) / wpb);
     return launch(axis_topk_reg_kernel<NPL, CAP>, dim3(grid), dim3(32 * wpb), smem, st, in_r, in_c,
                   mode, reinterpret_cast<const float2 *>(part_r),
                   reinterpret_cast<const float2 *>(part_c), p_r_out, p_c_out, L, N_r, N_c, K,
-                  row_val, row_idx, col_val, col_idx, flags);
+                  row_val, row_idx, col_val, col_idx, nmax, kmax, words);
 }
 
 template <int CAP>
@@ -1704,12 +1724,13 @@ static cudaError_t launch_axis_reg_npl(int npl, const float *in_r, const float *
                                        const float *part_r, const float *part_c, float *p_r_out,
                                        float *p_c_out, int L, int N_r, int N_c, int K,
                                        float *row_val, int *row_idx, float *col_val,
-                                       int *col_idx, int *flags, cudaStream_t st) {
-#define OMNI_RG(np) return launch_axis_reg<np, CAP>(in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, flags, st);
+                                       int *col_idx, cudaStream_t st) {
+#define OMNI_RG(np) return launch_axis_reg<np, CAP>(in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
     if (npl <= 1) { OMNI_RG(1) }
     if (npl <= 2) { OMNI_RG(2) }
     if (npl <= 4) { OMNI_RG(4) }
     if (npl <= 8) { OMNI_RG(8) }
+    if (npl <= 11) { OMNI_RG(11) }
     if (npl <= 12) { OMNI_RG(12) }
     OMNI_RG(16)
 #undef OMNI_RG
@@ -1731,12 +1752,11 @@ cudaError_t launch_axis_topk(const float *in_r, const float *in_c, bool logsoftm
     const int mode = !logsoftmax ? 0 : (part_r && part_c ? 1 : 2);
     cudaError_t e;
     const int *only = nullptr;
-    if (reg) {
-        if (cap <= 96) e = launch_axis_reg_npl<96>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, flags, st);
-        else if (cap <= 192) e = launch_axis_reg_npl<192>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, flags, st);
-        else e = launch_axis_reg_npl<320>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, flags, st);
-        if (e != cudaSuccess) return e;
-        only = flags;                      // the general kernel redoes the flagged rows
+    if (reg) {                             // the register kernel finishes every row itself
+        if (cap <= 96) e = launch_axis_reg_npl<96>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
+        else if (cap <= 192) e = launch_axis_reg_npl<192>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
+        else e = launch_axis_reg_npl<320>(npl, in_r, in_c, mode, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, st);
+        return e;
     }
 #define OMNI_AX(c) return launch_axis_e<c>(in_r, in_c, logsoftmax, part_r, part_c, p_r_out, p_c_out, L, N_r, N_c, K, row_val, row_idx, col_val, col_idx, only, st);
     if (cap == 0) { OMNI_AX(0) }
