@@ -18,7 +18,7 @@ from ._lib import (OMNI_ROUTER_LOGPROBS_IN, OMNI_TOKEN_ORDER, OMNI_TOPK_BLOCKWIS
                    expert_workspace, omni_expert_workspace_size, omni_get_device_status,
                    omni_grouped_expert_fwd, omni_grouped_expert_fwd_noalloc,
                    omni_noalloc_get_device_status, omni_routed_bwd,
-                   omni_routed_fwd,
+                   omni_routed_bwd_workspace_size, omni_routed_fwd,
                    omni_router_topk,
                    omni_router_workspace_size, omni_schedule, omni_schedule_workspace_size,
                    omni_selftest_wait_timeout, omni_shared_mlp_fwd,
@@ -33,6 +33,7 @@ __all__ = [
     "omni_routed_fwd", "omni_get_device_status", "workspace", "omni_grouped_expert_fwd_noalloc",
     "omni_noalloc_get_device_status",
     "router_topk", "schedule", "grouped_expert_fwd", "routed_fwd", "omni_routed_bwd", "routed_bwd",
+    "omni_routed_bwd_workspace_size",
     "omni_shared_mlp_workspace_size", "omni_shared_mlp_fwd", "shared_mlp_fwd", "layer_fwd",
 ]
 
@@ -132,7 +133,9 @@ def routed_bwd(x, W, V, W_r, W_c, idx, gate, dy, dW=None, dV=None, dW_r=None, dW
     dV = torch.zeros(V.shape, **f32) if dV is None else dV
     dW_r = torch.zeros(W_r.shape, **f32) if dW_r is None else dW_r
     dW_c = torch.zeros(W_c.shape, **f32) if dW_c is None else dW_c
-    ws = torch.zeros(256, dtype=torch.uint8, device=dev) if ws is None else ws
+    if ws is None:
+        ws = torch.empty(omni_routed_bwd_workspace_size(L, d, N_r, N_c, K), dtype=torch.uint8,
+                         device=dev)
     omni_routed_bwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, idx, gate, dy, dx, dW, dV, dW_r, dW_c,
                     0, ws, stream)
     return dict(dx=dx, dW=dW, dV=dV, dW_r=dW_r, dW_c=dW_c)

@@ -44,6 +44,7 @@ SIGNATURES = {
                                  _U, _P, _Z, _P], _I),
     "omni_routed_fwd": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _U, _P, _Z, _P],
                         _I),
+    "omni_routed_bwd_workspace_size": ([_I, _I, _I, _I, _I], _Z),
     "omni_routed_bwd": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                          _U, _P, _Z, _P], _I),
     "omni_shared_mlp_workspace_size": ([_I, _I, _I], _Z),
@@ -187,6 +188,10 @@ def omni_routed_fwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, B, y, idx_out, gate_ou
                                 K, B, _ptr(y), _ptr(idx_out), _ptr(gate_out), flags, _ptr(ws),
                                 ws.numel(), _stream(stream))
     _check("omni_routed_fwd", rc)
+
+
+def omni_routed_bwd_workspace_size(L, d, N_r, N_c, K) -> int:
+    return load().omni_routed_bwd_workspace_size(L, d, N_r, N_c, K)
 
 
 def omni_routed_bwd(x, W, V, W_r, W_c, L, d, N_r, N_c, K, idx, gate, dy, dx, dW, dV, dW_r, dW_c,

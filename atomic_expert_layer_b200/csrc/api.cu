@@ -502,9 +502,22 @@ int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
         return OMNI_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     first_launch_in_call();
-    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return OMNI_ERR_CUDA;
+    // with room for them, two bitmaps over the experts (seen, used more than once)
+    const size_t map = align256(4 * (size_t)((sz.N + 31) / 32));
+    const bool marks = ws_bytes >= sizeof(WsHeader) + 2 * map;
+    if (cudaMemsetAsync(ws, 0, marks ? sizeof(WsHeader) + 2 * map : sizeof(WsHeader), st) !=
+        cudaSuccess)
+        return OMNI_ERR_CUDA;
+    uint32_t *seen = marks ? ws_at<uint32_t>(ws, sizeof(WsHeader)) : nullptr;
+    uint32_t *shared_rows = marks ? ws_at<uint32_t>(ws, sizeof(WsHeader) + map) : nullptr;
     return cuda_rc(launch_routed_bwd(x, W, V, W_r, W_c, sz, idx, gate, dy, dx, dW, dV, dW_r,
-                                     dW_c, ws_at<int>(ws, 0), st));
+                                     dW_c, seen, shared_rows, ws_at<int>(ws, 0), st));
+}
+
+size_t omni_routed_bwd_workspace_size(int L, int d, int N_r, int N_c, int K) {
+    Sizes sz;
+    if (check_common(L, d, N_r, N_c, K, 1, true, &sz)) return 0;
+    return sizeof(WsHeader) + 2 * align256(4 * (size_t)((sz.N + 31) / 32));
 }
 
 size_t omni_shared_mlp_workspace_size(int L, int d, int F) {

@@ -17,10 +17,14 @@
 //   dW_r[i] += dp_r[i] x_t,  dW_c[j] += dp_c[j] x_t.
 //
 // One warp per token: x_t and dy_t stay in registers, the K expert rows of W
-// and V are gathered, dx_t is accumulated in registers and written once; the
-// weight gradients are scatter-added with 16-byte fp32 reductions, the
-// router rows once per distinct row / column of the token (its K cells sit
-// in few rows and columns, (a+1)(b+1) <= K).
+// and V are gathered, dx_t is accumulated in registers and written once.  The
+// dW and dV rows of an expert that only this task uses (most of them, when
+// the tasks spread over many experts) get a plain read-add-write; the others
+// are scatter-added with 16-byte fp32 reductions, which the L2 runs well
+// below HBM bandwidth.  A first kernel marks the experts used more than once
+// (two bitmaps over the N experts) when the workspace has room for them.
+// The router rows are added once per distinct row / column of the token (its
+// K cells sit in few rows and columns, (a+1)(b+1) <= K).
 #include "omni_common.cuh"
 #include "omni_internal.h"
 
@@ -28,6 +32,7 @@ namespace omni {
 namespace {
 
 constexpr int kBwdWarps = 4;
+constexpr int kPrefetch = 1;              // tasks whose rows are asked of L2 ahead (2 measured slower)
 
 __device__ __forceinline__ void bf16x8_f32(const uint4 &u, float *f) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -66,6 +71,39 @@ __device__ __forceinline__ void red_row_bf16(float *row, float s, const uint4 *u
         red_add_f32x4(p + 4, s * q[4], s * q[5], s * q[6], s * q[7]);
     }
 }
+// The same two updates as a plain read-add-write, for a row no other task
+// touches (both rows are read before either is written back).
+template <int VPL>
+__device__ __forceinline__ void rmw_rows(float *rv, float sv, const float *fv, float *rw, float sw,
+                                         const uint4 *uw, unsigned lane) {
+    float4 ov[2 * VPL], ow[2 * VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        const float4 *pv = reinterpret_cast<const float4 *>(rv + (size_t)(v * 32 + lane) * 8);
+        const float4 *pw = reinterpret_cast<const float4 *>(rw + (size_t)(v * 32 + lane) * 8);
+        ov[2 * v] = pv[0];
+        ov[2 * v + 1] = pv[1];
+        ow[2 * v] = pw[0];
+        ow[2 * v + 1] = pw[1];
+    }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        const float *q = fv + 8 * v;
+        float w[8];
+        bf16x8_f32(uw[v], w);
+        float4 *pv = reinterpret_cast<float4 *>(rv + (size_t)(v * 32 + lane) * 8);
+        float4 *pw = reinterpret_cast<float4 *>(rw + (size_t)(v * 32 + lane) * 8);
+        pv[0] = make_float4(fmaf(sv, q[0], ov[2 * v].x), fmaf(sv, q[1], ov[2 * v].y),
+                            fmaf(sv, q[2], ov[2 * v].z), fmaf(sv, q[3], ov[2 * v].w));
+        pv[1] = make_float4(fmaf(sv, q[4], ov[2 * v + 1].x), fmaf(sv, q[5], ov[2 * v + 1].y),
+                            fmaf(sv, q[6], ov[2 * v + 1].z), fmaf(sv, q[7], ov[2 * v + 1].w));
+        pw[0] = make_float4(fmaf(sw, w[0], ow[2 * v].x), fmaf(sw, w[1], ow[2 * v].y),
+                            fmaf(sw, w[2], ow[2 * v].z), fmaf(sw, w[3], ow[2 * v].w));
+        pw[1] = make_float4(fmaf(sw, w[4], ow[2 * v + 1].x), fmaf(sw, w[5], ow[2 * v + 1].y),
+                            fmaf(sw, w[6], ow[2 * v + 1].z), fmaf(sw, w[7], ow[2 * v + 1].w));
+    }
+}
+
 // acc += s * (raw bf16 slice u)
 template <int VPL>
 __device__ __forceinline__ void axpy_bf16(float *acc, float s, const uint4 *u) {
@@ -77,6 +115,14 @@ __device__ __forceinline__ void axpy_bf16(float *acc, float s, const uint4 *u) {
         for (int c = 0; c < 8; ++c) acc[8 * v + c] = fmaf(s, q[c], acc[8 * v + c]);
     }
 }
+// Asks L2 for the 128-byte lines of a row of `bytes` bytes (one line per
+// lane and round), so that a later load of it does not wait for HBM.
+__device__ __forceinline__ void prefetch_row_l2(const void *row, int bytes, unsigned lane) {
+    const char *p = static_cast<const char *>(row);
+    for (int o = (int)lane * 128; o < bytes; o += 32 * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p + o));
+}
+
 template <int VPL>
 __device__ __forceinline__ void load_raw(const uint16_t *row, uint4 *u, unsigned lane) {
     const uint4 *r4 = reinterpret_cast<const uint4 *>(row);
@@ -137,7 +183,7 @@ routed_bwd_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
                   const int32_t *__restrict__ idx, const float *__restrict__ gate,
                   const float *__restrict__ dy, float *__restrict__ dx, float *__restrict__ dW,
                   float *__restrict__ dV, float *__restrict__ dW_r, float *__restrict__ dW_c,
-                  int *status) {
+                  const uint32_t *__restrict__ shared_rows, int *status) {
     constexpr int D = 256 * VPL;
     constexpr int E = 8 * VPL;                       // columns per lane
     extern __shared__ __align__(16) uint8_t smem[];
@@ -185,6 +231,17 @@ routed_bwd_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
     for (int k = 0; k < K; ++k) {
         const int e = se[k];
         const float g = sg[k];
+        // the rows of the task kPrefetch ahead, into L2 (the first ones
+        // before the loop)
+        for (int kk = k == 0 ? 1 : k + kPrefetch; kk <= k + kPrefetch && kk < K; ++kk) {
+            const int en = se[kk];
+            prefetch_row_l2(W + (size_t)en * D, 2 * D, lane);
+            prefetch_row_l2(V + (size_t)en * D, 2 * D, lane);
+            prefetch_row_l2(dW + (size_t)en * D, 4 * D, lane);
+            prefetch_row_l2(dV + (size_t)en * D, 4 * D, lane);
+        }
+        // an expert no other task uses gets a plain read-add-write of its rows
+        const bool own = shared_rows && !((shared_rows[e >> 5] >> (e & 31)) & 1u);
         uint4 wu[VPL], vu[VPL];
         load_raw<VPL>(W + (size_t)e * D, wu, lane);
         load_raw<VPL>(V + (size_t)e * D, vu, lane);
@@ -207,8 +264,12 @@ routed_bwd_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
         const float a = h * s;
         const float dg = a * c;
         const float dh = g * c * (s * (1.f + h * (1.f - s)));
-        red_row_f32<VPL>(dV + (size_t)e * D, g * a, dyf, lane);
-        red_row_bf16<VPL>(dW + (size_t)e * D, dh, xu, lane);
+        if (own) {
+            rmw_rows<VPL>(dV + (size_t)e * D, g * a, dyf, dW + (size_t)e * D, dh, xu, lane);
+        } else {
+            red_row_f32<VPL>(dV + (size_t)e * D, g * a, dyf, lane);
+            red_row_bf16<VPL>(dW + (size_t)e * D, dh, xu, lane);
+        }
         axpy_bf16<VPL>(acc, dh, wu);
         if (lane == 0) sd[k] = dg;
         sgd = fmaf(g, dg, sgd);
@@ -244,12 +305,27 @@ routed_bwd_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
     }
 }
 
+// Experts used by more than one task: seen / shared bitmaps over the N
+// experts (both zeroed), one thread per task.  Ids outside [0, N) count as
+// expert 0, as in the backward kernel.
+__global__ void bwd_mark_kernel(const int32_t *__restrict__ idx, int64_t M, int N,
+                                uint32_t *__restrict__ seen, uint32_t *__restrict__ shared_rows) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= M) return;
+    int e = idx[i];
+    if (e < 0 || e >= N) e = 0;
+    const uint32_t bit = 1u << (e & 31);
+    if (atomicOr(&seen[e >> 5], bit) & bit) atomicOr(&shared_rows[e >> 5], bit);
+}
+
 template <int VPL>
 cudaError_t launch_bwd_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V,
                            const uint16_t *W_r, const uint16_t *W_c, const Sizes &sz,
                            const int32_t *idx, const float *gate, const float *dy, float *dx,
-                           float *dW, float *dV, float *dW_r, float *dW_c, int *status,
-                           cudaStream_t st) {
+                           float *dW, float *dV, float *dW_r, float *dW_c,
+                           const uint32_t *shared_rows, int *status, cudaStream_t st) {
     const size_t smem = (size_t)kBwdWarps * 6 * sz.K * 4;
     cudaError_t e = cudaFuncSetAttribute(routed_bwd_kernel<VPL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -257,7 +333,7 @@ cudaError_t launch_bwd_vpl(const uint16_t *x, const uint16_t *W, const uint16_t 
     const unsigned grid = (unsigned)((sz.L + kBwdWarps - 1) / kBwdWarps);
     return launch(routed_bwd_kernel<VPL>, dim3(grid), dim3(32 * kBwdWarps), smem, st, x, W, V,
                   W_r, W_c, sz.L, (int)sz.N, sz.N_c, sz.K, idx, gate, dy, dx, dW, dV, dW_r, dW_c,
-                  status);
+                  shared_rows, status);
 }
 
 }  // namespace
@@ -265,12 +341,20 @@ cudaError_t launch_bwd_vpl(const uint16_t *x, const uint16_t *W, const uint16_t 
 cudaError_t launch_routed_bwd(const uint16_t *x, const uint16_t *W, const uint16_t *V,
                               const uint16_t *W_r, const uint16_t *W_c, const Sizes &sz,
                               const int32_t *idx, const float *gate, const float *dy, float *dx,
-                              float *dW, float *dV, float *dW_r, float *dW_c, int *status,
-                              cudaStream_t st) {
+                              float *dW, float *dV, float *dW_r, float *dW_c, uint32_t *seen,
+                              uint32_t *shared_rows, int *status, cudaStream_t st) {
+    if (seen && shared_rows) {
+        const unsigned grid = (unsigned)((sz.M + 255) / 256);
+        cudaError_t e = launch(bwd_mark_kernel, dim3(grid), dim3(256), 0, st, idx, (int64_t)sz.M,
+                               (int)sz.N, seen, shared_rows);
+        if (e != cudaSuccess) return e;
+    } else {
+        shared_rows = nullptr;
+    }
     switch (sz.d / 256) {
 #define OMNI_BCASE(n) \
         case n: return launch_bwd_vpl<n>(x, W, V, W_r, W_c, sz, idx, gate, dy, dx, dW, dV, dW_r, \
-                                         dW_c, status, st);
+                                         dW_c, shared_rows, status, st);
         OMNI_BCASE(1) OMNI_BCASE(2) OMNI_BCASE(3) OMNI_BCASE(4)
         OMNI_BCASE(5) OMNI_BCASE(6) OMNI_BCASE(7) OMNI_BCASE(8)
 #undef OMNI_BCASE

@@ -179,8 +179,8 @@ cudaError_t launch_exclusive_scan(int32_t *a, int64_t n, int32_t *total, cudaStr
 cudaError_t launch_routed_bwd(const uint16_t *x, const uint16_t *W, const uint16_t *V,
                               const uint16_t *W_r, const uint16_t *W_c, const Sizes &sz,
                               const int32_t *idx, const float *gate, const float *dy, float *dx,
-                              float *dW, float *dV, float *dW_r, float *dW_c, int *status,
-                              cudaStream_t st);
+                              float *dW, float *dV, float *dW_r, float *dW_c, uint32_t *seen,
+                              uint32_t *shared_rows, int *status, cudaStream_t st);
 
 // ---- shared dense MLP (two tile GEMMs; h is [L, F] bf16 scratch)
 cudaError_t launch_shared_mlp(const uint16_t *x, const uint16_t *W_g, const uint16_t *W_u,

@@ -402,7 +402,8 @@ def run_omni(args, cfg, world, rank, local):
         gen = torch.Generator(device=dev)
         gen.manual_seed(11)
         g_dy = torch.randn((L, d), generator=gen, **f32)
-        ws_b = torch.zeros(256, dtype=torch.uint8, device=dev)
+        ws_b = torch.empty(omni.omni_routed_bwd_workspace_size(L, d, cfg.N_r, cfg.N_c, cfg.K),
+                           dtype=torch.uint8, device=dev)        # with the expert bitmaps
 
         def bstep():
             omni.omni_routed_bwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r,

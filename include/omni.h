@@ -259,9 +259,14 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
  *   dx [L, d] fp32     output, overwritten
  *   dW, dV [N, d] fp32 accumulated (+=) in the rows of the experts used
  *   dW_r [N_r, d], dW_c [N_c, d] fp32  accumulated (+=)
- * The weight gradients are sums of fp32 reductions: their last bits vary
- * between runs.  ws: at least 256 bytes (the status word).  All fp32 arrays
- * 16-byte aligned.  Limits: d % 256 == 0, d <= OMNI_MAX_D, K <= OMNI_MAX_K.
+ * ws: at least 256 bytes (the status word).  With at least
+ * omni_routed_bwd_workspace_size() bytes the call first marks, in two
+ * bitmaps over the N experts, the experts that more than one task uses; the
+ * dW and dV rows of every other expert then get one plain read-add-write
+ * (the fastest path, and bit-reproducible), and only the shared rows go
+ * through fp32 reductions, whose last bits vary between runs.  With less,
+ * every row is reduced.  All fp32 arrays 16-byte aligned.
+ * Limits: d % 256 == 0, d <= OMNI_MAX_D, K <= OMNI_MAX_K.
  */
 int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                     const omni_bf16 *W_r, const omni_bf16 *W_c,
@@ -269,6 +274,11 @@ int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                     const int32_t *idx, const float *gate, const float *dy,
                     float *dx, float *dW, float *dV, float *dW_r, float *dW_c,
                     unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
+
+/* Workspace bytes of omni_routed_bwd with its expert bitmaps: 256 plus two
+ * bitmaps of N bits, each rounded up to 256 bytes (0 for invalid sizes).  The
+ * pages have no counterpart; it only sizes the backward's scratch. */
+size_t omni_routed_bwd_workspace_size(int L, int d, int N_r, int N_c, int K);
 
 /*
  * The shared dense MLP that the layer adds to the routed branch

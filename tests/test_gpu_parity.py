@@ -324,14 +324,18 @@ def _check_grad(got, ref, name, tol=2e-4):
     assert rel <= tol, (name, rel)
 
 
-def _bwd_case(cfg, L_sub, seed):
+def _bwd_case(cfg, L_sub, seed, marks=True):
+    """marks: a workspace with the expert bitmaps (rows used once get a plain
+    read-add-write), else the 256-byte minimum (every row reduced)."""
     t = inputs.make_inputs(cfg, DEV, seed=0)
     x = t["x"][:L_sub].contiguous()
     rt = omni.router_topk(x, t["W_r"], t["W_c"], cfg.K)
     g = torch.Generator(device=DEV)
     g.manual_seed(seed)
     dy = torch.randn((L_sub, cfg.d), generator=g, device=DEV, dtype=torch.float32)
-    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    n_ws = (omni.omni_routed_bwd_workspace_size(L_sub, cfg.d, cfg.N_r, cfg.N_c, cfg.K) if marks
+            else 256)
+    ws = torch.full((n_ws,), 0xff, dtype=torch.uint8, device=DEV)   # the call clears what it uses
     out = omni.routed_bwd(x, t["W"], t["V"], t["W_r"], t["W_c"], rt["idx"], rt["gate"], dy, ws=ws)
     assert omni.omni_get_device_status(ws) == 0
     # oracle on the GPU's routing; expert rows compacted to the ones used
@@ -355,16 +359,22 @@ def _bwd_case(cfg, L_sub, seed):
     return t, x, rt, dy, out
 
 
+@pytest.mark.parametrize("marks", [True, False], ids=["bitmaps", "min_ws"])
 @pytest.mark.parametrize("cfg,L_sub", [(configs.TINY, configs.TINY.L),
                                        (configs.HEADLINE, 48),
                                        (configs.sweep(16), 16)],
                          ids=lambda v: getattr(v, "name", str(v)))
-def test_routed_bwd_against_oracle(cfg, L_sub):
+def test_routed_bwd_against_oracle(cfg, L_sub, marks):
     """Backward through the C ABI against the fp64 oracle backward on the
-    GPU's own routing: every token of the tiny layer, and a token batch at
-    the full headline and d = 2048 shapes (N = 1.7M experts)."""
+    GPU's own routing: every token of the tiny layer (experts shared by many
+    tasks), and a token batch at the full headline and d = 2048 shapes
+    (N = 1.7M experts, almost all used once); with the expert bitmaps (rows
+    used once read-add-written, shared rows reduced) and without them."""
     torch.cuda.empty_cache()
-    _bwd_case(cfg, L_sub, seed=5)
+    t, x, rt, dy, out = _bwd_case(cfg, L_sub, seed=5, marks=marks)
+    if cfg is configs.TINY:
+        counts = torch.bincount(rt["idx"].long().flatten(), minlength=cfg.N)
+        assert int((counts == 1).sum()) > 0 and int((counts > 1).sum()) > 0   # both kinds of row
     torch.cuda.empty_cache()
 
 
