@@ -427,7 +427,10 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
     prep.bitmap = nullptr;
     // the expert stage needs each group's tasks together, in no particular
     // order inside the group: no radix pass, so no first-pass digit counts
-    if (sched_unordered(sz)) prep.hist0 = nullptr;
+    if (sched_unordered(sz)) {
+        prep.hist0 = nullptr;
+        prep.unordered = 1;
+    }
     if (fused) {
         // a handful of tokens: the whole step in one cooperative launch
         static std::atomic<unsigned> epochs{0};

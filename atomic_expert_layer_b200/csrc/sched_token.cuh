@@ -1,7 +1,9 @@
 // sched_token.cuh -- the per-token first step of the expert-centric schedule,
 // shared by the schedule's own prepare kernel and by the router's merge
 // kernel (which already holds a token's K experts and gates on chip when the
-// whole routed forward runs).
+// whole routed forward runs).  When the schedule only groups the tasks (the
+// routed forward with uncrowded groups), the order inside a token does not
+// matter and the rank sort is skipped.
 //
 // "OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at Scale"
 // (rainbus review page, method paragraph, step 3): the routing decisions
@@ -31,6 +33,8 @@ struct SchedPrep {          // where the per-token step writes (all in the works
     int64_t ntiles;
     uint32_t dmask0;        // digit mask of the first pass
     int B;
+    int unordered;          // the tasks are only grouped (no radix pass follows): a token's
+                            // tasks keep the routing's order, no rank sort by expert
 };
 
 __device__ __forceinline__ uint32_t sched_digit(int32_t e, int B, int shift, uint32_t dmask) {
@@ -48,10 +52,13 @@ __device__ __forceinline__ void sched_token(const SchedPrep &o, int t, int K, co
         bool fresh = false;
         if (u < K) {
             const int32_t eu = e_s[u];
-            int r = 0;
-            for (int v = 0; v < K; ++v) {
-                const int32_t ev = e_s[v];
-                r += (ev < eu) | ((ev == eu) & (v < u));
+            int r = u;
+            if (!o.unordered) {
+                r = 0;
+                for (int v = 0; v < K; ++v) {
+                    const int32_t ev = e_s[v];
+                    r += (ev < eu) | ((ev == eu) & (v < u));
+                }
             }
             const size_t pos = row + r;
             o.a_tok[pos] = t;

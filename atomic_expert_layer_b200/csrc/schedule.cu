@@ -67,7 +67,7 @@ __global__ void sched_prepare_kernel(const int32_t *__restrict__ idx,
     SchedPrep o;
     o.a_tok = a_tok; o.a_exp = a_exp; o.a_gate = a_gate;
     o.counts = counts; o.bitmap = bitmap; o.num_distinct = num_distinct;
-    o.hist0 = hist0; o.ntiles = ntiles; o.dmask0 = dmask0; o.B = B;
+    o.hist0 = hist0; o.ntiles = ntiles; o.dmask0 = dmask0; o.B = B; o.unordered = 0;
     sched_token(o, t, K, e_s, [&](int u) {
         const int32_t raw = idx[row + u];
         return (raw < 0 || raw >= N) ? 0.f : gate[row + u];
@@ -475,6 +475,7 @@ SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay) {
     o.ntiles = sz.ntiles;
     o.dmask0 = sz.passes ? sched_pass_mask(sz, 0) : 0u;
     o.B = sz.B;
+    o.unordered = 0;
     return o;
 }
 
