@@ -982,11 +982,178 @@ __device__ __forceinline__ float group_max(float v, int ht, int nt, int bar_id, 
 // fall in those buckets (or fewer than kx in range), an exact radix select
 // takes over.  Shared: vals (n words), hist, cur (kNB each), tmp
 // (max(tmp_cap, kx) 64-bit keys), scr (8 words).
+// The exact selection of group_axis_select from the keys of p (in vals as
+// raw words): radix select, ties by the smaller index, compaction and a rank
+// sort into oval / oidx.
+__device__ void group_axis_exact_keys(int n, int kx, int ht, int nt, int bar_id, float *vals,
+                                      uint32_t *hist, uint64_t *tmp, int *scr, float *oval,
+                                      int *oidx) {
+    float *red = reinterpret_cast<float *>(scr + 2);
+    auto key_of = [&](int i) { return __float_as_uint(vals[i]); };
+    int take_eq;
+    const uint32_t T = group_radix_select(key_of, n, kx, ht, nt, bar_id, hist, scr, &take_eq);
+    // keys equal to T: the take_eq smallest indices (by radix select on the
+    // inverted index among them, when there are more)
+    int n_eq = 0;
+    for (int i = ht; i < n; i += nt) n_eq += key_of(i) == T ? 1 : 0;
+    n_eq = (int)group_sum((float)n_eq, ht, nt, bar_id, red);
+    uint32_t Tl = 0u;
+    if (n_eq > take_eq) {
+        int tl_eq;
+        Tl = group_radix_select([&](int i) { return key_of(i) == T ? 0xffffffffu - (uint32_t)i : 0u; },
+                                n, take_eq, ht, nt, bar_id, hist, scr, &tl_eq);
+    }
+    // compact the kx selected (64-bit keys: p key, inverted index), one
+    // atomic per warp and round
+    if (ht == 0) scr[0] = 0;
+    named_sync(bar_id, nt);
+    for (int i0 = 0; i0 < n; i0 += nt) {
+        const int i = i0 + ht;
+        bool take = false;
+        uint32_t key = 0u, lo = 0u;
+        if (i < n) {
+            key = key_of(i);
+            lo = 0xffffffffu - (uint32_t)i;
+            take = key > T || (key == T && (n_eq == take_eq || lo >= Tl));
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        int base = 0;
+        if (bal && lane_id() == 0) base = atomicAdd(&scr[0], __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (take) {
+            const int at = base + __popc(bal & lanemask_lt());
+            if (at < kx) tmp[at] = ((uint64_t)key << 32) | lo;
+        }
+    }
+    named_sync(bar_id, nt);
+    // rank sort (keys are distinct)
+    for (int j = ht; j < kx; j += nt) {
+        const uint64_t kj = tmp[j];
+        int r = 0;
+        for (int i = 0; i < kx; ++i) r += tmp[i] > kj;
+        oval[r] = key2f((uint32_t)(kj >> 32));
+        oidx[r] = (int)(0xffffffffu - (uint32_t)kj);
+    }
+    named_sync(bar_id, nt);
+}
+
+// (m, s) pairs of a running logsumexp: s = sum exp(v - m) over the values
+// seen; m = -inf with s = 0 for none.
+__device__ __forceinline__ void lse_combine(float &m, float &s, float m2, float s2) {
+    const float mx = fmaxf(m, m2);
+    if (mx == -INFINITY) return;
+    s = (m == -INFINITY ? 0.f : s * __expf(m - mx)) + (m2 == -INFINITY ? 0.f : s2 * __expf(m2 - mx));
+    m = mx;
+}
+
+constexpr int kAxisRegJ = 4;    // float4 per thread held in registers by group_axis_select
+
 __device__ void group_axis_select(const float *__restrict__ in, int n, int kx, int ht, int nt,
                                   int bar_id, float *vals, uint32_t *hist, uint32_t *cur,
                                   uint64_t *tmp, int tmp_cap, int *scr, float *oval, int *oidx) {
     float *red = reinterpret_cast<float *>(scr + 2);
     for (int b = ht; b < kNB; b += nt) hist[b] = 0u;
+    const int n4 = n >> 2;
+    if ((n & 3) == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0 && n4 <= kAxisRegJ * nt) {
+        // ---- the row in registers: one (max, sum exp) reduction, then the
+        // bucket counts, the scatter and the rank without shared-memory passes
+        const float4 *in4 = reinterpret_cast<const float4 *>(in);
+        float4 v[kAxisRegJ];
+#pragma unroll
+        for (int j = 0; j < kAxisRegJ; ++j) {
+            const int i4 = ht + j * nt;
+            v[j] = i4 < n4 ? in4[i4] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+        float m = -INFINITY, sm_ = 0.f;
+#pragma unroll
+        for (int j = 0; j < kAxisRegJ; ++j)
+            m = fmaxf(fmaxf(m, fmaxf(v[j].x, v[j].y)), fmaxf(v[j].z, v[j].w));
+        if (m > -INFINITY) {
+#pragma unroll
+            for (int j = 0; j < kAxisRegJ; ++j)
+                sm_ += __expf(v[j].x - m) + __expf(v[j].y - m) + __expf(v[j].z - m) + __expf(v[j].w - m);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+            const float s2 = __shfl_xor_sync(0xffffffffu, sm_, o);
+            lse_combine(m, sm_, m2, s2);
+        }
+        float2 *red2 = reinterpret_cast<float2 *>(tmp);          // nt / 32 pairs, before tmp is used
+        if ((ht & 31) == 0) red2[ht >> 5] = make_float2(m, sm_);
+        named_sync(bar_id, nt);
+        float M = -INFINITY, S = 0.f;
+        for (int w = 0; w < nt / 32; ++w) lse_combine(M, S, red2[w].x, red2[w].y);
+        const float lse = M + __logf(S);
+        const float vmax = M - lse;                 // the p of the largest logit, same rounding
+#pragma unroll
+        for (int j = 0; j < kAxisRegJ; ++j) {
+            v[j].x -= lse; v[j].y -= lse; v[j].z -= lse; v[j].w -= lse;
+            if (ht + j * nt < n4) {
+                const float q[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int b = bucket_of(vmax, q[c]);
+                    if (b < kNB) atomicAdd(&hist[b], 1u);
+                }
+            }
+        }
+        named_sync(bar_id, nt);                     // counts complete; red2 no longer read
+        if (ht < 32) {
+            int bs = 0;
+            const int nc = bucket_scan(hist, cur, kx, &bs);
+            if (ht == 0) {
+                scr[0] = nc >= kx && nc <= tmp_cap ? nc : -1;
+                scr[1] = bs;
+            }
+        }
+        named_sync(bar_id, nt);
+        const int ncand = scr[0], bstar = scr[1];
+        if (ncand >= 0) {
+#pragma unroll
+            for (int j = 0; j < kAxisRegJ; ++j) {
+                if (ht + j * nt < n4) {
+                    const float q[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int b = bucket_of(vmax, q[c]);
+                        if (b <= bstar) {
+                            const int i = 4 * (ht + j * nt) + c;
+                            tmp[atomicAdd(&cur[b], 1u)] =
+                                ((uint64_t)f2key(q[c]) << 32) | (uint64_t)(0xffffffffu - (uint32_t)i);
+                        }
+                    }
+                }
+            }
+            named_sync(bar_id, nt);
+            for (int pos = ht; pos < ncand; pos += nt) {
+                const uint64_t k = tmp[pos];
+                const float p = key2f((uint32_t)(k >> 32));
+                const int b = bucket_of(vmax, p);
+                const int s0 = (int)hist[b], s1 = b < bstar ? (int)hist[b + 1] : ncand;
+                int r = 0;
+                for (int q = s0; q < s1; ++q) r += tmp[q] > k ? 1 : 0;
+                if (s0 + r < kx) {
+                    oval[s0 + r] = p;
+                    oidx[s0 + r] = (int)(0xffffffffu - (uint32_t)k);
+                }
+            }
+            named_sync(bar_id, nt);
+            return;
+        }
+        // the exact fallback below starts from the keys of p in shared memory
+#pragma unroll
+        for (int j = 0; j < kAxisRegJ; ++j) {
+            const int i4 = ht + j * nt;
+            if (i4 < n4)
+                reinterpret_cast<float4 *>(vals)[i4] =
+                    make_float4(__uint_as_float(f2key(v[j].x)), __uint_as_float(f2key(v[j].y)),
+                                __uint_as_float(f2key(v[j].z)), __uint_as_float(f2key(v[j].w)));
+        }
+        named_sync(bar_id, nt);
+        group_axis_exact_keys(n, kx, ht, nt, bar_id, vals, hist, tmp, scr, oval, oidx);
+        return;
+    }
     // the row with every load in flight, its maximum
     float mx = -INFINITY;
     if ((n & 3) == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0) {
@@ -1057,52 +1224,7 @@ __device__ void group_axis_select(const float *__restrict__ in, int n, int kx, i
     // ---- exact fallback: radix select on the keys of p
     for (int i = ht; i < n; i += nt) vals[i] = __uint_as_float(f2key(vals[i]));
     named_sync(bar_id, nt);
-    auto key_of = [&](int i) { return __float_as_uint(vals[i]); };
-    int take_eq;
-    const uint32_t T = group_radix_select(key_of, n, kx, ht, nt, bar_id, hist, scr, &take_eq);
-    // keys equal to T: the take_eq smallest indices (by radix select on the
-    // inverted index among them, when there are more)
-    int n_eq = 0;
-    for (int i = ht; i < n; i += nt) n_eq += key_of(i) == T ? 1 : 0;
-    n_eq = (int)group_sum((float)n_eq, ht, nt, bar_id, red);
-    uint32_t Tl = 0u;
-    if (n_eq > take_eq) {
-        int tl_eq;
-        Tl = group_radix_select([&](int i) { return key_of(i) == T ? 0xffffffffu - (uint32_t)i : 0u; },
-                                n, take_eq, ht, nt, bar_id, hist, scr, &tl_eq);
-    }
-    // compact the kx selected (64-bit keys: p key, inverted index), one
-    // atomic per warp and round
-    if (ht == 0) scr[0] = 0;
-    named_sync(bar_id, nt);
-    for (int i0 = 0; i0 < n; i0 += nt) {
-        const int i = i0 + ht;
-        bool take = false;
-        uint32_t key = 0u, lo = 0u;
-        if (i < n) {
-            key = key_of(i);
-            lo = 0xffffffffu - (uint32_t)i;
-            take = key > T || (key == T && (n_eq == take_eq || lo >= Tl));
-        }
-        const unsigned bal = __ballot_sync(0xffffffffu, take);
-        int base = 0;
-        if (bal && lane_id() == 0) base = atomicAdd(&scr[0], __popc(bal));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (take) {
-            const int at = base + __popc(bal & lanemask_lt());
-            if (at < kx) tmp[at] = ((uint64_t)key << 32) | lo;
-        }
-    }
-    named_sync(bar_id, nt);
-    // rank sort (keys are distinct)
-    for (int j = ht; j < kx; j += nt) {
-        const uint64_t kj = tmp[j];
-        int r = 0;
-        for (int i = 0; i < kx; ++i) r += tmp[i] > kj;
-        oval[r] = key2f((uint32_t)(kj >> 32));
-        oidx[r] = (int)(0xffffffffu - (uint32_t)kj);
-    }
-    named_sync(bar_id, nt);
+    group_axis_exact_keys(n, kx, ht, nt, bar_id, vals, hist, tmp, scr, oval, oidx);
 }
 
 // Shared words of the block-wide merge (group_merge) ahead of its candidate
