@@ -129,9 +129,9 @@ SchedPrep sched_prep_of(const Sizes &sz, void *ws, const WsLayout &lay);
 // groups, see schedule.cu)
 bool sched_aggregate(const Sizes &sz);
 // with any_order, launch_schedule groups the tasks by q without ordering a
-// group's tasks by (token, expert) when the groups are not crowded (one scan
-// and one scatter instead of the radix passes); the per-token step then need
-// not count the first pass's digits
+// group's tasks by (token, expert) (one scan and one scatter instead of the
+// radix passes); the per-token step then need not count the first pass's
+// digits nor sort a token's experts
 bool sched_unordered(const Sizes &sz);
 
 // ---- grouped expert stage (expects the per-token slot counters zeroed).

@@ -2,8 +2,8 @@
 // shared by the schedule's own prepare kernel and by the router's merge
 // kernel (which already holds a token's K experts and gates on chip when the
 // whole routed forward runs).  When the schedule only groups the tasks (the
-// routed forward with uncrowded groups), the order inside a token does not
-// matter and the rank sort is skipped.
+// routed forward), the order inside a token does not matter and the rank
+// sort is skipped.
 //
 // "OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at Scale"
 // (rainbus review page, method paragraph, step 3): the routing decisions
