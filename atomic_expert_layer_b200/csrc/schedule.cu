@@ -441,6 +441,75 @@ __global__ void __launch_bounds__(kScatterThreads) group_scatter_kernel(
         }
     }
 }
+
+// The same scatter for crowded groups (a few groups hold thousands of tasks):
+// a CTA of 1024 threads first gathers its tasks' groups in a shared-memory
+// hash table (kAggSlots open-addressed slots, at most 1024 keys), each task
+// taking its rank inside the CTA's share of its group; then one thread per
+// distinct group takes the CTA's share from counts[q] with one atomic, so a
+// hot group's counter sees one atomic per CTA instead of one per warp.
+constexpr int kAggThreads = 1024;
+constexpr int kAggSlots = 2048;
+__global__ void __launch_bounds__(kAggThreads) group_scatter_agg_kernel(
+    const int32_t *__restrict__ a_tok, const int32_t *__restrict__ a_exp,
+    const float *__restrict__ a_gate, int64_t M, int B, int64_t G,
+    const int32_t *__restrict__ offsets, int32_t *__restrict__ counts, int32_t *__restrict__ d_tok,
+    int32_t *__restrict__ d_exp, float *__restrict__ d_gate, int *status) {
+    __shared__ int keys[kAggSlots];
+    __shared__ int cnt[kAggSlots];
+    __shared__ int base[kAggSlots];
+    grid_dependency_wait();
+    grid_dependents_launch();
+    for (int h = threadIdx.x; h < kAggSlots; h += kAggThreads) {
+        keys[h] = -1;
+        cnt[h] = 0;
+    }
+    const int64_t i = (int64_t)blockIdx.x * kAggThreads + threadIdx.x;
+    int32_t t = 0, e = 0;
+    float g = 0.f;
+    int q = -1;
+    if (i < M) {
+        t = a_tok[i];
+        e = a_exp[i];
+        g = a_gate[i];
+        const int64_t qq = e >= 0 ? e / B : -1;
+        q = qq < G ? (int)qq : -1;
+        if (q < 0) set_status(status, OMNI_DEV_BAD_EXPERT);
+    }
+    __syncthreads();
+    int slot = -1, r = 0;
+    if (q >= 0) {
+        // at most kAggThreads keys in kAggSlots slots: the probe ends
+        int h = (int)(((uint32_t)q * 2654435761u) >> 21);          // 11 bits
+        for (int probe = 0; probe < kAggSlots; ++probe) {
+            const int k = atomicCAS(&keys[h], -1, q);
+            if (k == -1 || k == q) {
+                slot = h;
+                break;
+            }
+            h = (h + 1) & (kAggSlots - 1);
+        }
+        if (slot >= 0) r = atomicAdd(&cnt[slot], 1);
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < kAggSlots; h += kAggThreads) {
+        const int c = cnt[h];
+        if (c > 0) base[h] = atomicSub(&counts[keys[h]], c) - c;
+    }
+    __syncthreads();
+    if (slot >= 0) {
+        const int64_t o0 = offsets[q], o1 = offsets[q + 1];
+        const int rr = base[slot] + r;
+        const int64_t pos = o0 + rr;
+        if (rr < 0 || pos >= o1) {
+            set_status(status, OMNI_DEV_BAD_SCHEDULE);
+        } else {
+            d_tok[pos] = t;
+            d_exp[pos] = e;
+            d_gate[pos] = g;
+        }
+    }
+}
 }  // namespace
 
 int sched_pass_width(const Sizes &sz) {
@@ -527,6 +596,12 @@ cudaError_t launch_schedule(const int32_t *idx, const float *gate, const Sizes &
                    group_offsets, active_groups, num_active, ndist, num_distinct,
                    (int32_t *)nullptr, (int64_t)0);
         if (e != cudaSuccess) return e;
+        if (sched_aggregate(sz)) {
+            const unsigned grid = (unsigned)((M + kAggThreads - 1) / kAggThreads);
+            return launch(group_scatter_agg_kernel, dim3(grid), dim3(kAggThreads), 0, st, a_tok,
+                          a_exp, a_gate, M, sz.B, G, (const int32_t *)group_offsets, counts,
+                          task_token, task_expert, task_gate, status);
+        }
         const unsigned grid = (unsigned)((M + kScatterThreads - 1) / kScatterThreads);
         return launch(group_scatter_kernel, dim3(grid), dim3(kScatterThreads), 0, st, a_tok, a_exp,
                       a_gate, M, sz.B, G, (const int32_t *)group_offsets, counts, task_token,
