@@ -1,6 +1,5 @@
 // router_small.cuh -- the streamed router projection for a handful of
-// tokens (shared by the small-batch projection kernel and the fused decode
-// step).
+// tokens (the small-batch projection kernel of the router stage call).
 //
 // "OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at Scale"
 // (rainbus review page, method paragraph, step 2): s_r = x W_r and
@@ -23,8 +22,8 @@ namespace {
 // memory, and each (row, token) dot product is reduced over the warp.  Only
 // s is written; the axis selection then takes LogSoftmax itself.  Measured
 // on B200 at d = 2048: faster than the tile GEMM at L = 1 (5.7 vs ~14 us).
-// It serves the stand-alone projection for L <= 4 and the fused decode step
-// (up to 16 tokens).
+// It serves the stand-alone projection for L <= 4; its slice width also
+// bounds d in the fused decode step (d <= 32 * 8 * kSmallSlices).
 constexpr int kSmallRows = 2;          // grid rows per warp
 constexpr int kSmallWarps = 8;
 constexpr int kSmallSlices = 8;        // 8-wide slices per lane: d <= 32 * 8 * 8

@@ -1354,14 +1354,15 @@ __device__ void group_merge(const uint32_t *table, const float *rv, const int *r
 // roofline.  Tokens are independent once the router projection is done, so
 // one cooperative launch (every CTA resident) runs the whole step in three
 // phases separated by a grid barrier (a bounded wait):
-//   A. all CTAs: the streamed router projection (small_rows_dot, the
-//      arithmetic of the small-batch projection kernel) into s; y zeroed
-//      unless accumulating; the CTAs that select build the merge's
-//      candidate table;
+//   A. the first gridDim.x - L CTAs: the router projection of their block
+//      of router rows, pulled with the token rows into shared memory by
+//      bulk copies (CUDA-core dot products for 1-2 tokens, mma.sync for
+//      3-16) into s; y zeroed unless accumulating; the last L CTAs build the
+//      merge's candidate table;
 //   B. CTA gridDim.x - 1 - t, token t: LogSoftmax and the exact row and
 //      column top-K (128 threads per axis, group_axis_select), then the
-//      merge and the gates (the whole CTA, group_merge): the selection of
-//      the separate kernels, with the same ranking rule and results;
+//      merge and the gates (the whole CTA, group_merge), with the ranking
+//      rule of the separate kernels;
 //   C. chunks of up to 8 tasks of one token per CTA: h = x_t . w_e,
 //      p = g SiLU(h) per warp, the chunk's sum of p v_e per CTA, added to
 //      y_t with 16-byte fp32 reductions (the order in which a token's chunks
