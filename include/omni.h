@@ -216,18 +216,25 @@ int omni_grouped_expert_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_b
                             omni_stream_t stream);
 
 /*
- * The whole routed branch: omni_router_topk, omni_schedule and
+ * The whole routed branch: omni_router_topk, the schedule and
  * omni_grouped_expert_fwd back to back on `stream`, with every intermediate in
  * `ws` and no host synchronisation:  y = routed(x)  (the shared dense MLP of
  * [G] section 2.1 is not part of it).  OMNI_EXPERT_DENSE / OMNI_EXPERT_SPARSE
  * choose the expert stage's paths as for omni_grouped_expert_fwd (its
- * schedule is produced here, so its offsets are not re-checked).
+ * schedule is produced here, so its offsets are not re-checked).  The
+ * schedule built here only groups the tasks by q = e / B, with no order
+ * inside a group (the expert stage needs no more; omni_schedule returns the
+ * full (group, token, expert) order).
  *   x [L, d], W [N, d], V [N, d], W_r [N_r, d], W_c [N_c, d]  bf16
  *   y [L, d] fp32 output;  idx_out [L, K] int32, gate_out [L, K] fp32 are
  *   optional copies of the routing (NULL to skip).
  * Token order: with flag OMNI_TOKEN_ORDER, and always for L <= 16 tokens,
  * the expert stage takes the tasks in token order straight from the router
  * (task t*K + k = (t, idx[t,k], gate[t,k])) and the schedule is skipped.
+ * For L <= 16 (d <= 2048, K <= 128, within the kernel's shared memory) the
+ * whole step is one cooperative launch (projection, per-token selection and
+ * gates, expert work, separated by bounded grid barriers); it clears its own
+ * status word and needs no cleared workspace.
  * y is the same sum (up to summation order); only the order in which expert
  * rows are fetched changes.  For a few tokens the grouping has nothing to
  * reuse and the schedule's launches are pure latency; for large batches the
