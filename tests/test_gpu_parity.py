@@ -301,6 +301,34 @@ def test_routed_fwd_full_size_sampled(cfg):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("L,d,N_r,N_c,K,B", [
+    (17, 256, 40, 24, 20, 7),      # just above the fused decode size; ragged groups
+    (33, 512, 1, 300, 40, 300),    # a single group: no radix pass, tasks copied in token order
+    (50, 256, 300, 1, 40, 1),      # one expert per group (G = N)
+    (64, 256, 8, 8, 32, 4),        # crowded groups (M >= 64 G): the CTA-gathered scatter
+    (300, 256, 64, 48, 64, 16),    # crowded, several CTAs of tasks
+])
+def test_routed_fwd_schedule_variants(L, d, N_r, N_c, K, B):
+    """The routed forward on shapes that reach each way it builds its
+    schedule (grouping by one atomic scatter, by CTA-gathered atomics for
+    crowded groups, or no grouping with a single group), and the first size
+    past the fused decode step: every token's routing under the near-tie rule
+    and every y row against the oracle on the GPU's routing."""
+    cfg = configs.LayerConfig("variant", L, d, N_r, N_c, K, B)
+    t = inputs.make_inputs(cfg, DEV, seed=4)
+    u = {k: host(v) for k, v in t.items()}
+    ws = omni.workspace(L, d, N_r, N_c, K, B)
+    ws.fill_(0xff)
+    y, idx, gate = omni.routed_fwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], K, B, ws=ws,
+                                   want_routing=True)
+    assert omni.omni_get_device_status(ws) == 0
+    p_r, p_c = oracle.router_logprobs(u["x"], u["W_r"], u["W_c"])
+    idx_ref, score_ref, _ = oracle.topk_from_logprobs(p_r, p_c, K)
+    check_routing_near_ties(host(idx), idx_ref, score_ref, p_r, p_c, N_c)
+    check_y(host(y), oracle.expert_fwd_token_centric(u["x"], u["W"], u["V"], host(idx),
+                                                     host(gate)))
+
+
 def test_routed_fwd_skips_mlp_and_accumulates():
     cfg = configs.LayerConfig("acc", 40, 256, 16, 16, 8, 16)
     t = inputs.make_inputs(cfg, DEV, seed=4)
