@@ -2020,9 +2020,25 @@ static bool decode_plan(int L, int d, int N_r, int N_c, int K, int Kr, int Kc, i
     return false;
 }
 
+// The plan for these sizes, with every CTA of its grid resident at once on
+// this device (a cooperative launch needs that); false otherwise, and the
+// routed forward then takes the separate kernels.
+static bool decode_plan_resident(int L, int d, int N_r, int N_c, int K, int Kr, int Kc, int C,
+                                 DecodePlan *plan) {
+    if (!decode_plan(L, d, N_r, N_c, K, Kr, Kc, C, plan)) return false;
+    if (cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)plan->smem) != cudaSuccess)
+        return false;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel,
+                                                      32 * kDecodeWarps, plan->smem) != cudaSuccess)
+        return false;
+    return per_sm * device_sm_count() >= plan->grid;
+}
+
 bool decode_fused_ok(int L, int d, int N_r, int N_c, int K, int Kr, int Kc, int C) {
     DecodePlan plan;
-    return decode_plan(L, d, N_r, N_c, K, Kr, Kc, C, &plan);
+    return decode_plan_resident(L, d, N_r, N_c, K, Kr, Kc, C, &plan);
 }
 
 cudaError_t launch_decode_fused(const uint16_t *x, const uint16_t *W, const uint16_t *V,
@@ -2033,16 +2049,7 @@ cudaError_t launch_decode_fused(const uint16_t *x, const uint16_t *W, const uint
                                 bool accumulate, unsigned long long *bar, unsigned epoch,
                                 int *status, cudaStream_t st) {
     DecodePlan plan;
-    if (!decode_plan(L, d, N_r, N_c, K, Kr, Kc, C, &plan)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)plan.smem);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel,
-                                                      32 * kDecodeWarps, plan.smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm * device_sm_count() < plan.grid) return cudaErrorInvalidValue;   // not all resident
+    if (!decode_plan_resident(L, d, N_r, N_c, K, Kr, Kc, C, &plan)) return cudaErrorInvalidValue;
     DecodeArgs a;
     a.x = x; a.W = W; a.V = V; a.W_r = W_r; a.W_c = W_c;
     a.L = L; a.d = d; a.N_r = N_r; a.N_c = N_c; a.K = K; a.Kr = Kr; a.Kc = Kc; a.C = C;
