@@ -72,5 +72,10 @@ def mlp_hidden(d: int) -> int:
     return -(-8 * d // (3 * 64)) * 64
 
 
-ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L] + [PROFILE, SKEW_ROUTER_PROFILE]
+# One decode token at the sweep's width on a 512 x 512 grid (W and V of 1 GB
+# each), for profiler captures of the fused decode step.
+DECODE_PROFILE = LayerConfig("decode_profile_L1_d2048_N262144_K64_B128", 1, 2048, 512, 512, 64, 128)
+
+ALL = [TINY, SMALL, HEADLINE, SKEW] + [sweep(L) for L in SWEEP_L] + [PROFILE, SKEW_ROUTER_PROFILE,
+                                                                    DECODE_PROFILE]
 BY_NAME = {c.name: c for c in ALL}
