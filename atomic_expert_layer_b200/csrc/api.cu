@@ -505,22 +505,32 @@ int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
         return OMNI_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     first_launch_in_call();
-    // with room for them, two bitmaps over the experts (seen, used more than once)
+    // with room for them: two bitmaps over the experts (seen, used more than
+    // once), then per router row a pair counter and kBwdRowCap (token, ds) slots
     const size_t map = align256(4 * (size_t)((sz.N + 31) / 32));
-    const bool marks = ws_bytes >= sizeof(WsHeader) + 2 * map;
-    if (cudaMemsetAsync(ws, 0, marks ? sizeof(WsHeader) + 2 * map : sizeof(WsHeader), st) !=
-        cudaSuccess)
-        return OMNI_ERR_CUDA;
+    const size_t nrows = (size_t)sz.N_r + sz.N_c;
+    const size_t cnt_bytes = align256(4 * nrows);
+    const size_t marks_end = sizeof(WsHeader) + 2 * map;
+    const size_t rows_end = marks_end + cnt_bytes + 8 * nrows * kBwdRowCap;
+    const bool marks = ws_bytes >= marks_end;
+    const bool rows = ws_bytes >= rows_end;
+    const size_t clear = rows ? marks_end + cnt_bytes : (marks ? marks_end : sizeof(WsHeader));
+    if (cudaMemsetAsync(ws, 0, clear, st) != cudaSuccess) return OMNI_ERR_CUDA;
     uint32_t *seen = marks ? ws_at<uint32_t>(ws, sizeof(WsHeader)) : nullptr;
     uint32_t *shared_rows = marks ? ws_at<uint32_t>(ws, sizeof(WsHeader) + map) : nullptr;
+    int *rcnt = rows ? ws_at<int>(ws, marks_end) : nullptr;
+    int2 *rslots = rows ? ws_at<int2>(ws, marks_end + cnt_bytes) : nullptr;
     return cuda_rc(launch_routed_bwd(x, W, V, W_r, W_c, sz, idx, gate, dy, dx, dW, dV, dW_r,
-                                     dW_c, seen, shared_rows, ws_at<int>(ws, 0), st));
+                                     dW_c, seen, shared_rows, rcnt, rslots, kBwdRowCap,
+                                     ws_at<int>(ws, 0), st));
 }
 
 size_t omni_routed_bwd_workspace_size(int L, int d, int N_r, int N_c, int K) {
     Sizes sz;
     if (check_common(L, d, N_r, N_c, K, 1, true, &sz)) return 0;
-    return sizeof(WsHeader) + 2 * align256(4 * (size_t)((sz.N + 31) / 32));
+    const size_t nrows = (size_t)sz.N_r + sz.N_c;
+    return sizeof(WsHeader) + 2 * align256(4 * (size_t)((sz.N + 31) / 32)) +
+           align256(4 * nrows) + 8 * nrows * kBwdRowCap;
 }
 
 size_t omni_shared_mlp_workspace_size(int L, int d, int F) {

@@ -183,7 +183,8 @@ routed_bwd_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
                   const int32_t *__restrict__ idx, const float *__restrict__ gate,
                   const float *__restrict__ dy, float *__restrict__ dx, float *__restrict__ dW,
                   float *__restrict__ dV, float *__restrict__ dW_r, float *__restrict__ dW_c,
-                  const uint32_t *__restrict__ shared_rows, int *status) {
+                  const uint32_t *__restrict__ shared_rows, int *__restrict__ rcnt,
+                  int2 *__restrict__ rslots, int rcap, int N_r, int *status) {
     constexpr int D = 256 * VPL;
     constexpr int E = 8 * VPL;                       // columns per lane
     extern __shared__ __align__(16) uint8_t smem[];
@@ -286,13 +287,25 @@ routed_bwd_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ W
         const int n = combine_by_key(key, sd, ord, tmp, sg, K);   // sums into sg
         const uint16_t *Wa = axis == 0 ? W_r : W_c;
         float *dWa = axis == 0 ? dW_r : dW_c;
+        const int base = axis == 0 ? 0 : N_r;                    // row of the slot lists
+        // a slot in each distinct row's list, all of the token's rows at once
+        // (ord is free after combine_by_key); rcap = 0: no lists
+        for (int u = lane; u < n; u += 32)
+            ord[u] = rcap > 0 ? atomicAdd(&rcnt[base + key[u]], 1) : 0;
+        __syncwarp();
         for (int u = 0; u < n; ++u) {
             const int r = key[u];
             const float ds = sg[u];
             uint4 wu[VPL];
             load_raw<VPL>(Wa + (size_t)r * D, wu, lane);
             axpy_bf16<VPL>(acc, ds, wu);
-            red_row_bf16<VPL>(dWa + (size_t)r * D, ds, xu, lane);
+            const int slot = ord[u];
+            if (slot < rcap) {
+                if (lane == 0)
+                    rslots[(size_t)(base + r) * rcap + slot] = make_int2(t, __float_as_int(ds));
+            } else {
+                red_row_bf16<VPL>(dWa + (size_t)r * D, ds, xu, lane);   // a full list
+            }
         }
         __syncwarp();
     }
@@ -320,20 +333,83 @@ __global__ void bwd_mark_kernel(const int32_t *__restrict__ idx, int64_t M, int 
     if (atomicOr(&seen[e >> 5], bit) & bit) atomicOr(&shared_rows[e >> 5], bit);
 }
 
+// The router rows' weight gradients from their slot lists: one warp per grid
+// row (W_r rows, then W_c rows) sums ds * x_t over the row's (t, ds) pairs
+// (four x rows in flight at a time) and adds the sum to its dW_r / dW_c row
+// with one plain read-add-write: the warp owns the row, and the reductions of
+// a full list's extra pairs finished with the previous kernel.
+template <int VPL>
+__global__ void __launch_bounds__(32 * kBwdWarps)
+bwd_router_rows_kernel(const uint16_t *__restrict__ x, int L, int nrows, int N_r,
+                       const int *__restrict__ rcnt, const int2 *__restrict__ rslots, int rcap,
+                       float *__restrict__ dW_r, float *__restrict__ dW_c, int *status) {
+    constexpr int D = 256 * VPL;
+    constexpr int E = 8 * VPL;
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int row = blockIdx.x * kBwdWarps + (int)(threadIdx.x >> 5);
+    if (row >= nrows) return;                        // the same in every lane
+    const unsigned lane = lane_id();
+    const int cnt = min(rcnt[row], rcap);
+    if (cnt <= 0) return;
+    float acc[E];
+#pragma unroll
+    for (int c = 0; c < E; ++c) acc[c] = 0.f;
+    const int2 *sl = rslots + (size_t)row * rcap;
+    for (int s0 = 0; s0 < cnt; s0 += 32) {
+        const int2 mine = s0 + (int)lane < cnt ? sl[s0 + lane] : make_int2(0, 0);
+        const int m = min(32, cnt - s0);
+        for (int j0 = 0; j0 < m; j0 += 4) {
+            uint4 xu[4][VPL];
+            float ds[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                int tq = __shfl_sync(0xffffffffu, mine.x, (j0 + q) & 31);
+                ds[q] = __int_as_float(__shfl_sync(0xffffffffu, mine.y, (j0 + q) & 31));
+                if (j0 + q >= m) ds[q] = 0.f;
+                if (tq < 0 || tq >= L) {
+                    set_status(status, OMNI_DEV_BAD_SCHEDULE);
+                    tq = 0;
+                    ds[q] = 0.f;
+                }
+                load_raw<VPL>(x + (size_t)tq * D, xu[q], lane);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) axpy_bf16<VPL>(acc, ds[q], xu[q]);
+        }
+    }
+    float *dst = row < N_r ? dW_r + (size_t)row * D : dW_c + (size_t)(row - N_r) * D;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        float4 *p = reinterpret_cast<float4 *>(dst + (size_t)(v * 32 + lane) * 8);
+        const float4 a = p[0], b = p[1];
+        p[0] = make_float4(a.x + acc[8 * v], a.y + acc[8 * v + 1], a.z + acc[8 * v + 2],
+                           a.w + acc[8 * v + 3]);
+        p[1] = make_float4(b.x + acc[8 * v + 4], b.y + acc[8 * v + 5], b.z + acc[8 * v + 6],
+                           b.w + acc[8 * v + 7]);
+    }
+}
+
 template <int VPL>
 cudaError_t launch_bwd_vpl(const uint16_t *x, const uint16_t *W, const uint16_t *V,
                            const uint16_t *W_r, const uint16_t *W_c, const Sizes &sz,
                            const int32_t *idx, const float *gate, const float *dy, float *dx,
                            float *dW, float *dV, float *dW_r, float *dW_c,
-                           const uint32_t *shared_rows, int *status, cudaStream_t st) {
+                           const uint32_t *shared_rows, int *rcnt, int2 *rslots, int rcap,
+                           int *status, cudaStream_t st) {
     const size_t smem = (size_t)kBwdWarps * 6 * sz.K * 4;
     cudaError_t e = cudaFuncSetAttribute(routed_bwd_kernel<VPL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((sz.L + kBwdWarps - 1) / kBwdWarps);
-    return launch(routed_bwd_kernel<VPL>, dim3(grid), dim3(32 * kBwdWarps), smem, st, x, W, V,
+    e = launch(routed_bwd_kernel<VPL>, dim3(grid), dim3(32 * kBwdWarps), smem, st, x, W, V,
                   W_r, W_c, sz.L, (int)sz.N, sz.N_c, sz.K, idx, gate, dy, dx, dW, dV, dW_r, dW_c,
-                  shared_rows, status);
+                  shared_rows, rslots ? rcnt : nullptr, rslots, rslots ? rcap : 0, sz.N_r, status);
+    if (e != cudaSuccess || !rslots) return e;
+    const int nrows = sz.N_r + sz.N_c;
+    return launch(bwd_router_rows_kernel<VPL>, dim3((unsigned)((nrows + kBwdWarps - 1) / kBwdWarps)),
+                  dim3(32 * kBwdWarps), 0, st, x, sz.L, nrows, sz.N_r, (const int *)rcnt,
+                  (const int2 *)rslots, rcap, dW_r, dW_c, status);
 }
 
 }  // namespace
@@ -342,7 +418,8 @@ cudaError_t launch_routed_bwd(const uint16_t *x, const uint16_t *W, const uint16
                               const uint16_t *W_r, const uint16_t *W_c, const Sizes &sz,
                               const int32_t *idx, const float *gate, const float *dy, float *dx,
                               float *dW, float *dV, float *dW_r, float *dW_c, uint32_t *seen,
-                              uint32_t *shared_rows, int *status, cudaStream_t st) {
+                              uint32_t *shared_rows, int *rcnt, int2 *rslots, int rcap,
+                              int *status, cudaStream_t st) {
     if (seen && shared_rows) {
         const unsigned grid = (unsigned)((sz.M + 255) / 256);
         cudaError_t e = launch(bwd_mark_kernel, dim3(grid), dim3(256), 0, st, idx, (int64_t)sz.M,
@@ -354,7 +431,7 @@ cudaError_t launch_routed_bwd(const uint16_t *x, const uint16_t *W, const uint16
     switch (sz.d / 256) {
 #define OMNI_BCASE(n) \
         case n: return launch_bwd_vpl<n>(x, W, V, W_r, W_c, sz, idx, gate, dy, dx, dW, dV, dW_r, \
-                                         dW_c, shared_rows, status, st);
+                                         dW_c, shared_rows, rcnt, rslots, rcap, status, st);
         OMNI_BCASE(1) OMNI_BCASE(2) OMNI_BCASE(3) OMNI_BCASE(4)
         OMNI_BCASE(5) OMNI_BCASE(6) OMNI_BCASE(7) OMNI_BCASE(8)
 #undef OMNI_BCASE

@@ -180,7 +180,11 @@ cudaError_t launch_routed_bwd(const uint16_t *x, const uint16_t *W, const uint16
                               const uint16_t *W_r, const uint16_t *W_c, const Sizes &sz,
                               const int32_t *idx, const float *gate, const float *dy, float *dx,
                               float *dW, float *dV, float *dW_r, float *dW_c, uint32_t *seen,
-                              uint32_t *shared_rows, int *status, cudaStream_t st);
+                              uint32_t *shared_rows, int *rcnt, int2 *rslots, int rcap,
+                              int *status, cudaStream_t st);
+// slots per router row in the backward's lists (a row used by more tokens
+// reduces the extra pairs into dW_r / dW_c directly)
+constexpr int kBwdRowCap = 256;
 
 // ---- shared dense MLP (two tile GEMMs; h is [L, F] bf16 scratch)
 cudaError_t launch_shared_mlp(const uint16_t *x, const uint16_t *W_g, const uint16_t *W_u,

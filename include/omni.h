@@ -271,8 +271,12 @@ int omni_routed_fwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
  * bitmaps over the N experts, the experts that more than one task uses; the
  * dW and dV rows of every other expert then get one plain read-add-write
  * (the fastest path, and bit-reproducible), and only the shared rows go
- * through fp32 reductions, whose last bits vary between runs.  With less,
- * every row is reduced.  All fp32 arrays 16-byte aligned.
+ * through fp32 reductions, whose last bits vary between runs.  The router
+ * rows' dW_r / dW_c then collect their tokens' (token, dS) pairs in lists of
+ * up to 256 per row, summed by a second kernel (one plain read-add-write per
+ * row; a row with more pairs reduces the extra ones directly).  With room
+ * for the bitmaps only, the router rows are reduced; with 256 bytes, every
+ * row is.  All fp32 arrays 16-byte aligned.
  * Limits: d % 256 == 0, d <= OMNI_MAX_D, K <= OMNI_MAX_K.
  */
 int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
@@ -282,9 +286,11 @@ int omni_routed_bwd(const omni_bf16 *x, const omni_bf16 *W, const omni_bf16 *V,
                     float *dx, float *dW, float *dV, float *dW_r, float *dW_c,
                     unsigned flags, void *ws, size_t ws_bytes, omni_stream_t stream);
 
-/* Workspace bytes of omni_routed_bwd with its expert bitmaps: 256 plus two
- * bitmaps of N bits, each rounded up to 256 bytes (0 for invalid sizes).  The
- * pages have no counterpart; it only sizes the backward's scratch. */
+/* Workspace bytes of omni_routed_bwd with its expert bitmaps and router-row
+ * lists: 256, two bitmaps of N bits (each rounded up to 256 bytes), a counter
+ * per router row (N_r + N_c int32, rounded up to 256 bytes) and 256 slots of
+ * 8 bytes per router row (0 for invalid sizes).  The pages have no
+ * counterpart; it only sizes the backward's scratch. */
 size_t omni_routed_bwd_workspace_size(int L, int d, int N_r, int N_c, int K);
 
 /*

@@ -42,7 +42,7 @@ int main(void) {
     EXPECT(omni_schedule_workspace_size(L, K, Nr * Nc, B) > 0);
     EXPECT(omni_expert_workspace_size(L, d, K, Nr * Nc, B) > 0);
     EXPECT(omni_shared_mlp_workspace_size(L, d, 128) == 256 + 2 * (size_t)L * 128);
-    EXPECT(omni_routed_bwd_workspace_size(L, d, Nr, Nc, K) == 256 + 2 * 256);
+    EXPECT(omni_routed_bwd_workspace_size(L, d, Nr, Nc, K) == 256 + 2 * 256 + 256 + 8 * (size_t)(Nr + Nc) * 256);
     EXPECT(omni_routed_bwd_workspace_size(L, d, Nr, Nc, 0) == 0);
 
     /* null input */

@@ -79,10 +79,12 @@ def test_workspace_sizes(lib):
     F = configs.mlp_hidden(h.d)
     assert omni.omni_shared_mlp_workspace_size(h.L, h.d, F) == 256 + 2 * h.L * F
     assert omni.omni_shared_mlp_workspace_size(0, h.d, F) == 0
-    # backward: the status header plus two bitmaps over the N experts
+    # backward: the status header, two bitmaps over the N experts, a counter
+    # and 256 (token, ds) slots per router row
     words = -(-h.N // 32)
+    rows = h.N_r + h.N_c
     assert omni.omni_routed_bwd_workspace_size(h.L, h.d, h.N_r, h.N_c, h.K) == \
-        256 + 2 * (-(-4 * words // 256) * 256)
+        256 + 2 * (-(-4 * words // 256) * 256) + (-(-4 * rows // 256) * 256) + 8 * rows * 256
     assert omni.omni_routed_bwd_workspace_size(h.L, h.d, h.N_r, h.N_c, 0) == 0
 
 
