@@ -607,6 +607,8 @@ def profile_stage(args, cfg):
                  dV=torch.zeros((cfg.N, d), **f32), dW_r=torch.zeros((cfg.N_r, d), **f32),
                  dW_c=torch.zeros((cfg.N_c, d), **f32))
         dy = torch.ones((L, d), **f32)
+        ws = torch.empty(omni.omni_routed_bwd_workspace_size(L, d, cfg.N_r, cfg.N_c, cfg.K),
+                         dtype=torch.uint8, device=dev)
     for _ in range(args.warmup + args.steps):
         if args.profile_stage == "backward":
             omni.omni_routed_bwd(t["x"], t["W"], t["V"], t["W_r"], t["W_c"], L, d, cfg.N_r,
