@@ -23,8 +23,12 @@
 // are scatter-added with 16-byte fp32 reductions, which the L2 runs well
 // below HBM bandwidth.  A first kernel marks the experts used more than once
 // (two bitmaps over the N experts) when the workspace has room for them.
-// The router rows are added once per distinct row / column of the token (its
-// K cells sit in few rows and columns, (a+1)(b+1) <= K).
+// The router rows are touched once per distinct row / column of the token (its
+// K cells sit in few rows and columns, (a+1)(b+1) <= K).  With room in the
+// workspace, the token stores (t, dS) in that row's slot list instead of
+// reducing dS x_t onto it; a second kernel then sums each list and adds it to
+// its dW_r / dW_c row once.  A pair that finds its list full, or every pair
+// when there are no lists, is reduced into the row in fp32.
 #include "omni_common.cuh"
 #include "omni_internal.h"
 
