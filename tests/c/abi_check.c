@@ -63,6 +63,18 @@ int main(void) {
     /* backward: flags must be 0 */
     EXPECT(omni_routed_bwd(fb, fb, fb, fb, fb, L, d, Nr, Nc, K, fi, ff, ff, ff, ff, ff, ff, ff, 1,
                            fake, 256, NULL) == OMNI_ERR_INVALID_ARG);
+    /* backward: every gradient buffer is required */
+    EXPECT(omni_routed_bwd(fb, fb, fb, fb, fb, L, d, Nr, Nc, K, fi, ff, ff, ff, ff, ff, ff, NULL, 0,
+                           fake, 256, NULL) == OMNI_ERR_INVALID_ARG);
+    /* backward: d off its 256 grid */
+    EXPECT(omni_routed_bwd(fb, fb, fb, fb, fb, L, 384, Nr, Nc, K, fi, ff, ff, ff, ff, ff, ff, ff, 0,
+                           fake, 256, NULL) == OMNI_ERR_UNSUPPORTED);
+    /* backward: below the 256-byte minimum workspace, or a misaligned one */
+    EXPECT(omni_routed_bwd(fb, fb, fb, fb, fb, L, d, Nr, Nc, K, fi, ff, ff, ff, ff, ff, ff, ff, 0,
+                           fake, 128, NULL) == OMNI_ERR_WORKSPACE);
+    EXPECT(omni_routed_bwd(fb, fb, fb, fb, fb, L, d, Nr, Nc, K, fi, ff, ff, ff, ff, ff, ff, ff, 0,
+                           (char *)fake + 64, 4096, NULL) == OMNI_ERR_WORKSPACE);
+    EXPECT(omni_routed_bwd_workspace_size(0, d, Nr, Nc, K) == 0);
     /* shared MLP: F off the 64 grid */
     EXPECT(omni_shared_mlp_fwd(fb, fb, fb, fb, L, d, 96, ff, 0, fake, 1u << 20, NULL) ==
            OMNI_ERR_UNSUPPORTED);
